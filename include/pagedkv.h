@@ -1,0 +1,212 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv, the B200 (sm_100a) paged KV-cache decode path.
+ *
+ * Three operations, as the PagedAttention pages state the problem:
+ *
+ *   pkv_paged_kv_write          write each new token's K/V into its cache slot
+ *   pkv_paged_attention_decode  single-query attention over a block-paged cache
+ *   pkv_kv_block_copy           copy-on-write copies of shared blocks
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers marked "device" are CUDA device memory owned by the caller.  The
+ *   library allocates no device memory; the caller passes the decode
+ *   workspace.  Pointers must be 16-byte aligned (cache and q/k/v bases);
+ *   integer arrays need natural alignment.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and return PKV_OK or a negative PKV_ERR_* code.  A negative code
+ *   means nothing was launched.
+ * - `validate` != 0 copies the index arrays (block tables, context lengths,
+ *   slots, copy pairs) to the host, checks every id against the pool and
+ *   returns PKV_ERR_OUT_OF_RANGE / PKV_ERR_BAD_COPY_PAIRS before launching.
+ *   This synchronises the stream; it is meant for tests and debugging.
+ * - Independently of `validate`, the kernels check every index they
+ *   dereference.  An id outside the pool is never read or written: the access
+ *   is skipped (reads yield zeros) and a bit is set in the library's device
+ *   status word, read back with pkv_device_status().
+ * - Cache layout (both caches, every dtype):
+ *       [num_blocks][block_size][num_kv_heads][head_dim], contiguous.
+ *   The pages give only the block's byte count (block_size x num_kv_heads x
+ *   head_dim x dtype bytes, "vLLM — 把操作系统的分页搬进 GPU KV cache",
+ *   实践案例 1); the dimension order is this library's choice.  A physical
+ *   block is one contiguous span of block_size * num_kv_heads * head_dim
+ *   elements.
+ * - Element types: PKV_DTYPE_F32, PKV_DTYPE_BF16, PKV_DTYPE_FP8_E4M3 (OCP E4M3,
+ *   per-tensor scale: a stored code c reads back as value(c) * scale).
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define PKV_DTYPE_F32 0
+#define PKV_DTYPE_BF16 1
+#define PKV_DTYPE_FP8_E4M3 2
+
+/* status codes */
+#define PKV_OK 0
+#define PKV_ERR_NULL_POINTER (-1)       /* a required pointer is NULL */
+#define PKV_ERR_BAD_DTYPE (-2)          /* dtype code or dtype combination not supported */
+#define PKV_ERR_HEAD_DIM (-3)           /* head_dim not in {64, 128} */
+#define PKV_ERR_BLOCK_SIZE (-4)         /* block_size not in {8, 16, 32} */
+#define PKV_ERR_HEAD_GROUPING (-5)      /* num_q_heads % num_kv_heads != 0, or group not in {1,2,4,8} */
+#define PKV_ERR_WORKSPACE (-6)          /* workspace NULL or smaller than pkv_decode_workspace_bytes() */
+#define PKV_ERR_BAD_SHAPE (-7)          /* a negative or zero size where a positive one is needed */
+#define PKV_ERR_OUT_OF_RANGE (-8)       /* validate: a block id, slot or context length outside the pool */
+#define PKV_ERR_BAD_COPY_PAIRS (-9)     /* validate: copy pairs whose result would depend on their order */
+#define PKV_ERR_MISALIGNED (-10)        /* a data pointer is not 16-byte aligned */
+#define PKV_ERR_CUDA (-11)              /* a CUDA runtime call or kernel launch failed */
+#define PKV_ERR_TENSOR_MAP (-12)        /* the TMA descriptor for a cache could not be encoded */
+#define PKV_ERR_PARTITION (-13)         /* partition_tokens not a positive multiple of block_size */
+
+/* bits of the device status word (pkv_device_status) */
+#define PKV_STATUS_BAD_BLOCK_ID 0x1u    /* decode met a block id outside [0, num_blocks) */
+#define PKV_STATUS_BAD_CONTEXT 0x2u     /* decode met context_len < 0 or > max_blocks_per_seq * block_size */
+#define PKV_STATUS_BAD_SLOT 0x4u        /* write met a slot >= num_blocks * block_size */
+#define PKV_STATUS_BAD_COPY_PAIR 0x8u   /* block copy met an id outside [0, num_blocks) */
+#define PKV_STATUS_WAIT_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up */
+
+/*
+ * Human-readable name of a PKV_* status code (static storage).
+ */
+const char* pkv_status_string(int status);
+
+/*
+ * New-token KV write ("reshape_and_cache").
+ *
+ * Source: "vLLM 与 KV Cache", KV Cache：为什么需要缓存 -- each decode step
+ * computes K and V of the new token only and appends them to the cache;
+ * "vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点 -- the cache is a pool
+ * of fixed-size blocks addressed through the sequence's block table.
+ *
+ * k, v            device, [num_tokens][num_kv_heads][head_dim] of in_dtype
+ *                 (F32 or BF16), contiguous.
+ * slot_mapping    device int64 [num_tokens]: the flat slot of each token,
+ *                 block = slot / block_size, row = slot % block_size.  A
+ *                 negative slot is a padding token and is skipped.  Slots
+ *                 must be distinct (two tokens on one slot race); validate
+ *                 rejects a repeated slot with PKV_ERR_OUT_OF_RANGE.
+ * key_cache,      device, [num_blocks][block_size][num_kv_heads][head_dim] of
+ * value_cache     cache_dtype; written in place.
+ * cache_dtype     == in_dtype (the bytes are copied), or FP8_E4M3: the stored
+ *                 code is E4M3(x * r) with r = 1/k_scale (1/v_scale for V)
+ *                 rounded once to fp32 on the host, one fp32 multiply, round
+ *                 to nearest even, saturating to +-448.
+ * k_scale,        fp8 dequantisation scales (ignored for other cache types).
+ * v_scale
+ * Errors: PKV_ERR_NULL_POINTER, _BAD_DTYPE, _BAD_SHAPE, _MISALIGNED,
+ * _OUT_OF_RANGE (validate), _CUDA.  num_tokens == 0 launches nothing.
+ */
+int pkv_paged_kv_write(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
+                       void* key_cache, void* value_cache, int64_t num_blocks, int block_size,
+                       int num_kv_heads, int head_dim, int in_dtype, int cache_dtype, float k_scale,
+                       float v_scale, int validate, void* stream);
+
+/*
+ * Paged single-query decode attention.
+ *
+ * Source: "vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点 -- the kernel
+ * reads the physical block id from the sequence's block_table, computes the
+ * offset ("one more int load and one multiply"), then computes attention as
+ * before; "vLLM KV Cache 实现机制", 1.2 -- logically contiguous, physically
+ * scattered.  For every sequence b and query head hq:
+ *     s_t = scale * <q[b,hq], K_t>  (t < context_lens[b]),
+ *     out[b,hq] = sum_t softmax(s)_t V_t,
+ * K_t / V_t being row t % block_size of physical block
+ * block_tables[b][t / block_size], KV head hq / (num_q_heads / num_kv_heads).
+ *
+ * out             device, [num_seqs][num_q_heads][head_dim] of q_dtype.
+ * q               device, [num_seqs][num_q_heads][head_dim] of q_dtype (F32 or BF16).
+ * key_cache,      device, cache layout above, cache_dtype == q_dtype or FP8_E4M3.
+ * value_cache
+ * block_tables    device int32 [num_seqs][max_blocks_per_seq].
+ * context_lens    device int32 [num_seqs]: tokens to attend, including the
+ *                 one written by this step's pkv_paged_kv_write.  0 gives a
+ *                 zero output row.
+ * scale           softmax scale (usually 1/sqrt(head_dim)).
+ * k_scale,        fp8 dequantisation scales (ignored for other cache types).
+ * v_scale
+ * partition_tokens  0 = automatic; otherwise the split-context partition
+ *                 length in tokens (a positive multiple of block_size).  Each
+ *                 (sequence, kv head, partition) is one CTA; sequences with
+ *                 more than one partition are merged by a second kernel.
+ * workspace       device scratch of at least pkv_decode_workspace_bytes(...)
+ *                 bytes (same arguments); not read before it is written.
+ *                 Layout, with P = pkv_decode_max_partitions(...):
+ *                 float ml[num_seqs][num_q_heads][P][2]  (max logit, exp-sum)
+ *                 then float o[num_seqs][num_q_heads][P][head_dim] (normalised
+ *                 partial outputs), starting at a 256-byte aligned offset.
+ * Supported: head_dim in {64, 128}, block_size in {8, 16, 32}, query heads
+ * per KV head in {1, 2, 4, 8}.
+ * Errors: PKV_ERR_NULL_POINTER, _BAD_DTYPE, _HEAD_DIM, _BLOCK_SIZE,
+ * _HEAD_GROUPING, _WORKSPACE, _BAD_SHAPE, _MISALIGNED, _PARTITION,
+ * _OUT_OF_RANGE (validate), _TENSOR_MAP, _CUDA.  num_seqs == 0 launches nothing.
+ */
+int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                               float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                               void* workspace, size_t workspace_bytes, int validate, void* stream);
+
+/*
+ * Partition length (tokens) the decode call uses for these arguments:
+ * partition_tokens if it is non-zero, else the automatic choice, which
+ * depends on the shape and on the current device's SM count.  Returns a
+ * negative PKV_ERR_* code for unsupported arguments.
+ */
+int pkv_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                                int partition_tokens);
+
+/* Partitions per sequence the workspace must hold (max over sequences). */
+int pkv_decode_max_partitions(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                              int partition_tokens);
+
+/* Workspace bytes pkv_paged_attention_decode needs for these arguments
+ * (0 when no sequence can need more than one partition). */
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int max_blocks_per_seq, int partition_tokens);
+
+/*
+ * Copy-on-write block copy.
+ *
+ * Source: "vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点 (引用计数 +
+ * copy-on-write), 实践案例 2 and 踩过的坑 -- blocks shared by n sequences
+ * carry ref_count n; a sequence about to write into a shared block first
+ * gets a private copy (n-1 copies on the first parallel-sampling step).
+ *
+ * src_dst_pairs   device int64 [num_pairs][2] of (src, dst) physical block ids.
+ *                 Every pair copies block src onto block dst in BOTH caches,
+ *                 byte for byte.  The destinations must be distinct and no
+ *                 destination may also be a source (so the result does not
+ *                 depend on order); validate checks this.
+ * key_cache,      device pools of num_blocks blocks of block_bytes bytes each.
+ * value_cache
+ * block_bytes     bytes of one block of one cache: block_size * num_kv_heads
+ *                 * head_dim * dtype size; a multiple of 16.
+ * Errors: PKV_ERR_NULL_POINTER, _BAD_SHAPE, _MISALIGNED, _OUT_OF_RANGE /
+ * _BAD_COPY_PAIRS (validate), _CUDA.  num_pairs == 0 launches nothing.
+ */
+int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key_cache, void* value_cache,
+                      int64_t num_blocks, int64_t block_bytes, int validate, void* stream);
+
+/*
+ * Reads the current device's status word (PKV_STATUS_* bits) into *status,
+ * after synchronising `stream`; clears it if `clear` != 0.
+ */
+int pkv_device_status(unsigned* status, int clear, void* stream);
+
+/* Number of kernel launches this library issued on this process (all devices). */
+uint64_t pkv_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

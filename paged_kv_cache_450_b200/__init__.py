@@ -1,1 +1,191 @@
-"""B200-native paged KV-cache decode path (placeholder; the binding follows)."""
+"""paged_kv_cache_450_b200 -- B200 (sm_100a) paged KV-cache decode path.
+
+Python binding of libpagedkv (C ABI in include/pagedkv.h).  Each function
+only checks and marshals torch tensors (pointers, sizes, the current CUDA
+stream) and calls the library; every step of the path runs in the CUDA
+kernels.  Torch provides device memory and streams.  There is no CPU path:
+CPU tensors are rejected, and a missing library raises.
+
+    paged_kv_write(k, v, slot_mapping, key_cache, value_cache, ...)
+    paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens, scale, ...)
+    kv_block_copy(src_dst_pairs, key_cache, value_cache, ...)
+
+Cache layout: key_cache / value_cache are [num_blocks, block_size,
+num_kv_heads, head_dim] (float32, bfloat16 or float8_e4m3fn).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+DTYPE_F32, DTYPE_BF16, DTYPE_FP8_E4M3 = 0, 1, 2
+_DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float8_e4m3fn: DTYPE_FP8_E4M3}
+
+STATUS_BAD_BLOCK_ID = 0x1
+STATUS_BAD_CONTEXT = 0x2
+STATUS_BAD_SLOT = 0x4
+STATUS_BAD_COPY_PAIR = 0x8
+STATUS_WAIT_TIMEOUT = 0x10
+
+__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_workspace_bytes",
+           "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
+           "library_path"]
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = _lib.load().pkv_status_string(code).decode()
+        super().__init__(f"{where}: {msg} (status {code})")
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise PagedKVError(code, where)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _cuda(*ts: torch.Tensor):
+    dev = ts[0].device
+    for t in ts:
+        if t.device.type != "cuda":
+            raise ValueError("libpagedkv works on CUDA tensors only (there is no CPU path)")
+        if t.device != dev:
+            raise ValueError("all tensors must be on one device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    return dev
+
+
+def _stream(dev, stream):
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def library_path() -> str:
+    return _lib.path()
+
+
+def paged_kv_write(k, v, slot_mapping, key_cache, value_cache, *, k_scale: float = 1.0, v_scale: float = 1.0,
+                   validate: bool = False, stream=None) -> None:
+    """Write each token's K/V into its slot (block = slot // bs, row = slot % bs).
+
+    k, v: [T, Hkv, d] float32 / bfloat16; slot_mapping: int64 [T] (negative =
+    skip); caches [NB, bs, Hkv, d] of k's dtype or float8_e4m3fn (then the
+    stored code is E4M3(x * (1/k_scale)), saturating)."""
+    dev = _cuda(k, v, slot_mapping, key_cache, value_cache)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    NB, bs, Hkv, d = key_cache.shape
+    if value_cache.shape != key_cache.shape or k.shape != v.shape or k.shape[1:] != (Hkv, d) \
+            or slot_mapping.shape != (k.shape[0],):
+        raise ValueError("shape mismatch")
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        _check(lib.pkv_paged_kv_write(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), k.shape[0],
+                                      key_cache.data_ptr(), value_cache.data_ptr(), NB, bs, Hkv, d, _dtype(k),
+                                      _dtype(key_cache), float(k_scale), float(v_scale), int(validate),
+                                      _stream(dev, stream)), "paged_kv_write")
+
+
+def decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens=0) -> int:
+    r = _lib.load().pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
+                                                partition_tokens)
+    _check(min(r, 0), "decode_partition_tokens")
+    return r
+
+
+def decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens=0) -> int:
+    r = _lib.load().pkv_decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
+                                              partition_tokens)
+    _check(min(r, 0), "decode_max_partitions")
+    return r
+
+
+def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           partition_tokens=0) -> int:
+    return int(_lib.load().pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                      max_blocks_per_seq, partition_tokens))
+
+
+def paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens, scale: float,
+                           block_size: int | None = None, num_kv_heads: int | None = None, *,
+                           k_scale: float = 1.0, v_scale: float = 1.0, out=None, workspace=None,
+                           partition_tokens: int = 0, validate: bool = False, stream=None):
+    """Single-query decode attention over the block-paged cache.
+
+    q: [B, Hq, d]; caches: [NB, bs, Hkv, d]; block_tables int32 [B, MB];
+    context_lens int32 [B].  Returns out [B, Hq, d] in q's dtype.  The
+    split-context workspace is allocated with torch when not given."""
+    dev = _cuda(q, key_cache, value_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, Hq, d = q.shape
+    NB, bs, Hkv, d2 = key_cache.shape
+    if block_size is not None and block_size != bs:
+        raise ValueError(f"block_size {block_size} does not match the cache's {bs}")
+    if num_kv_heads is not None and num_kv_heads != Hkv:
+        raise ValueError(f"num_kv_heads {num_kv_heads} does not match the cache's {Hkv}")
+    if d2 != d or value_cache.shape != key_cache.shape or block_tables.dim() != 2 or \
+            block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("shape mismatch")
+    MB = block_tables.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out)
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out must match q")
+    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, MB, partition_tokens) if B else 0
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        _check(lib.pkv_paged_attention_decode(
+            out.data_ptr(), q.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), block_tables.data_ptr(),
+            context_lens.data_ptr(), B, Hq, Hkv, d, bs, MB, NB, float(scale), float(k_scale), float(v_scale),
+            _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr, ws_bytes, int(validate),
+            _stream(dev, stream)), "paged_attention_decode")
+    return out
+
+
+def kv_block_copy(src_dst_pairs, key_cache, value_cache, *, validate: bool = False, stream=None) -> None:
+    """Copy block src onto block dst in both caches for every (src, dst) row of
+    src_dst_pairs (int64 [n, 2]); destinations distinct and never a source."""
+    dev = _cuda(src_dst_pairs, key_cache, value_cache)
+    if src_dst_pairs.dtype != torch.int64 or src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be int64 [n, 2]")
+    if value_cache.shape != key_cache.shape or value_cache.dtype != key_cache.dtype:
+        raise ValueError("caches must match")
+    NB = key_cache.shape[0]
+    block_bytes = key_cache[0].numel() * key_cache.element_size()
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        _check(lib.pkv_kv_block_copy(src_dst_pairs.data_ptr(), src_dst_pairs.shape[0], key_cache.data_ptr(),
+                                     value_cache.data_ptr(), NB, block_bytes, int(validate),
+                                     _stream(dev, stream)), "kv_block_copy")
+
+
+def device_status(clear: bool = True, device=None, stream=None) -> int:
+    """The library's device status word (STATUS_* bits) on `device`."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    v = ctypes.c_uint(0)
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_device_status(ctypes.byref(v), int(clear), _stream(dev, stream)), "device_status")
+    return int(v.value)
+
+
+def launch_count() -> int:
+    """Kernel launches the library has issued in this process."""
+    return int(_lib.load().pkv_launch_count())

@@ -1,0 +1,358 @@
+// abi.cu -- the C ABI of libpagedkv (declared in include/pagedkv.h):
+// argument checks, optional host-side validation of index arrays, TMA
+// descriptor encoding for the caches, the split-context partition choice and
+// the kernel dispatch.
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "launch.h"
+
+namespace pkv {
+
+// The device status word (PKV_STATUS_* bits), one per device that loads the module.
+__device__ unsigned g_status_word;
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_mu;
+
+static unsigned* status_word() {
+  static unsigned* ptr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return ptr[dev];
+}
+
+static int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map of one cache [NB][BS][Hkv][D] seen as a 4-D tensor
+// (D, Hkv, BS, NB) innermost first; the box is one (block, kv head) tile.
+static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blocks, int block_size, int num_kv_heads,
+                             int head_dim, int dtype) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  CUtensorMapDataType dt;
+  int es;
+  switch (dtype) {
+    case PKV_DTYPE_F32: dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; es = 4; break;
+    case PKV_DTYPE_BF16: dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; es = 2; break;
+    case PKV_DTYPE_FP8_E4M3: dt = CU_TENSOR_MAP_DATA_TYPE_UINT8; es = 1; break;
+    default: return false;
+  }
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
+                              static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * es;
+  const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1, static_cast<cuuint32_t>(block_size), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <typename T>
+static bool copy_to_host(std::vector<T>& dst, const T* src, size_t n, cudaStream_t st) {
+  dst.resize(n);
+  if (n == 0) return true;
+  if (cudaMemcpyAsync(dst.data(), src, n * sizeof(T), cudaMemcpyDeviceToHost, st) != cudaSuccess) return false;
+  return cudaStreamSynchronize(st) == cudaSuccess;
+}
+
+constexpr int kMaxPartitionTokens = 16384;
+
+// Automatic split-context partition length: 512 tokens, halved (down to 128)
+// while the grid would hold fewer than ~4 waves of 3 CTAs per SM; a single
+// partition when the longest possible context fits in one.
+static int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq) {
+  const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
+  const int64_t target = 4LL * 3 * sm_count();
+  int pt = 512;
+  while (pt > 128 && pairs * cdiv64(max_ctx, pt) < target) pt /= 2;
+  if (pt < block_size) pt = block_size;
+  if (max_ctx <= pt) pt = static_cast<int>(cdiv64(max_ctx, block_size) * block_size);
+  if (pt < block_size) pt = block_size;
+  return pt;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case PKV_ERR_BAD_DTYPE: return "unsupported dtype or dtype combination";
+    case PKV_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
+    case PKV_ERR_BLOCK_SIZE: return "block_size must be 8, 16 or 32";
+    case PKV_ERR_HEAD_GROUPING: return "num_q_heads / num_kv_heads must be 1, 2, 4 or 8";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_BAD_SHAPE: return "bad size argument";
+    case PKV_ERR_OUT_OF_RANGE: return "an index (block id, slot, context length) is outside the pool";
+    case PKV_ERR_BAD_COPY_PAIRS: return "copy pairs repeat a destination or use a destination as a source";
+    case PKV_ERR_MISALIGNED: return "a data pointer is not 16-byte aligned";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_TENSOR_MAP: return "TMA descriptor encoding failed";
+    case PKV_ERR_PARTITION: return "partition_tokens must be a positive multiple of block_size (at most 16384)";
+    default: return "unknown status";
+  }
+}
+
+uint64_t pkv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int pkv_device_status(unsigned* status, int clear, void* stream) {
+  if (!status) return PKV_ERR_NULL_POINTER;
+  unsigned* w = status_word();
+  if (!w) return PKV_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(status, w, sizeof(unsigned), cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ERR_CUDA;
+  if (clear && cudaMemsetAsync(w, 0, sizeof(unsigned), st) != cudaSuccess) return PKV_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_paged_kv_write(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
+                       void* key_cache, void* value_cache, int64_t num_blocks, int block_size, int num_kv_heads,
+                       int head_dim, int in_dtype, int cache_dtype, float k_scale, float v_scale, int validate,
+                       void* stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !key_cache || !value_cache) return PKV_ERR_NULL_POINTER;
+  if (in_dtype != PKV_DTYPE_F32 && in_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (cache_dtype != in_dtype && cache_dtype != PKV_DTYPE_FP8_E4M3) return PKV_ERR_BAD_DTYPE;
+  if (head_dim % 16 != 0) return PKV_ERR_HEAD_DIM;
+  if (num_tokens > 0x7fffffffLL) return PKV_ERR_BAD_SHAPE;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
+  if (cache_dtype == PKV_DTYPE_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_BAD_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    std::vector<int64_t> h;
+    if (!copy_to_host(h, slot_mapping, static_cast<size_t>(num_tokens), st)) return PKV_ERR_CUDA;
+    const int64_t slots = num_blocks * block_size;
+    std::vector<int64_t> seen;
+    for (int64_t s : h) {
+      if (s >= slots) return PKV_ERR_OUT_OF_RANGE;
+      if (s >= 0) seen.push_back(s);
+    }
+    std::sort(seen.begin(), seen.end());
+    for (size_t i = 1; i < seen.size(); ++i)
+      if (seen[i] == seen[i - 1]) return PKV_ERR_OUT_OF_RANGE;
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  KvWriteArgs a;
+  a.k = k;
+  a.v = v;
+  a.slot_mapping = slot_mapping;
+  a.num_tokens = num_tokens;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.num_blocks = num_blocks;
+  a.block_size = block_size;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.in_dtype = in_dtype;
+  a.cache_dtype = cache_dtype;
+  a.k_inv = 1.0f / k_scale;  // rounded once to fp32 on the host
+  a.v_inv = 1.0f / v_scale;
+  a.status = status;
+  return launch_kv_write(a, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                                int partition_tokens) {
+  if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_BAD_SHAPE;
+  if (partition_tokens != 0) {
+    if (partition_tokens < 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
+      return PKV_ERR_PARTITION;
+    return partition_tokens;
+  }
+  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq);
+}
+
+int pkv_decode_max_partitions(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                              int partition_tokens) {
+  const int pt = pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
+                                             partition_tokens);
+  if (pt < 0) return pt;
+  return static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
+}
+
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int partition_tokens) {
+  const int P = pkv_decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens);
+  if (P <= 1 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * P;
+  return align256(rows * 2 * sizeof(float)) + rows * head_dim * sizeof(float);
+}
+
+int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                               float v_scale, int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                               size_t workspace_bytes, int validate, void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_ERR_NULL_POINTER;
+  if (q_dtype != PKV_DTYPE_F32 && q_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (cache_dtype != q_dtype && cache_dtype != PKV_DTYPE_FP8_E4M3) return PKV_ERR_BAD_DTYPE;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_HEAD_DIM;
+  if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_HEAD_GROUPING;
+  if (num_blocks > 0x7fffffffLL || num_seqs > 65535) return PKV_ERR_BAD_SHAPE;
+  if (static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffffLL) return PKV_ERR_BAD_SHAPE;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
+  if (cache_dtype == PKV_DTYPE_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_BAD_SHAPE;
+  const int pt = pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
+                                             partition_tokens);
+  if (pt < 0) return pt;
+  const int P = static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
+  if (P > 65535) return PKV_ERR_PARTITION;
+  const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                 max_blocks_per_seq, partition_tokens);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    std::vector<int32_t> lens, tables;
+    if (!copy_to_host(lens, context_lens, static_cast<size_t>(num_seqs), st)) return PKV_ERR_CUDA;
+    if (!copy_to_host(tables, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st))
+      return PKV_ERR_CUDA;
+    for (int b = 0; b < num_seqs; ++b) {
+      const int64_t ctx = lens[b];
+      if (ctx < 0 || ctx > static_cast<int64_t>(max_blocks_per_seq) * block_size) return PKV_ERR_OUT_OF_RANGE;
+      for (int64_t j = 0; j < cdiv64(ctx, block_size); ++j) {
+        const int64_t id = tables[static_cast<size_t>(b) * max_blocks_per_seq + j];
+        if (id < 0 || id >= num_blocks) return PKV_ERR_OUT_OF_RANGE;
+      }
+    }
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype) ||
+      !encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype))
+    return PKV_ERR_TENSOR_MAP;
+
+  DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_ml = nullptr;
+  p.ws_o = nullptr;
+  if (need > 0) {
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * P;
+    p.ws_ml = static_cast<float*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * 2 * sizeof(float)));
+  }
+  p.status = status;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = static_cast<int>(num_blocks);
+  p.block_size = block_size;
+  p.partition_blocks = pt / block_size;
+  p.max_partitions = P;
+  const bool fp8 = cache_dtype == PKV_DTYPE_FP8_E4M3;
+  p.q_scale = scale * kLog2e * (fp8 ? k_scale : 1.0f);
+  p.out_scale = fp8 ? v_scale : 1.0f;
+  const bool reduce = P > 1;
+
+  cudaError_t e;
+  if (q_dtype == PKV_DTYPE_F32 && cache_dtype == PKV_DTYPE_F32)
+    e = launch_decode_f32_f32(kmap, vmap, p, head_dim, group, num_kv_heads, reduce, st);
+  else if (q_dtype == PKV_DTYPE_BF16 && cache_dtype == PKV_DTYPE_BF16)
+    e = launch_decode_bf16_bf16(kmap, vmap, p, head_dim, group, num_kv_heads, reduce, st);
+  else if (q_dtype == PKV_DTYPE_F32)
+    e = launch_decode_f32_fp8(kmap, vmap, p, head_dim, group, num_kv_heads, reduce, st);
+  else
+    e = launch_decode_bf16_fp8(kmap, vmap, p, head_dim, group, num_kv_heads, reduce, st);
+  return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key_cache, void* value_cache,
+                      int64_t num_blocks, int64_t block_bytes, int validate, void* stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_bytes <= 0 || block_bytes % 16 != 0) return PKV_ERR_BAD_SHAPE;
+  if (num_pairs == 0) return PKV_OK;
+  if (!src_dst_pairs || !key_cache || !value_cache) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    std::vector<int64_t> h;
+    if (!copy_to_host(h, src_dst_pairs, static_cast<size_t>(num_pairs) * 2, st)) return PKV_ERR_CUDA;
+    std::vector<int64_t> dsts, srcs;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+      const int64_t s = h[2 * i], d = h[2 * i + 1];
+      if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PKV_ERR_OUT_OF_RANGE;
+      srcs.push_back(s);
+      dsts.push_back(d);
+    }
+    std::sort(dsts.begin(), dsts.end());
+    std::sort(srcs.begin(), srcs.end());
+    for (size_t i = 1; i < dsts.size(); ++i)
+      if (dsts[i] == dsts[i - 1]) return PKV_ERR_BAD_COPY_PAIRS;
+    for (int64_t d : dsts)
+      if (std::binary_search(srcs.begin(), srcs.end(), d)) return PKV_ERR_BAD_COPY_PAIRS;
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  return launch_block_copy(src_dst_pairs, num_pairs, key_cache, value_cache, num_blocks, block_bytes, status, st) ==
+                 cudaSuccess
+             ? PKV_OK
+             : PKV_ERR_CUDA;
+}
+
+}  // extern "C"

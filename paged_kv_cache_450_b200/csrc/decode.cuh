@@ -1,0 +1,364 @@
+// decode.cuh -- paged single-query decode attention: partition pass + reduce.
+//
+// What is computed ("vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点):
+// for each sequence b and query head hq, attention of q[b,hq] over the
+// sequence's K/V, where logical token t lives in row t % block_size of the
+// physical block block_tables[b][t / block_size] -- one table load and one
+// multiply per block, then the usual q.K^T, softmax and weighted sum of V.
+//
+// Grid: one CTA per (kv head, partition, sequence).  A partition is a run of
+// partition_blocks logical blocks; with grouped-query attention the CTA serves
+// all G query heads that share the KV head, so every K/V byte is read from
+// HBM once per step.
+//
+// Inside a CTA four warps each own a private TMA pipeline of NS stages.  A
+// stage holds one (block, kv head) tile of K and of V: block_size rows of
+// head_dim contiguous elements at the pool's row stride, fetched by one 4-D
+// tensor-map load each (box {head_dim, 1, block_size, 1}).  Warp w takes the
+// partition's blocks w, w+4, w+8, ... and keeps its own online-softmax state
+// (running max m, running sum l, unnormalised accumulator); the four states
+// are merged in shared memory at the end.
+//
+// QK^T: a token row is split over TG = head_dim / 8 lanes, 8 elements each,
+// so one warp instruction covers 32 / TG tokens; the partial dots are summed
+// with xor shuffles.  Softmax works in base 2: q is pre-multiplied by
+// scale * log2(e) (and by the fp8 K scale), so e^{s-m} = 2^{s2-m2}.
+// P.V: lane l owns head_dim / 32 consecutive output elements and walks the
+// block's valid rows; the probabilities come from a per-warp shared array.
+//
+// A sequence with a single partition gets its normalised output written
+// directly.  Otherwise every partition writes (m, l, o = acc / l) to the
+// workspace and paged_decode_reduce_kernel merges them:
+//     out = sum_p l_p e^{m_p - M} o_p / sum_p l_p e^{m_p - M}.
+#pragma once
+
+#include "common.cuh"
+
+namespace pkv {
+
+struct DecodeParams {
+  void* out;                    // [B][Hq][D] of TQ
+  const void* q;                // [B][Hq][D] of TQ
+  const int32_t* block_tables;  // [B][max_blocks_per_seq]
+  const int32_t* context_lens;  // [B]
+  float* ws_ml;                 // [B][Hq][P][2]: max logit (natural units), exp-sum
+  float* ws_o;                  // [B][Hq][P][D]: normalised partial outputs
+  unsigned* status;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int block_size;
+  int partition_blocks;
+  int max_partitions;
+  float q_scale;    // scale * log2(e) * (fp8 ? k_scale : 1)
+  float out_scale;  // fp8 ? v_scale : 1
+};
+
+template <typename TQ, typename TC, int D, int BS, int G>
+struct DecodeTraits {
+  static constexpr int NW = 4;                      // warps per CTA, one pipeline each
+  static constexpr int ES = Elem<TC>::kBytes;
+  static constexpr int ROW_BYTES = D * ES;          // one token of one kv head
+  static constexpr int TILE_BYTES = BS * ROW_BYTES; // one (block, kv head) of K or V
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int NS = (16384 / STAGE_BYTES) >= 1 ? 16384 / STAGE_BYTES : 1;  // ~16 KB per warp
+  static constexpr int TG = D / 8;                  // lanes per token row in q.K
+  static constexpr int TPI = 32 / TG;               // tokens per warp instruction
+  static constexpr int NIT = BS / TPI;              // q.K steps per block
+  static constexpr int PVV = D / 32;                // output elements per lane
+  static constexpr int STAGE_AREA = NW * NS * STAGE_BYTES;
+  static constexpr int COMBINE_BYTES = NW * G * (D + 2) * 4;
+  static constexpr int DATA_BYTES = STAGE_AREA > COMBINE_BYTES ? STAGE_AREA : COMBINE_BYTES;
+  static constexpr int BAR_BYTES = NW * NS * 8;
+  static constexpr int Q_BYTES = G * D * 4;
+  static constexpr int P_BYTES = NW * G * BS * 4;
+  static_assert(32 % TG == 0 && BS % TPI == 0, "tile mapping");
+  static_assert(TILE_BYTES % 16 == 0, "TMA boxes are multiples of 16 bytes");
+
+  // Dynamic shared memory for a partition of pb blocks (1 KB alignment slack).
+  static constexpr size_t smem_bytes(int pb) {
+    return 1024 + DATA_BYTES + BAR_BYTES + Q_BYTES + P_BYTES + static_cast<size_t>(pb) * 4;
+  }
+};
+
+// Reads N consecutive elements of T at p (N * sizeof(T) in {2, 4, 8, 16, 32}).
+template <typename T, int N>
+__device__ __forceinline__ void load_elems(const uint8_t* p, float* out) {
+  constexpr int bytes = N * Elem<T>::kBytes;
+  if constexpr (bytes == 2) {
+    const uint32_t w = *reinterpret_cast<const uint16_t*>(p);
+    float tmp[4];
+    Elem<T>::unpack_word(w, tmp);
+    out[0] = tmp[0];
+    out[1] = tmp[1];
+  } else if constexpr (bytes == 4) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    unpack<T, N>(&w, out);
+  } else if constexpr (bytes == 8) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    const uint32_t ws[2] = {w.x, w.y};
+    unpack<T, N>(ws, out);
+  } else if constexpr (bytes == 16) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    unpack<T, N>(ws, out);
+  } else {
+    static_assert(bytes == 32, "unsupported slice");
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint4 c = *reinterpret_cast<const uint4*>(p + 16);
+    const uint32_t ws[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    unpack<T, N>(ws, out);
+  }
+}
+
+template <typename TQ, typename TC, int D, int BS, int G>
+__global__ void __launch_bounds__(128)
+    paged_decode_partition_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                                  const DecodeParams p) {
+  using T = DecodeTraits<TQ, TC, D, BS, G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::DATA_BYTES);
+  float* q_s = reinterpret_cast<float*>(data + T::DATA_BYTES + T::BAR_BYTES);
+  float* p_s = q_s + G * D;
+  int* ids = reinterpret_cast<int*>(p_s + T::NW * G * BS);
+
+  const int hk = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hq = p.num_q_heads;
+  const int max_ctx = p.max_blocks_per_seq * BS;
+  int ctx = p.context_lens[b];
+  if (ctx < 0 || ctx > max_ctx) {
+    if (threadIdx.x == 0 && hk == 0 && part == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
+    ctx = ctx < 0 ? 0 : max_ctx;
+  }
+  const int nblk = (ctx + BS - 1) / BS;
+  const int pb = p.partition_blocks;
+  const int nparts = (nblk + pb - 1) / pb;
+  TQ* out = static_cast<TQ*>(p.out);
+  const int64_t out_row0 = static_cast<int64_t>(b) * Hq + hk * G;  // first query head of the group
+  if (nparts == 0) {  // empty context: a zero output row
+    if (part == 0)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[out_row0 * D + i] = Elem<TQ>::from_float(0.f);
+    return;
+  }
+  if (part >= nparts) return;
+  const int blk0 = part * pb;
+  const int nb = min(pb, nblk - blk0);
+
+  // Block-table lookups for the whole partition, with the pool-range guard.
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + blk0 + i];
+    if (id < 0 || id >= p.num_blocks) {
+      set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
+      id = -1;
+    }
+    ids[i] = id;
+  }
+  // q of the G heads, pre-scaled into the base-2 logit domain.
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x)
+    q_s[i] = Elem<TQ>::to_float(static_cast<const TQ*>(p.q)[out_row0 * D + i]) * p.q_scale;
+  const uint32_t bar0 = smem_u32(bars) + warp * T::NS * 8;
+  if (lane == 0) {
+    for (int s = 0; s < T::NS; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int n_w = nb > warp ? (nb - warp + T::NW - 1) / T::NW : 0;  // blocks of this warp
+  const uint32_t stage0 = smem_u32(data) + warp * T::NS * T::STAGE_BYTES;
+  const uint64_t policy = l2_policy_evict_first();
+  auto issue = [&](int i) {
+    const int s = i % T::NS;
+    const uint32_t bar = bar0 + 8 * s;
+    const int id = ids[warp + i * T::NW];
+    if (id >= 0) {
+      mbar_arrive_expect_tx(bar, T::STAGE_BYTES);
+      const uint32_t dst = stage0 + s * T::STAGE_BYTES;
+      tma_load_4d(dst, &kmap, bar, 0, hk, 0, id, policy);
+      tma_load_4d(dst + T::TILE_BYTES, &vmap, bar, 0, hk, 0, id, policy);
+    } else {
+      mbar_arrive(bar);  // bad id: nothing to fetch, the block is skipped
+    }
+  };
+  if (lane == 0) {
+    const int pre = n_w < T::NS ? n_w : T::NS;
+    for (int i = 0; i < pre; ++i) issue(i);
+  }
+
+  const int gi = lane / T::TG;  // token slot within a q.K instruction
+  const int gl = lane % T::TG;  // 8-element slice of the row
+  float m[G], l[G], acc[G][T::PVV];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < T::PVV; ++e) acc[g][e] = 0.f;
+  }
+  float* pw = p_s + warp * G * BS;
+
+  int waited = 0;  // stages whose load this warp has waited for
+  bool ok = true;
+  for (int i = 0; i < n_w; ++i) {
+    const int s = i % T::NS;
+    if (!mbar_wait_bounded(bar0 + 8 * s, (i / T::NS) & 1, p.status)) {
+      ok = false;
+      break;
+    }
+    waited = i + 1;
+    const int j = warp + i * T::NW;
+    if (ids[j] >= 0) {
+      const uint8_t* kt = data + warp * T::NS * T::STAGE_BYTES + s * T::STAGE_BYTES;
+      const uint8_t* vt = kt + T::TILE_BYTES;
+      const int valid = min(BS, ctx - (blk0 + j) * BS);  // >= 1
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float qf[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qf[e] = q_s[g * D + gl * 8 + e];
+        float sc[T::NIT];
+#pragma unroll
+        for (int it = 0; it < T::NIT; ++it) {
+          const int t = it * T::TPI + gi;
+          float kf[8];
+          load_elems<TC, 8>(kt + t * T::ROW_BYTES + gl * 8 * T::ES, kf);
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a = fmaf(qf[e], kf[e], a);
+#pragma unroll
+          for (int off = T::TG / 2; off > 0; off >>= 1) a += __shfl_xor_sync(kFullMask, a, off);
+          sc[it] = t < valid ? a : -INFINITY;
+        }
+        float bm = -INFINITY;
+#pragma unroll
+        for (int it = 0; it < T::NIT; ++it) bm = fmaxf(bm, sc[it]);
+#pragma unroll
+        for (int off = T::TG; off < 32; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, off));
+        const float mn = fmaxf(m[g], bm);
+        const float alpha = fast_exp2(m[g] - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int it = 0; it < T::NIT; ++it) {
+          sc[it] = fast_exp2(sc[it] - mn);
+          ps += sc[it];
+        }
+#pragma unroll
+        for (int off = T::TG; off < 32; off <<= 1) ps += __shfl_xor_sync(kFullMask, ps, off);
+        l[g] = l[g] * alpha + ps;
+#pragma unroll
+        for (int e = 0; e < T::PVV; ++e) acc[g][e] *= alpha;
+        m[g] = mn;
+        if (gl == 0) {
+#pragma unroll
+          for (int it = 0; it < T::NIT; ++it) pw[g * BS + it * T::TPI + gi] = sc[it];
+        }
+      }
+      __syncwarp();
+      for (int t = 0; t < valid; ++t) {  // rows past the context are never read
+        float vf[T::PVV];
+        load_elems<TC, T::PVV>(vt + t * T::ROW_BYTES + lane * T::PVV * T::ES, vf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pt = pw[g * BS + t];
+#pragma unroll
+          for (int e = 0; e < T::PVV; ++e) acc[g][e] = fmaf(pt, vf[e], acc[g][e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && i + T::NS < n_w) {
+      fence_proxy_async_smem();
+      issue(i + T::NS);
+    }
+  }
+  if (!ok) {
+    // Drain: wait (bounded) for every load still in flight before the
+    // shared memory is released.
+    const int issued = min(n_w, waited + T::NS);
+    for (int i = waited; i < issued; ++i) mbar_wait_bounded(bar0 + 8 * (i % T::NS), (i / T::NS) & 1, p.status);
+  }
+  __syncthreads();  // every warp is done with the stage area
+
+  float* c_m = reinterpret_cast<float*>(data);
+  float* c_l = c_m + T::NW * G;
+  float* c_acc = c_l + T::NW * G;
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      c_m[warp * G + g] = m[g];
+      c_l[warp * G + g] = l[g];
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < T::PVV; ++e) c_acc[(warp * G + g) * D + lane * T::PVV + e] = acc[g][e];
+  __syncthreads();
+
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, e = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < T::NW; ++w) M = fmaxf(M, c_m[w * G + g]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < T::NW; ++w) {
+      const float f = fast_exp2(c_m[w * G + g] - M);  // warps without blocks: 2^-inf = 0
+      L = fmaf(c_l[w * G + g], f, L);
+      O = fmaf(c_acc[(w * G + g) * D + e], f, O);
+    }
+    const float o = L > 0.f ? O / L * p.out_scale : 0.f;
+    if (nparts == 1) {
+      out[(out_row0 + g) * D + e] = Elem<TQ>::from_float(o);
+    } else {
+      const int64_t slot = (out_row0 + g) * p.max_partitions + part;
+      p.ws_o[slot * D + e] = o;
+      if (e == 0) {
+        p.ws_ml[slot * 2] = M * kLn2;
+        p.ws_ml[slot * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// Merge of split-context partials, one warp per (sequence, query head).
+template <typename TQ, int D>
+__global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeParams p) {
+  constexpr int PVV = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  if (row >= static_cast<int64_t>(p.num_seqs) * p.num_q_heads) return;
+  const int b = static_cast<int>(row / p.num_q_heads);
+  const int BS = p.block_size;
+  const int max_ctx = p.max_blocks_per_seq * BS;
+  int ctx = p.context_lens[b];
+  ctx = ctx < 0 ? 0 : (ctx > max_ctx ? max_ctx : ctx);
+  const int nparts = ((ctx + BS - 1) / BS + p.partition_blocks - 1) / p.partition_blocks;
+  if (nparts <= 1) return;  // written by the partition pass
+  const float* ml = p.ws_ml + row * p.max_partitions * 2;
+  const float* o = p.ws_o + row * p.max_partitions * D;
+  float M = -INFINITY;
+  for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[2 * i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+  float acc[PVV];
+#pragma unroll
+  for (int e = 0; e < PVV; ++e) acc[e] = 0.f;
+  float W = 0.f;
+  for (int i = 0; i < nparts; ++i) {
+    const float li = ml[2 * i + 1];
+    const float w = li > 0.f ? li * fast_exp2((ml[2 * i] - M) * kLog2e) : 0.f;
+    W += w;
+    const float* oi = o + static_cast<int64_t>(i) * D + lane * PVV;
+#pragma unroll
+    for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w, oi[e], acc[e]);
+  }
+  TQ* out = static_cast<TQ*>(p.out) + row * D + lane * PVV;
+#pragma unroll
+  for (int e = 0; e < PVV; ++e) out[e] = Elem<TQ>::from_float(W > 0.f ? acc[e] / W : 0.f);
+}
+
+}  // namespace pkv

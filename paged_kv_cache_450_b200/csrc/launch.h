@@ -1,0 +1,50 @@
+// launch.h -- internal interface between the C ABI (abi.cu) and the kernel
+// translation units.  Host code only; no CUDA kernels are declared here.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+struct DecodeParams;
+
+// Counts one kernel launch (pkv_launch_count()).
+void count_launch();
+
+struct KvWriteArgs {
+  const void* k;
+  const void* v;
+  const int64_t* slot_mapping;
+  int64_t num_tokens;
+  void* key_cache;
+  void* value_cache;
+  int64_t num_blocks;
+  int block_size;
+  int num_kv_heads;
+  int head_dim;
+  int in_dtype;
+  int cache_dtype;
+  float k_inv;  // 1/k_scale rounded to fp32 (fp8 caches)
+  float v_inv;
+  unsigned* status;
+};
+
+cudaError_t launch_kv_write(const KvWriteArgs& a, cudaStream_t st);
+cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, void* kc, void* vc, int64_t num_blocks,
+                              int64_t block_bytes, unsigned* status, cudaStream_t st);
+
+// Decode launchers, one per (q dtype, cache dtype); each dispatches on
+// head_dim, block_size and the query-head group.  `reduce` adds the merge
+// kernel (sequences with more than one partition).
+#define PKV_DECLARE_DECODE(NAME)                                                                            \
+  cudaError_t NAME(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p, int head_dim, \
+                   int group, int num_kv_heads, bool reduce, cudaStream_t st);
+PKV_DECLARE_DECODE(launch_decode_f32_f32)
+PKV_DECLARE_DECODE(launch_decode_bf16_bf16)
+PKV_DECLARE_DECODE(launch_decode_f32_fp8)
+PKV_DECLARE_DECODE(launch_decode_bf16_fp8)
+#undef PKV_DECLARE_DECODE
+
+}  // namespace pkv

@@ -1,0 +1,105 @@
+"""The C ABI library loads without a GPU, exports every function that
+include/pagedkv.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_450_b200 as pk
+from paged_kv_cache_450_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in pagedkv.h but not exported"
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures and header disagree"
+
+
+def test_header_constants_match_binding():
+    text = open(HEADER).read()
+    consts = dict(re.findall(r"#define (PKV_\w+) \(?(-?0x[0-9a-fA-F]+|-?\d+)u?\)?", text))
+    assert int(consts["PKV_DTYPE_F32"]) == pk.DTYPE_F32
+    assert int(consts["PKV_DTYPE_BF16"]) == pk.DTYPE_BF16
+    assert int(consts["PKV_DTYPE_FP8_E4M3"]) == pk.DTYPE_FP8_E4M3
+    assert int(consts["PKV_STATUS_BAD_BLOCK_ID"], 16) == pk.STATUS_BAD_BLOCK_ID
+    assert int(consts["PKV_STATUS_WAIT_TIMEOUT"], 16) == pk.STATUS_WAIT_TIMEOUT
+
+
+def test_status_strings():
+    lib = _lib.load()
+    assert lib.pkv_status_string(0) == b"ok"
+    for code in range(-13, 0):
+        assert lib.pkv_status_string(code) != b"unknown status"
+
+
+P = None
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), -3), (dict(block_size=24), -4), (dict(num_q_heads=12, num_kv_heads=8), -5),
+    (dict(num_q_heads=48, num_kv_heads=4), -5), (dict(q_dtype=2), -2), (dict(cache_dtype=7), -2),
+    (dict(q_dtype=0, cache_dtype=1), -2), (dict(num_seqs=-1), -7), (dict(partition_tokens=24), -13),
+    (dict(out=0), -1), (dict(out=0x1008), -10), (dict(workspace=0), -6),
+])
+def test_decode_argument_errors(kw, code):
+    lib = _lib.load()
+    a = dict(out=0x1000, q=0x2000, key_cache=0x3000, value_cache=0x4000, block_tables=0x5000, context_lens=0x6000,
+             num_seqs=4, num_q_heads=8, num_kv_heads=8, head_dim=128, block_size=16, max_blocks_per_seq=256,
+             num_blocks=100, scale=0.1, k_scale=1.0, v_scale=1.0, q_dtype=1, cache_dtype=1, partition_tokens=0,
+             workspace=0x7000, workspace_bytes=1 << 30, validate=0, stream=None)
+    a.update(kw)
+    args = [a[k] for k in ("out", "q", "key_cache", "value_cache", "block_tables", "context_lens", "num_seqs",
+                           "num_q_heads", "num_kv_heads", "head_dim", "block_size", "max_blocks_per_seq",
+                           "num_blocks", "scale", "k_scale", "v_scale", "q_dtype", "cache_dtype",
+                           "partition_tokens", "workspace", "workspace_bytes", "validate", "stream")]
+    if a["workspace"] == 0:
+        args[20] = 0
+    assert lib.pkv_paged_attention_decode(*args) == code
+
+
+def test_write_and_copy_argument_errors():
+    lib = _lib.load()
+    assert lib.pkv_paged_kv_write(0x10, 0x20, 0x30, 0, 0x40, 0x50, 10, 16, 4, 128, 1, 1, 1.0, 1.0, 0, None) == 0
+    assert lib.pkv_paged_kv_write(None, 0x20, 0x30, 5, 0x40, 0x50, 10, 16, 4, 128, 1, 1, 1.0, 1.0, 0, None) == -1
+    assert lib.pkv_paged_kv_write(0x10, 0x20, 0x30, 5, 0x40, 0x50, 10, 16, 4, 128, 1, 0, 1.0, 1.0, 0, None) == -2
+    assert lib.pkv_paged_kv_write(0x10, 0x20, 0x30, 5, 0x40, 0x50, 10, 16, 4, 128, 1, 2, 0.0, 1.0, 0, None) == -7
+    assert lib.pkv_paged_kv_write(0x18, 0x20, 0x30, 5, 0x40, 0x50, 10, 16, 4, 128, 1, 1, 1.0, 1.0, 0, None) == -10
+    assert lib.pkv_kv_block_copy(0x10, 0, 0x20, 0x30, 10, 4096, 0, None) == 0
+    assert lib.pkv_kv_block_copy(0x10, 3, 0x20, 0x30, 10, 4004, 0, None) == -7
+    assert lib.pkv_kv_block_copy(None, 3, 0x20, 0x30, 10, 4096, 0, None) == -1
+
+
+def test_partition_choice_and_workspace_size():
+    # single partition when the longest context fits: no workspace
+    assert pk.decode_partition_tokens(4, 4, 16, 7) == 112
+    assert pk.decode_workspace_bytes(4, 4, 4, 64, 16, 7) == 0
+    # 64 sequences x 32 heads x 2048 tokens: 512-token partitions
+    assert pk.decode_partition_tokens(64, 32, 16, 128) == 512
+    P = pk.decode_max_partitions(64, 32, 16, 128)
+    assert P == 4
+    rows = 64 * 32 * P
+    assert pk.decode_workspace_bytes(64, 32, 32, 128, 16, 128) == ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
+    # explicit partition lengths
+    assert pk.decode_partition_tokens(1, 1, 16, 100, 48) == 48
+    with pytest.raises(pk.PagedKVError):
+        pk.decode_partition_tokens(1, 1, 16, 100, 40)
+
+
+def test_ops_refuse_cpu_tensors():
+    import torch
+    x = torch.zeros(2, 2, 128)
+    with pytest.raises(ValueError):
+        pk.paged_attention_decode(x, torch.zeros(4, 16, 2, 128), torch.zeros(4, 16, 2, 128),
+                                  torch.zeros(2, 1, dtype=torch.int32), torch.zeros(2, dtype=torch.int32), 0.1)

@@ -1,0 +1,195 @@
+"""GPU parity: libpagedkv (through its C ABI) against the CPU oracle.
+
+Bit-exact for the cache write and the block copy; decode attention within
+the stated tolerances (bf16 2e-3 + 1e-2|ref|, fp8 KV 3e-2 relative, fp32 1e-4).
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_450_b200 as pk
+from paged_kv_cache_450_b200 import workloads as W
+from step_helpers import (assert_cache_equal, assert_close, gpu_step, ocode, oracle_step, sample_rows, to_np,
+                          tol_for)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+FP8 = torch.float8_e4m3fn
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_step(w, partition_tokens=0, rows=None, what=""):
+    kc, vc, out = gpu_step(w, partition_tokens=partition_tokens)
+    rk, rv, ref = oracle_step(w, rows=rows)
+    assert_cache_equal(kc, rk, f"{what} key_cache")
+    assert_cache_equal(vc, rv, f"{what} value_cache")
+    got = f64(out)
+    if rows is not None:
+        got = got.reshape(-1, w.spec.head_dim)[rows]
+    assert_close(got, ref, *tol_for(w), what=what)
+    return out
+
+
+def test_tiny_config_full_parity():
+    w = W.make_decode_workload(W.TINY, seed=0, device=DEV)
+    check_step(w, what="tiny")
+
+
+DTYPES = [(torch.float32, torch.float32), (torch.bfloat16, torch.bfloat16), (torch.bfloat16, FP8),
+          (torch.float32, FP8)]
+
+
+@pytest.mark.parametrize("dtypes,d,bs,g", list(itertools.product(DTYPES, [64, 128], [8, 16, 32], [1, 2, 4, 8])),
+                         ids=lambda x: str(x).replace("torch.", "").replace(" ", ""))
+def test_every_kernel_instance_small(dtypes, d, bs, g):
+    qd, cd = dtypes
+    spec = W.DecodeSpec("small", 5, 2 * g, 2, d, bs, qd, cd, ("list", (1, 700, bs, 3 * bs + 1, 257)),
+                        ("slack", 1.3))
+    w = W.make_decode_workload(spec, seed=d + bs + g, device=DEV)
+    # partition lengths: automatic, one block, three blocks
+    for pt in (0, bs, 3 * bs):
+        check_step(w, partition_tokens=pt, what=f"pt={pt}")
+
+
+@pytest.mark.parametrize("cd", [torch.bfloat16, FP8])
+def test_partition_partials_match_oracle(cd):
+    spec = W.DecodeSpec("partials", 3, 8, 2, 128, 16, torch.bfloat16, cd, ("list", (300, 17, 64)), ("slack", 1.2),
+                        new_tokens=False)
+    w = W.make_decode_workload(spec, seed=11, device=DEV)
+    pt = 64
+    B, Hq, d = 3, 8, 128
+    MB = w.block_tables.shape[1]
+    P = pk.decode_max_partitions(B, 2, 16, MB, pt)
+    nbytes = pk.decode_workspace_bytes(B, Hq, 2, d, 16, MB, pt)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
+    gpu_step(w, partition_tokens=pt, workspace=ws)
+    rows = B * Hq * P
+    ml_bytes = ((rows * 2 * 4 + 255) // 256) * 256
+    ml = ws[: rows * 8].view(torch.float32).view(B, Hq, P, 2).cpu().numpy().astype(np.float64)
+    o = ws[ml_bytes: ml_bytes + rows * d * 4].view(torch.float32).view(B, Hq, P, d).cpu().numpy()
+    m_ref, l_ref, o_ref = oracle.decode_partials(
+        to_np(w.q), to_np(w.key_cache), to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
+        scale=w.scale, partition_tokens=pt, max_partitions=P, q_dtype=oracle.BF16, cache_dtype=ocode(cd),
+        k_scale=w.k_scale, v_scale=w.v_scale)
+    atol, rtol = tol_for(w)
+    for b, c in enumerate(w.ctx_list):
+        n = -(-c // pt)
+        if n <= 1:
+            continue  # single-partition rows are written straight to the output
+        assert_close(ml[b, :, :n, 0], m_ref[b, :, :n], 1e-4, 1e-4, what="partition max")
+        assert_close(ml[b, :, :n, 1], l_ref[b, :, :n], 1e-4, 1e-3, what="partition exp-sum")
+        assert_close(o[b, :, :n], o_ref[b, :, :n], atol, rtol, what="partition output")
+
+
+def test_edge_contexts_zero_one_and_max():
+    bs = 16
+    spec = W.DecodeSpec("edges", 6, 4, 4, 128, bs, torch.bfloat16, torch.bfloat16,
+                        ("list", (0, 1, 16, 17, 64, 0)), ("slack", 1.5), new_tokens=False)
+    w = W.make_decode_workload(spec, seed=2, device=DEV)
+    out = check_step(w, what="edges")
+    assert torch.count_nonzero(out[0]) == 0 and torch.count_nonzero(out[5]) == 0
+    # ctx = max_blocks_per_seq * bs exactly, several partitions
+    spec = W.DecodeSpec("max", 2, 4, 4, 128, bs, torch.bfloat16, torch.bfloat16, ("fixed", 1024))
+    w = W.make_decode_workload(spec, seed=3, device=DEV)
+    assert w.block_tables.shape[1] * bs == 1024
+    for pt in (0, 16, 512, 1024):
+        check_step(w, partition_tokens=pt, what=f"max ctx pt={pt}")
+
+
+def test_empty_batch_is_a_no_op():
+    q = torch.zeros((0, 4, 128), dtype=torch.bfloat16, device=DEV)
+    kc = torch.zeros((4, 16, 4, 128), dtype=torch.bfloat16, device=DEV)
+    out = pk.paged_attention_decode(q, kc, kc, torch.zeros((0, 1), dtype=torch.int32, device=DEV),
+                                    torch.zeros((0,), dtype=torch.int32, device=DEV), 0.1)
+    assert out.shape == (0, 4, 128)
+
+
+def test_placement_invariance_on_gpu():
+    """Moving every physical block to another id (tables rewritten to match)
+    leaves the output bit-identical."""
+    spec = W.LLAMA7B.with_(num_seqs=6, num_q_heads=4, num_kv_heads=4, ctx=("uniform", 100, 900), new_tokens=False)
+    w = W.make_decode_workload(spec, seed=4, device=DEV)
+    out1 = pk.paged_attention_decode(w.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, w.scale)
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(9)).to(DEV)
+    kc, vc = torch.empty_like(w.key_cache), torch.empty_like(w.value_cache)
+    kc[perm] = w.key_cache
+    vc[perm] = w.value_cache
+    tables = perm[w.block_tables.long()].to(torch.int32)
+    out2 = pk.paged_attention_decode(w.q, kc, vc, tables, w.context_lens, w.scale)
+    assert torch.equal(out1, out2)
+
+
+FULL = [W.LLAMA7B, W.LLAMA13B, W.SPECS["llama13b_decode_b256_bf16_bs32"], W.PARALLEL_SAMPLING, W.GQA_LONG,
+        W.GQA_BATCH]
+
+
+@pytest.mark.parametrize("spec", FULL, ids=lambda s: s.name)
+def test_full_size_configs_sampled(spec):
+    w = W.make_decode_workload(spec, seed=0, device=DEV)
+    rows = sample_rows(w, 512)
+    check_step(w, rows=rows, what=spec.name)
+
+
+def test_parallel_sampling_cow_semantics_prompt_1020():
+    """Prompt of 1020 tokens: the last prompt block is partial, so each
+    candidate's first new token goes into its own copy of it (ref_count 4
+    shared prompt, 3 copy-on-write copies, one candidate keeps the block)."""
+    spec = W.PARALLEL_SAMPLING.with_(num_seqs=16, sampling=(4, 4, 1020, 1, 1))
+    w = W.make_decode_workload(spec, seed=5, device=DEV)
+    assert len(w.copy_pairs) == 4 * 3
+    check_step(w, what="cow-1020")
+
+
+def test_validate_rejects_bad_inputs_without_launching():
+    w = W.make_decode_workload(W.TINY, seed=0, device=DEV)
+    before = pk.launch_count()
+    bad = w.block_tables.clone()
+    bad[0, 0] = w.num_blocks
+    with pytest.raises(pk.PagedKVError) as e:
+        pk.paged_attention_decode(w.q, w.key_cache, w.value_cache, bad, w.context_lens, w.scale, validate=True)
+    assert e.value.code == -8
+    pairs = torch.tensor([[1, 5], [2, 5]], dtype=torch.int64, device=DEV)
+    with pytest.raises(pk.PagedKVError) as e:
+        pk.kv_block_copy(pairs, w.key_cache.clone(), w.value_cache.clone(), validate=True)
+    assert e.value.code == -9
+    slots = w.slot_mapping.clone()
+    slots[0] = w.num_blocks * 16
+    with pytest.raises(pk.PagedKVError) as e:
+        pk.paged_kv_write(w.new_k, w.new_v, slots, w.key_cache.clone(), w.value_cache.clone(), validate=True)
+    assert e.value.code == -8
+    assert pk.launch_count() == before
+
+
+def test_kernel_guards_set_status_instead_of_reading_outside_the_pool():
+    """Ids past the pool reach the kernels only without validate; the kernels
+    skip them (no access outside the pool) and report through the status word."""
+    w = W.make_decode_workload(W.TINY, seed=0, device=DEV)
+    pk.device_status(clear=True)
+    bad = w.block_tables.clone()
+    bad[1, 0] = w.num_blocks + 5
+    out = pk.paged_attention_decode(w.q, w.key_cache, w.value_cache, bad, w.context_lens, w.scale)
+    torch.cuda.synchronize()
+    assert pk.device_status(clear=True) & pk.STATUS_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+    slots = w.slot_mapping.clone()
+    slots[2] = w.num_blocks * 16 + 3
+    kc, vc = w.key_cache.clone(), w.value_cache.clone()
+    pk.paged_kv_write(w.new_k, w.new_v, slots, kc, vc)
+    assert pk.device_status(clear=True) & pk.STATUS_BAD_SLOT
+    pairs = torch.tensor([[0, w.num_blocks]], dtype=torch.int64, device=DEV)
+    pk.kv_block_copy(pairs, kc, vc)
+    assert pk.device_status(clear=True) & pk.STATUS_BAD_COPY_PAIR
+    assert pk.device_status(clear=True) == 0
+
+
+def test_launch_count_counts_kernels():
+    w = W.make_decode_workload(W.LLAMA7B.with_(num_seqs=4, num_q_heads=4, num_kv_heads=4), seed=1, device=DEV)
+    n0 = pk.launch_count()
+    gpu_step(w, partition_tokens=128, validate=False)
+    assert pk.launch_count() - n0 == 3   # write, partition pass, reduce
