@@ -30,7 +30,7 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_workspace_bytes",
+__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_step", "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
            "library_path"]
 
@@ -189,3 +189,40 @@ def device_status(clear: bool = True, device=None, stream=None) -> int:
 def launch_count() -> int:
     """Kernel launches the library has issued in this process."""
     return int(_lib.load().pkv_launch_count())
+
+
+def decode_step(q, new_k, new_v, slot_mapping, block_tables, context_lens, key_cache, value_cache, scale: float, *,
+                copy_pairs=None, k_scale: float = 1.0, v_scale: float = 1.0, out=None, workspace=None,
+                partition_tokens: int = 0, stream=None):
+    """One decode step of one attention layer over a device-resident paged cache.
+
+    Order: copy-on-write block copies (``copy_pairs``, if any), the new-token
+    write (``new_k``/``new_v`` at ``slot_mapping``), then decode attention over
+    ``context_lens`` (which include the new token).  The per-step inputs may be
+    host tensors (pinned memory makes the copies asynchronous): they are copied
+    to the cache's device on the stream, and the result is copied back into
+    ``out`` (a host tensor, allocated pinned when not given).  With device
+    inputs everything stays on the device.  Returns the output."""
+    dev = key_cache.device
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    host = q.device.type == "cpu"
+
+    def to_dev(t):
+        return t.to(dev, non_blocking=True) if t is not None and t.device != dev else t
+
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        qd, kd, vd, sd, td, ld, pd = (to_dev(t) for t in (q, new_k, new_v, slot_mapping, block_tables,
+                                                           context_lens, copy_pairs))
+        if pd is not None and pd.numel():
+            kv_block_copy(pd, key_cache, value_cache, stream=st)
+        if kd is not None:
+            paged_kv_write(kd, vd, sd, key_cache, value_cache, k_scale=k_scale, v_scale=v_scale, stream=st)
+        res = paged_attention_decode(qd, key_cache, value_cache, td, ld, scale, k_scale=k_scale, v_scale=v_scale,
+                                     out=None if host else out, workspace=workspace,
+                                     partition_tokens=partition_tokens, stream=st)
+        if host:
+            if out is None:
+                out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+            out.copy_(res, non_blocking=True)
+            return out
+        return res
