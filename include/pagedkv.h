@@ -156,6 +156,47 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
                                void* workspace, size_t workspace_bytes, int validate, void* stream);
 
 /*
+ * Paged decode attention that allocates nothing and takes no workspace.
+ *
+ * The PagedAttention pages have no counterpart of this call; it is a
+ * convenience of this library.  pkv_paged_attention_decode needs device
+ * scratch for its split-context partials and takes it from the caller.
+ * Some callers have none to give at that point: an engine that reserved
+ * nearly all device memory for its KV block pool up front and keeps no
+ * allocator for temporaries, code that must not call cudaMalloc inside a
+ * decode step (cudaMalloc can synchronise the whole device), or a binding
+ * from an environment without a device allocator.  This call computes
+ * exactly what pkv_paged_attention_decode computes, with the same arguments
+ * (minus workspace, workspace_bytes and validate) and the same kernels, but
+ * keeps the partials in a fixed array of PKV_DECODE_STATIC_SCRATCH_BYTES
+ * compiled into the library.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * - Every GPU on which the library's device code is loaded holds that array
+ *   until the process exits.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make
+ *   that first call before any stream capture.
+ * - All calls on a device share the array, and it keeps the partials of the
+ *   last call.  Nothing in it has to start at zero.  Calls that may run at
+ *   the same time on the GPU (other streams, or host threads without an
+ *   order between them) race on the array and give wrong results: order
+ *   them on one stream.
+ * - A call whose partials need more than PKV_DECODE_STATIC_SCRATCH_BYTES
+ *   (pkv_decode_workspace_bytes() with the same arguments) returns
+ *   PKV_ERR_WORKSPACE and launches nothing; a larger partition_tokens lowers
+ *   the need.
+ * Other errors: as pkv_paged_attention_decode.
+ */
+#define PKV_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+int pkv_paged_attention_decode_static(void* out, const void* q, const void* key_cache, const void* value_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                      int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                                      float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                                      void* stream);
+
+/*
  * Partition length (tokens) the decode call uses for these arguments:
  * partition_tokens if it is non-zero, else the automatic choice, which
  * depends on the shape and on the current device's SM count.  Returns a
