@@ -66,8 +66,10 @@ static EncodeTiledFn encode_tiled() {
 
 // Tensor map of one cache [NB][BS][Hkv][D] seen as a 4-D tensor
 // (D, Hkv, BS, NB) innermost first; the box is one (block, kv head) tile.
+// With `swizzle128` the tile lands in shared memory with the 128-byte swizzle
+// (16-byte chunk q of row t at chunk q ^ (t % 8)); the row must be 128 bytes.
 static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blocks, int block_size, int num_kv_heads,
-                             int head_dim, int dtype) {
+                             int head_dim, int dtype, bool swizzle128) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   CUtensorMapDataType dt;
@@ -84,8 +86,9 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blo
   const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
   const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1, static_cast<cuuint32_t>(block_size), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (swizzle128 && row != 128) return false;
   return fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -281,8 +284,9 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
   unsigned* status = status_word();
   if (!status) return PKV_ERR_CUDA;
   CUtensorMap kmap, vmap;
-  if (!encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype) ||
-      !encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype))
+  const bool mma = decode_uses_mma(cache_dtype, head_dim, group, block_size);
+  if (!encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, mma) ||
+      !encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, mma))
     return PKV_ERR_TENSOR_MAP;
 
   DecodeParams p;

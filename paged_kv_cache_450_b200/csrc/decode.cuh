@@ -113,6 +113,40 @@ __device__ __forceinline__ void load_elems(const uint8_t* p, float* out) {
   }
 }
 
+// Merges the NW warp states of one CTA (left in shared memory as c_m[w][g],
+// c_l[w][g] in base-2 units and c_acc[w][g][D] unnormalised) and writes the
+// normalised output row (single partition) or the partition's (m, l, o)
+// partial.  Called by all threads of the CTA after a __syncthreads().
+template <typename TQ, int D, int G, int NW>
+__device__ __forceinline__ void finish_partition(const float* c_m, const float* c_l, const float* c_acc,
+                                                 const DecodeParams& p, int64_t out_row0, int part, int nparts) {
+  TQ* out = static_cast<TQ*>(p.out);
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, e = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, c_m[w * G + g]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = fast_exp2(c_m[w * G + g] - M);  // warps without blocks: 2^-inf = 0
+      L = fmaf(c_l[w * G + g], f, L);
+      O = fmaf(c_acc[(w * G + g) * D + e], f, O);
+    }
+    const float o = L > 0.f ? O / L * p.out_scale : 0.f;
+    if (nparts == 1) {
+      out[(out_row0 + g) * D + e] = Elem<TQ>::from_float(o);
+    } else {
+      const int64_t slot = (out_row0 + g) * p.max_partitions + part;
+      p.ws_o[slot * D + e] = o;
+      if (e == 0) {
+        p.ws_ml[slot * 2] = M * kLn2;
+        p.ws_ml[slot * 2 + 1] = L;
+      }
+    }
+  }
+}
+
 template <typename TQ, typename TC, int D, int BS, int G>
 __global__ void __launch_bounds__(128)
     paged_decode_partition_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -297,31 +331,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int e = 0; e < T::PVV; ++e) c_acc[(warp * G + g) * D + lane * T::PVV + e] = acc[g][e];
   __syncthreads();
-
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int g = idx / D, e = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < T::NW; ++w) M = fmaxf(M, c_m[w * G + g]);
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < T::NW; ++w) {
-      const float f = fast_exp2(c_m[w * G + g] - M);  // warps without blocks: 2^-inf = 0
-      L = fmaf(c_l[w * G + g], f, L);
-      O = fmaf(c_acc[(w * G + g) * D + e], f, O);
-    }
-    const float o = L > 0.f ? O / L * p.out_scale : 0.f;
-    if (nparts == 1) {
-      out[(out_row0 + g) * D + e] = Elem<TQ>::from_float(o);
-    } else {
-      const int64_t slot = (out_row0 + g) * p.max_partitions + part;
-      p.ws_o[slot * D + e] = o;
-      if (e == 0) {
-        p.ws_ml[slot * 2] = M * kLn2;
-        p.ws_ml[slot * 2 + 1] = L;
-      }
-    }
-  }
+  finish_partition<TQ, D, G, T::NW>(c_m, c_l, c_acc, p, out_row0, part, nparts);
 }
 
 // Merge of split-context partials, one warp per (sequence, query head).

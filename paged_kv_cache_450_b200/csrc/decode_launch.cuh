@@ -3,7 +3,10 @@
 // instances compile in parallel.
 #pragma once
 
+#include <type_traits>
+
 #include "decode.cuh"
+#include "decode_mma.cuh"
 #include "launch.h"
 
 namespace pkv {
@@ -13,6 +16,20 @@ static cudaError_t launch_partition(const CUtensorMap& kmap, const CUtensorMap& 
                                    int num_kv_heads, cudaStream_t st) {
   using T = DecodeTraits<TQ, TC, D, BS, G>;
   auto kern = paged_decode_partition_kernel<TQ, TC, D, BS, G>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(num_kv_heads, p.max_partitions, p.num_seqs);
+  kern<<<grid, T::NW * 32, smem, st>>>(kmap, vmap, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename TQ, int BS>
+static cudaError_t launch_mma(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p, int num_kv_heads,
+                              cudaStream_t st) {
+  using T = MmaTraits<BS>;
+  auto kern = paged_decode_gqa8_fp8_mma_kernel<TQ, BS>;
   const size_t smem = T::smem_bytes(p.partition_blocks);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -33,6 +50,9 @@ static cudaError_t launch_reduce(const DecodeParams& p, cudaStream_t st) {
 template <typename TQ, typename TC, int D, int BS>
 static cudaError_t dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p, int group,
                                   int num_kv_heads, cudaStream_t st) {
+  if constexpr (std::is_same_v<TC, __nv_fp8_e4m3> && D == 128 && (BS == 16 || BS == 32)) {
+    if (group == 8) return launch_mma<TQ, BS>(kmap, vmap, p, num_kv_heads, st);
+  }
   switch (group) {
     case 1: return launch_partition<TQ, TC, D, BS, 1>(kmap, vmap, p, num_kv_heads, st);
     case 2: return launch_partition<TQ, TC, D, BS, 2>(kmap, vmap, p, num_kv_heads, st);

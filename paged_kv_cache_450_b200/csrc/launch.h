@@ -35,6 +35,14 @@ cudaError_t launch_kv_write(const KvWriteArgs& a, cudaStream_t st);
 cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, void* kc, void* vc, int64_t num_blocks,
                               int64_t block_bytes, unsigned* status, cudaStream_t st);
 
+// The tensor-core decode kernel serves fp8 caches with head_dim 128, 8 query
+// heads per KV head and 16- or 32-token blocks; its cache tensor maps use the
+// 128-byte swizzle.  Everything else runs on the CUDA-core kernel.
+inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_size) {
+  return cache_dtype == 2 /* PKV_DTYPE_FP8_E4M3 */ && head_dim == 128 && group == 8 &&
+         (block_size == 16 || block_size == 32);
+}
+
 // Decode launchers, one per (q dtype, cache dtype); each dispatches on
 // head_dim, block_size and the query-head group.  `reduce` adds the merge
 // kernel (sequences with more than one partition).
