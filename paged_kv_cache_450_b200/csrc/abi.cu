@@ -107,12 +107,12 @@ static bool copy_to_host(std::vector<T>& dst, const T* src, size_t n, cudaStream
 constexpr int kMaxPartitionTokens = 16384;
 
 // Automatic split-context partition length: 512 tokens, halved (down to 128)
-// while the grid would hold fewer than ~4 waves of 3 CTAs per SM; a single
+// while the grid would hold fewer than ~4 waves of 6 CTAs per SM; a single
 // partition when the longest possible context fits in one.
 static int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq) {
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
-  const int64_t target = 4LL * 3 * sm_count();
+  const int64_t target = 4LL * 6 * sm_count();
   int pt = 512;
   while (pt > 128 && pairs * cdiv64(max_ctx, pt) < target) pt /= 2;
   if (pt < block_size) pt = block_size;

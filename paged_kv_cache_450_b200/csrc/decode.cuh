@@ -56,14 +56,19 @@ struct DecodeParams {
   float out_scale;  // fp8 ? v_scale : 1
 };
 
-template <typename TQ, typename TC, int D, int BS, int G>
+// NW warps per CTA, each with a private pipeline of NS stages (0: about 8 KB of
+// stages per warp).  Small CTAs win: with ~34 KB of shared memory per CTA six
+// CTAs share an SM, and while one warp computes the others' loads stay in
+// flight (a sweep on B200 put 4 warps x 1 stage of 8 KB at 96% of the
+// streaming rate of the same TMA pattern without compute).
+template <typename TQ, typename TC, int D, int BS, int G, int NW_ = 4, int NS_ = 0>
 struct DecodeTraits {
-  static constexpr int NW = 4;                      // warps per CTA, one pipeline each
+  static constexpr int NW = NW_;
   static constexpr int ES = Elem<TC>::kBytes;
   static constexpr int ROW_BYTES = D * ES;          // one token of one kv head
   static constexpr int TILE_BYTES = BS * ROW_BYTES; // one (block, kv head) of K or V
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NS = (16384 / STAGE_BYTES) >= 1 ? 16384 / STAGE_BYTES : 1;  // ~16 KB per warp
+  static constexpr int NS = NS_ > 0 ? NS_ : ((8192 / STAGE_BYTES) >= 1 ? 8192 / STAGE_BYTES : 1);
   static constexpr int TG = D / 8;                  // lanes per token row in q.K
   static constexpr int TPI = 32 / TG;               // tokens per warp instruction
   static constexpr int NIT = BS / TPI;              // q.K steps per block
@@ -147,11 +152,11 @@ __device__ __forceinline__ void finish_partition(const float* c_m, const float* 
   }
 }
 
-template <typename TQ, typename TC, int D, int BS, int G>
-__global__ void __launch_bounds__(128)
+template <typename TQ, typename TC, int D, int BS, int G, int NW = 4, int NS = 0, int MINB = 1>
+__global__ void __launch_bounds__(NW * 32, MINB)
     paged_decode_partition_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                                   const DecodeParams p) {
-  using T = DecodeTraits<TQ, TC, D, BS, G>;
+  using T = DecodeTraits<TQ, TC, D, BS, G, NW, NS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::DATA_BYTES);

@@ -35,13 +35,18 @@
 
 namespace pkv {
 
-template <int BS>
+// NW warps per CTA, each with a private pipeline of NS stages.  Defaults from
+// a sweep on B200: 2 warps x 12 KB of stages and at least 8 resident CTAs per
+// SM (registers capped at 128) -- many small CTAs hide the dependent
+// convert -> MMA -> softmax chains better than deep per-warp pipelines.
+template <int BS, int NW_ = 2, int NS_ = 0>
 struct MmaTraits {
-  static constexpr int D = 128, G = 8, NW = 4;
+  static constexpr int D = 128, G = 8, NW = NW_;
   static constexpr int ROW_BYTES = 128;  // one fp8 token row of one kv head
   static constexpr int TILE_BYTES = BS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NS = 16384 / STAGE_BYTES;  // ~16 KB of stages per warp
+  static constexpr int NS = NS_ > 0 ? NS_ : (12288 / STAGE_BYTES >= 1 ? 12288 / STAGE_BYTES : 1);
+  static constexpr int MIN_BLOCKS = 8;
   static constexpr int NT = BS / 16;              // 16-token MMA tiles per block
   static constexpr int STAGE_AREA = NW * NS * STAGE_BYTES;
   static constexpr int COMBINE_BYTES = NW * G * (D + 2) * 4;
@@ -54,9 +59,13 @@ struct MmaTraits {
   }
 };
 
-__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t codes) {  // low 16 bits: two codes
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xffffu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four E4M3 codes (bytes 0..3 of w) -> two fp16x2 words: lo = bytes {0,1}, hi = bytes {2,3}
+// (the lower byte of each pair lands in the lower half).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t f16x2_pack(float lo, float hi) {
@@ -83,11 +92,11 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 // Byte offset of logical 16-byte chunk q of row t in a 128-byte-swizzled tile.
 __device__ __forceinline__ int swz(int t, int q) { return t * 128 + ((q ^ (t & 7)) << 4); }
 
-template <typename TQ, int BS>
-__global__ void __launch_bounds__(128)
+template <typename TQ, int BS, int NW = 2, int NS = 0, int MINB = 8>
+__global__ void __launch_bounds__(NW * 32, MINB)
     paged_decode_gqa8_fp8_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                                      const DecodeParams p) {
-  using T = MmaTraits<BS>;
+  using T = MmaTraits<BS, NW, NS>;
   constexpr int D = T::D, G = T::G;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -179,8 +188,21 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int k = 0; k < 4; ++k) o[i][k] = 0.f;
 
-  const int rho_r = r ^ ((r & 1) << 2);                 // K rows of this lane: rho_r, rho_r + 8
-  const int vrow0 = 2 * c, vrow1 = (2 * c + 1) ^ 4;     // V rows: vrow0, vrow1, vrow0 + 8, vrow1 + 8
+  // Shared-memory byte offsets (within a 16-token tile) of this lane's loads,
+  // fixed for the whole kernel: K rows rho(r), rho(r)+8 at chunks c, 4+c;
+  // V rows 2c, (2c+1)^4, and +8, at the chunks holding dims 8r.. and 8r+64..
+  const int rho_r = r ^ ((r & 1) << 2);
+  const int vrow[4] = {2 * c, (2 * c + 1) ^ 4, 2 * c + 8, ((2 * c + 1) ^ 4) + 8};
+  int koff[2][2], voff[4][2];
+#pragma unroll
+  for (int i2 = 0; i2 < 2; ++i2) {
+    koff[0][i2] = swz(rho_r, 4 * i2 + c);
+    koff[1][i2] = swz(rho_r + 8, 4 * i2 + c);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) voff[k][h] = swz(vrow[k], (r >> 1) + 4 * h) + 8 * (r & 1);
 
   int waited = 0;
   bool ok = true;
@@ -193,32 +215,42 @@ __global__ void __launch_bounds__(128)
     waited = i + 1;
     const int j = warp + i * T::NW;
     if (ids[j] >= 0) {
-      const uint8_t* kt = data + warp * T::NS * T::STAGE_BYTES + s * T::STAGE_BYTES;
-      const uint8_t* vt = kt + T::TILE_BYTES;
+      const uint8_t* kt0 = data + warp * T::NS * T::STAGE_BYTES + s * T::STAGE_BYTES;
       const int valid = min(BS, ctx - (blk0 + j) * BS);
 #pragma unroll
       for (int t = 0; t < T::NT; ++t) {
         const int t0 = 16 * t;
         if (t0 >= valid) break;
+        const uint8_t* kt = kt0 + t0 * T::ROW_BYTES;  // 16-row tiles start at 2 KB multiples: same swizzle
+        const uint8_t* vt = kt + T::TILE_BYTES;
+        const bool full = t0 + 16 <= valid;            // warp-uniform: no masking needed
         // ---- S = K . Q^T -------------------------------------------------------
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-chunks
 #pragma unroll
         for (int i2 = 0; i2 < 2; ++i2) {
-          const uint4 ka = *reinterpret_cast<const uint4*>(kt + swz(t0 + rho_r, 4 * i2 + c));
-          const uint4 kb = *reinterpret_cast<const uint4*>(kt + swz(t0 + rho_r + 8, 4 * i2 + c));
+          const uint4 ka = *reinterpret_cast<const uint4*>(kt + koff[0][i2]);
+          const uint4 kb = *reinterpret_cast<const uint4*>(kt + koff[1][i2]);
           const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w};
           const uint32_t kbw[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            mma_16816(sacc, f16x2_from_e4m3x2(kaw[q]), f16x2_from_e4m3x2(kbw[q]), f16x2_from_e4m3x2(kaw[q] >> 16),
-                      f16x2_from_e4m3x2(kbw[q] >> 16), qf[4 * i2 + q][0], qf[4 * i2 + q][1]);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_f16x2x2(kaw[q], a0, a2);
+            e4m3x4_to_f16x2x2(kbw[q], a1, a3);
+            mma_16816((q & 1) ? sacc2 : sacc, a0, a1, a2, a3, qf[4 * i2 + q][0], qf[4 * i2 + q][1]);
+          }
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sacc[k] += sacc2[k];
         // ---- online softmax (base 2), heads 2c and 2c+1 --------------------------
-        const bool va = t0 + rho_r < valid, vb = t0 + rho_r + 8 < valid;
-        const float s0 = va ? sacc[0] * qk : -INFINITY;
-        const float s1 = va ? sacc[1] * qk : -INFINITY;
-        const float s2 = vb ? sacc[2] * qk : -INFINITY;
-        const float s3 = vb ? sacc[3] * qk : -INFINITY;
+        float s0 = sacc[0] * qk, s1 = sacc[1] * qk, s2 = sacc[2] * qk, s3 = sacc[3] * qk;
+        if (!full) {
+          const bool va = t0 + rho_r < valid, vb = t0 + rho_r + 8 < valid;
+          s0 = va ? s0 : -INFINITY;
+          s1 = va ? s1 : -INFINITY;
+          s2 = vb ? s2 : -INFINITY;
+          s3 = vb ? s3 : -INFINITY;
+        }
         float bm0 = fmaxf(s0, s2), bm1 = fmaxf(s1, s3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -226,51 +258,53 @@ __global__ void __launch_bounds__(128)
           bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
         }
         const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-        const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-        const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-        const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
-        l0 = fmaf(l0, al0, p0 + p2);
-        l1 = fmaf(l1, al1, p1 + p3);
-        m0 = mn0;
-        m1 = mn1;
+        // Rescale only when some head's running max moved (rare after the first blocks).
+        if (__any_sync(kFullMask, mn0 != m0 || mn1 != m1)) {
+          const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+          l0 *= al0;
+          l1 *= al1;
 #pragma unroll
-        for (int i3 = 0; i3 < 8; ++i3) {
-          o[i3][0] *= al0;
-          o[i3][1] *= al1;
-          o[i3][2] *= al0;
-          o[i3][3] *= al1;
+          for (int i3 = 0; i3 < 8; ++i3) {
+            o[i3][0] *= al0;
+            o[i3][1] *= al1;
+            o[i3][2] *= al0;
+            o[i3][3] *= al1;
+          }
+          m0 = mn0;
+          m1 = mn1;
         }
+        const float p0 = fast_exp2(s0 - m0), p1 = fast_exp2(s1 - m1);
+        const float p2 = fast_exp2(s2 - m0), p3 = fast_exp2(s3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
         const uint32_t pb0 = movmatrix_trans(f16x2_pack(p0, p1));
         const uint32_t pb1 = movmatrix_trans(f16x2_pack(p2, p3));
         // ---- O^T += V^T . P^T ---------------------------------------------------
-        uint2 w[4][2];  // [row: vrow0, vrow1, vrow0+8, vrow1+8][dims 8r.. / 8r+64..]
-        const int vr[4] = {t0 + vrow0, t0 + vrow1, t0 + vrow0 + 8, t0 + vrow1 + 8};
+        uint2 w[4][2];  // [row: 2c, (2c+1)^4, +8, +8][dims 8r.. / 8r+64..]
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            w[k][h] = *reinterpret_cast<const uint2*>(vt + swz(vr[k], (r >> 1) + 4 * h) + 8 * (r & 1));
-            if (vr[k] >= valid) w[k][h] = make_uint2(0u, 0u);  // rows past the context: zeros, never NaN codes
-          }
+          for (int h = 0; h < 2; ++h) w[k][h] = *reinterpret_cast<const uint2*>(vt + voff[k][h]);
+        if (!full) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (t0 + vrow[k] >= valid) w[k][0] = w[k][1] = make_uint2(0u, 0u);  // never feed NaN codes
+        }
 #pragma unroll
         for (int wi = 0; wi < 2; ++wi) {
-          uint32_t pr[2][2][2];  // [row pair 01 / 23][h][lo (dims +0,+1) / hi (+2,+3)]
+          uint32_t f[2][2][4];  // [row pair 01 / 23][h][dim byte e] fp16x2 (token pair)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t x0 = wi ? w[0][h].y : w[0][h].x, x1 = wi ? w[1][h].y : w[1][h].x;
             const uint32_t x2 = wi ? w[2][h].y : w[2][h].x, x3 = wi ? w[3][h].y : w[3][h].x;
-            pr[0][h][0] = __byte_perm(x0, x1, 0x5140);
-            pr[0][h][1] = __byte_perm(x0, x1, 0x7362);
-            pr[1][h][0] = __byte_perm(x2, x3, 0x5140);
-            pr[1][h][1] = __byte_perm(x2, x3, 0x7362);
+            e4m3x4_to_f16x2x2(__byte_perm(x0, x1, 0x5140), f[0][h][0], f[0][h][1]);
+            e4m3x4_to_f16x2x2(__byte_perm(x0, x1, 0x7362), f[0][h][2], f[0][h][3]);
+            e4m3x4_to_f16x2x2(__byte_perm(x2, x3, 0x5140), f[1][h][0], f[1][h][1]);
+            e4m3x4_to_f16x2x2(__byte_perm(x2, x3, 0x7362), f[1][h][2], f[1][h][3]);
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int it = 4 * wi + e;  // m-tile: output dims 8r + it and 8r + 64 + it
-            const int sh = (e & 1) * 16, hl = e >> 1;
-            mma_16816(o[it], f16x2_from_e4m3x2(pr[0][0][hl] >> sh), f16x2_from_e4m3x2(pr[0][1][hl] >> sh),
-                      f16x2_from_e4m3x2(pr[1][0][hl] >> sh), f16x2_from_e4m3x2(pr[1][1][hl] >> sh), pb0, pb1);
-          }
+          for (int e = 0; e < 4; ++e)  // m-tile 4wi+e: output dims 8r + 4wi + e and 8r + 64 + 4wi + e
+            mma_16816(o[4 * wi + e], f[0][0][e], f[0][1][e], f[1][0][e], f[1][1][e], pb0, pb1);
         }
       }
     }
