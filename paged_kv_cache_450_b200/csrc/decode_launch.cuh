@@ -34,7 +34,7 @@ static cudaError_t launch_mma(const CUtensorMap& kmap, const CUtensorMap& vmap, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(num_kv_heads, p.max_partitions, p.num_seqs);
-  kern<<<grid, T::NW * 32, smem, st>>>(kmap, vmap, p);
+  kern<<<grid, 32, smem, st>>>(kmap, vmap, p);
   count_launch();
   return cudaGetLastError();
 }
