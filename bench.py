@@ -199,9 +199,10 @@ def run_gpu(args, rank, world, local_rank):
     s = spec
     kv_bytes = w.kv_bytes()
     MB = w.block_tables.shape[1]
-    pt = pk.decode_partition_tokens(s.num_seqs, s.num_kv_heads, s.block_size, MB, args.partition_tokens)
+    pt = pk.decode_partition_tokens(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
+                                    s.cache_dtype, args.partition_tokens)
     ws_bytes = pk.decode_workspace_bytes(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
-                                         pt)
+                                         s.cache_dtype, pt)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     out = torch.empty_like(w.q)
     kc, vc = w.key_cache, w.value_cache

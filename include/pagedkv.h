@@ -183,7 +183,7 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
  *   order between them) race on the array and give wrong results: order
  *   them on one stream.
  * - A call whose partials need more than PKV_DECODE_STATIC_SCRATCH_BYTES
- *   (pkv_decode_workspace_bytes() with the same arguments) returns
+ *   (pkv_decode_workspace_bytes() for the same call) returns
  *   PKV_ERR_WORKSPACE and launches nothing; a larger partition_tokens lowers
  *   the need.
  * Other errors: as pkv_paged_attention_decode.
@@ -198,21 +198,26 @@ int pkv_paged_attention_decode_static(void* out, const void* q, const void* key_
 
 /*
  * Partition length (tokens) the decode call uses for these arguments:
- * partition_tokens if it is non-zero, else the automatic choice, which
- * depends on the shape and on the current device's SM count.  Returns a
- * negative PKV_ERR_* code for unsupported arguments.
+ * partition_tokens if it is non-zero, else the automatic choice.  The
+ * automatic choice depends on the shape, on which kernel serves it
+ * (cache_dtype, head_dim and the query-head group select it) and on the
+ * current device's SM count: the largest power of two <= 4096 that still
+ * splits the longest possible context (max_blocks_per_seq * block_size) into
+ * at least 4 partitions and gives at least one CTA per resident slot of the
+ * kernel; a single partition when that context is 512 tokens or less.
+ * Returns a negative PKV_ERR_* code for unsupported arguments.
  */
-int pkv_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
-                                int partition_tokens);
+int pkv_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int max_blocks_per_seq, int cache_dtype, int partition_tokens);
 
-/* Partitions per sequence the workspace must hold (max over sequences). */
-int pkv_decode_max_partitions(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
-                              int partition_tokens);
+/* Partitions per sequence the workspace must hold (max over sequences); same arguments. */
+int pkv_decode_max_partitions(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int cache_dtype, int partition_tokens);
 
 /* Workspace bytes pkv_paged_attention_decode needs for these arguments
  * (0 when no sequence can need more than one partition). */
-size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                                  int block_size, int max_blocks_per_seq, int partition_tokens);
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int cache_dtype, int partition_tokens);
 
 /*
  * Copy-on-write block copy.

@@ -97,24 +97,32 @@ def paged_kv_write(k, v, slot_mapping, key_cache, value_cache, *, k_scale: float
                                       _stream(dev, stream)), "paged_kv_write")
 
 
-def decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens=0) -> int:
-    r = _lib.load().pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
-                                                partition_tokens)
+def _cache_code(cache_dtype) -> int:
+    return cache_dtype if isinstance(cache_dtype, int) else _DTYPES[cache_dtype]
+
+
+def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                            cache_dtype, partition_tokens=0) -> int:
+    """Split-context partition length (tokens) the decode call will use."""
+    r = _lib.load().pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                max_blocks_per_seq, _cache_code(cache_dtype), partition_tokens)
     _check(min(r, 0), "decode_partition_tokens")
     return r
 
 
-def decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens=0) -> int:
-    r = _lib.load().pkv_decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
-                                              partition_tokens)
+def decode_max_partitions(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                          cache_dtype, partition_tokens=0) -> int:
+    r = _lib.load().pkv_decode_max_partitions(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_blocks_per_seq, _cache_code(cache_dtype), partition_tokens)
     _check(min(r, 0), "decode_max_partitions")
     return r
 
 
 def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-                           partition_tokens=0) -> int:
+                           cache_dtype, partition_tokens=0) -> int:
     return int(_lib.load().pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                      max_blocks_per_seq, partition_tokens))
+                                                      max_blocks_per_seq, _cache_code(cache_dtype),
+                                                      partition_tokens))
 
 
 def paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens, scale: float,
@@ -145,7 +153,7 @@ def paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens
         _cuda(out)
         if out.shape != q.shape or out.dtype != q.dtype:
             raise ValueError("out must match q")
-    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, MB, partition_tokens) if B else 0
+    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, MB, key_cache.dtype, partition_tokens) if B else 0
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_ptr = workspace.data_ptr() if workspace is not None else None

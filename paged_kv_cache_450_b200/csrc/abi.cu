@@ -106,19 +106,26 @@ static bool copy_to_host(std::vector<T>& dst, const T* src, size_t n, cudaStream
 
 constexpr int kMaxPartitionTokens = 16384;
 
-// Automatic split-context partition length: 512 tokens, halved (down to 128)
-// while the grid would hold fewer than ~4 waves of 6 CTAs per SM; a single
-// partition when the longest possible context fits in one.
-static int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq) {
+// Resident CTAs per SM of the decode kernel that serves these arguments
+// (from the kernels' shared-memory and register budgets on B200).
+static int decode_ctas_per_sm(int cache_dtype, int head_dim, int group, int block_size) {
+  if (decode_uses_mma(cache_dtype, head_dim, group, block_size)) return 16;  // one warp, 13 KB
+  return 6;                                                                  // four warps, ~34 KB
+}
+
+// Automatic split-context partition length (see pkv_decode_partition_tokens).
+// Longer partitions cost less per token (one CTA set-up and one partial per
+// partition); at least 4 per long sequence keep mixed lengths balanced, and
+// at least one CTA per resident slot keeps every SM busy.
+static int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                                 int ctas_per_sm) {
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
-  const int64_t target = 4LL * 6 * sm_count();
-  int pt = 512;
-  while (pt > 128 && pairs * cdiv64(max_ctx, pt) < target) pt /= 2;
-  if (pt < block_size) pt = block_size;
-  if (max_ctx <= pt) pt = static_cast<int>(cdiv64(max_ctx, block_size) * block_size);
-  if (pt < block_size) pt = block_size;
-  return pt;
+  if (max_ctx <= 512) return static_cast<int>(cdiv64(max_ctx, block_size) * block_size);
+  const int64_t slots = static_cast<int64_t>(ctas_per_sm) * sm_count();
+  int pt = 4096;
+  while (pt > 128 && (cdiv64(max_ctx, pt) < 4 || pairs * cdiv64(max_ctx, pt) < slots)) pt /= 2;
+  return pt < block_size ? block_size : pt;
 }
 
 }  // namespace pkv
@@ -208,30 +215,33 @@ int pkv_paged_kv_write(const void* k, const void* v, const int64_t* slot_mapping
   return launch_kv_write(a, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
-int pkv_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
-                                int partition_tokens) {
+int pkv_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int max_blocks_per_seq, int cache_dtype, int partition_tokens) {
   if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
-  if (num_seqs < 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_BAD_SHAPE;
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_BAD_SHAPE;
   if (partition_tokens != 0) {
     if (partition_tokens < 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
       return PKV_ERR_PARTITION;
     return partition_tokens;
   }
-  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq);
+  const int group = num_q_heads % num_kv_heads == 0 ? num_q_heads / num_kv_heads : 0;
+  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
+                               decode_ctas_per_sm(cache_dtype, head_dim, group, block_size));
 }
 
-int pkv_decode_max_partitions(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
-                              int partition_tokens) {
-  const int pt = pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
-                                             partition_tokens);
+int pkv_decode_max_partitions(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int cache_dtype, int partition_tokens) {
+  const int pt = pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                             max_blocks_per_seq, cache_dtype, partition_tokens);
   if (pt < 0) return pt;
   return static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
 }
 
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                                  int max_blocks_per_seq, int partition_tokens) {
-  const int P = pkv_decode_max_partitions(num_seqs, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens);
-  if (P <= 1 || num_q_heads <= 0 || head_dim <= 0) return 0;
+                                  int max_blocks_per_seq, int cache_dtype, int partition_tokens) {
+  const int P = pkv_decode_max_partitions(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                          max_blocks_per_seq, cache_dtype, partition_tokens);
+  if (P <= 1 || head_dim <= 0) return 0;
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * P;
   return align256(rows * 2 * sizeof(float)) + rows * head_dim * sizeof(float);
 }
@@ -257,13 +267,13 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
   if (static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffffLL) return PKV_ERR_BAD_SHAPE;
   if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
   if (cache_dtype == PKV_DTYPE_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_BAD_SHAPE;
-  const int pt = pkv_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_blocks_per_seq,
-                                             partition_tokens);
+  const int pt = pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                             max_blocks_per_seq, cache_dtype, partition_tokens);
   if (pt < 0) return pt;
   const int P = static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
   if (P > 65535) return PKV_ERR_PARTITION;
   const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                 max_blocks_per_seq, partition_tokens);
+                                                 max_blocks_per_seq, cache_dtype, partition_tokens);
   if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -60,7 +60,7 @@ extern "C" int pkv_paged_attention_decode_static(void* out, const void* q, const
                                                  int partition_tokens, void* stream) {
   // Refuse, before touching the device, any call whose partials would not fit.
   const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                 max_blocks_per_seq, partition_tokens);
+                                                 max_blocks_per_seq, cache_dtype, partition_tokens);
   if (need > kScratchBytes) return PKV_ERR_WORKSPACE;
   int status = PKV_OK;
   void* scratch = scratch_address(&status);

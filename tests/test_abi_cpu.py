@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import paged_kv_cache_450_b200 as pk
 from paged_kv_cache_450_b200 import _lib
@@ -82,19 +83,26 @@ def test_write_and_copy_argument_errors():
 
 
 def test_partition_choice_and_workspace_size():
-    # single partition when the longest context fits: no workspace
-    assert pk.decode_partition_tokens(4, 4, 16, 7) == 112
-    assert pk.decode_workspace_bytes(4, 4, 4, 64, 16, 7) == 0
-    # 64 sequences x 32 heads x 2048 tokens: 512-token partitions
-    assert pk.decode_partition_tokens(64, 32, 16, 128) == 512
-    P = pk.decode_max_partitions(64, 32, 16, 128)
+    bf16, fp8 = torch.bfloat16, torch.float8_e4m3fn
+    # single partition when the longest context fits in 512 tokens: no workspace
+    assert pk.decode_partition_tokens(4, 4, 4, 64, 16, 7, torch.float32) == 112
+    assert pk.decode_workspace_bytes(4, 4, 4, 64, 16, 7, torch.float32) == 0
+    # 64 sequences x 32 heads, up to 2048 tokens: 512 (at least 4 partitions per long sequence)
+    assert pk.decode_partition_tokens(64, 32, 32, 128, 16, 128, bf16) == 512
+    P = pk.decode_max_partitions(64, 32, 32, 128, 16, 128, bf16)
     assert P == 4
     rows = 64 * 32 * P
-    assert pk.decode_workspace_bytes(64, 32, 32, 128, 16, 128) == ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
+    assert pk.decode_workspace_bytes(64, 32, 32, 128, 16, 128, bf16) == \
+        ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
+    # 256 x 40 heads up to 4096 tokens: 1024
+    assert pk.decode_partition_tokens(256, 40, 40, 128, 16, 256, bf16) == 1024
+    # fp8 GQA 64/8: 16 x 32k -> enough CTAs for one per resident slot (148 SMs assumed without a GPU)
+    assert pk.decode_partition_tokens(16, 64, 8, 128, 16, 2048, fp8) == 1024
+    assert pk.decode_partition_tokens(128, 64, 8, 128, 16, 512, fp8) == 2048
     # explicit partition lengths
-    assert pk.decode_partition_tokens(1, 1, 16, 100, 48) == 48
+    assert pk.decode_partition_tokens(1, 1, 1, 128, 16, 100, bf16, 48) == 48
     with pytest.raises(pk.PagedKVError):
-        pk.decode_partition_tokens(1, 1, 16, 100, 40)
+        pk.decode_partition_tokens(1, 1, 1, 128, 16, 100, bf16, 40)
 
 
 def test_ops_refuse_cpu_tensors():

@@ -65,8 +65,8 @@ def test_partition_partials_match_oracle(cd):
     pt = 64
     B, Hq, d = 3, 8, 128
     MB = w.block_tables.shape[1]
-    P = pk.decode_max_partitions(B, 2, 16, MB, pt)
-    nbytes = pk.decode_workspace_bytes(B, Hq, 2, d, 16, MB, pt)
+    P = pk.decode_max_partitions(B, Hq, 2, d, 16, MB, cd, pt)
+    nbytes = pk.decode_workspace_bytes(B, Hq, 2, d, 16, MB, cd, pt)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
     gpu_step(w, partition_tokens=pt, workspace=ws)
     rows = B * Hq * P

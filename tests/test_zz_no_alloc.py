@@ -55,7 +55,8 @@ def test_static_scratch_matches_workspace_entry_point_two_calls():
     cases = [(w1, 0), (w2, 128)]
     for w, pt in cases:
         need = pk.decode_workspace_bytes(w.spec.num_seqs, w.spec.num_q_heads, w.spec.num_kv_heads,
-                                         w.spec.head_dim, w.spec.block_size, w.block_tables.shape[1], pt)
+                                         w.spec.head_dim, w.spec.block_size, w.block_tables.shape[1],
+                                         w.spec.cache_dtype, pt)
         assert 0 < need <= STATIC_LIMIT       # the cases really use the split-context scratch
     refs = [reference(w, pt) for w, pt in cases]
     torch.cuda.synchronize()
@@ -86,7 +87,8 @@ def test_static_scratch_rejects_calls_that_need_more_than_the_array():
     MB = 4096  # a table wide enough that 128-token partitions need > 16 MiB of partials
     tables = torch.zeros((s.num_seqs, MB), dtype=torch.int32, device=DEV)
     tables[:, : w.block_tables.shape[1]] = w.block_tables
-    need = pk.decode_workspace_bytes(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB, 128)
+    need = pk.decode_workspace_bytes(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
+                                     s.cache_dtype, 128)
     assert need > STATIC_LIMIT
     big = W.DecodeWorkload(**{**w.__dict__, "block_tables": tables})
     out = torch.zeros_like(w.q)
