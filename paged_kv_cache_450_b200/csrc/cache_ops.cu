@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256)
     paged_kv_write_kernel(const TI* __restrict__ k, const TI* __restrict__ v, const int64_t* __restrict__ slots,
                           TC* __restrict__ kc, TC* __restrict__ vc, int64_t num_blocks, int block_size,
                           int row_elems, float k_inv, float v_inv, unsigned* status) {
+  pdl_wait_and_release();
   const int64_t t = blockIdx.x;
   const int64_t slot = slots[t];
   if (slot < 0) return;  // padding token
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(256)
     kv_block_copy_kernel(const int64_t* __restrict__ pairs, int64_t num_pairs, uint8_t* kc, uint8_t* vc,
                          int64_t num_blocks, int64_t block_bytes, unsigned* status) {
   constexpr int kIlp = 4;
+  pdl_wait_and_release();
   const int64_t vecs = block_bytes / 16;
   for (int64_t pi = blockIdx.y; pi < num_pairs; pi += gridDim.y) {
     const int64_t src = pairs[2 * pi], dst = pairs[2 * pi + 1];
@@ -114,11 +116,10 @@ static cudaError_t launch_write(const KvWriteArgs& a, cudaStream_t st) {
   const int row_elems = a.num_kv_heads * a.head_dim;
   const int chunks = row_elems / 8;
   const int threads = chunks >= 256 ? 256 : ((chunks + 31) / 32) * 32;
-  paged_kv_write_kernel<TI, TC><<<static_cast<unsigned>(a.num_tokens), threads, 0, st>>>(
-      static_cast<const TI*>(a.k), static_cast<const TI*>(a.v), a.slot_mapping, static_cast<TC*>(a.key_cache),
-      static_cast<TC*>(a.value_cache), a.num_blocks, a.block_size, row_elems, a.k_inv, a.v_inv, a.status);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(paged_kv_write_kernel<TI, TC>, dim3(static_cast<unsigned>(a.num_tokens)), dim3(threads), 0, st,
+                    static_cast<const TI*>(a.k), static_cast<const TI*>(a.v), a.slot_mapping,
+                    static_cast<TC*>(a.key_cache), static_cast<TC*>(a.value_cache), a.num_blocks, a.block_size,
+                    row_elems, a.k_inv, a.v_inv, a.status);
 }
 
 cudaError_t launch_kv_write(const KvWriteArgs& a, cudaStream_t st) {
@@ -138,10 +139,8 @@ cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, void* kc,
   const int64_t per_cta = 256 * 4;
   const unsigned gx = static_cast<unsigned>((vecs + per_cta - 1) / per_cta);
   const unsigned gy = static_cast<unsigned>(num_pairs < 65535 ? num_pairs : 65535);
-  kv_block_copy_kernel<<<dim3(gx, gy), 256, 0, st>>>(pairs, num_pairs, static_cast<uint8_t*>(kc),
-                                                       static_cast<uint8_t*>(vc), num_blocks, block_bytes, status);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(kv_block_copy_kernel, dim3(gx, gy), dim3(256), 0, st, pairs, num_pairs, static_cast<uint8_t*>(kc),
+                    static_cast<uint8_t*>(vc), num_blocks, block_bytes, status);
 }
 
 }  // namespace pkv

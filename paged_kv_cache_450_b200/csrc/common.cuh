@@ -32,6 +32,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so it may be scheduled while the previous grid on the stream
+// is still running.  It first waits for that grid to complete (and its writes
+// to become visible) -- nothing is read before -- and then lets its own
+// dependents be scheduled.  Only the launch latency overlaps, never data.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- mbarrier ---------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   float* p_s = q_s + G * D;
   int* ids = reinterpret_cast<int*>(p_s + T::NW * G * BS);
 
+  pdl_wait_and_release();
   const int hk = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 template <typename TQ, int D>
 __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeParams p) {
   constexpr int PVV = D / 32;
+  pdl_wait_and_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
   if (row >= static_cast<int64_t>(p.num_seqs) * p.num_q_heads) return;

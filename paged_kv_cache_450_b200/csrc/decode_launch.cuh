@@ -18,11 +18,10 @@ static cudaError_t launch_partition(const CUtensorMap& kmap, const CUtensorMap& 
   auto kern = paged_decode_partition_kernel<TQ, TC, D, BS, G>;
   const size_t smem = T::smem_bytes(p.partition_blocks);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(num_kv_heads, p.max_partitions, p.num_seqs);
-  kern<<<grid, T::NW * 32, smem, st>>>(kmap, vmap, p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(T::NW * 32), smem, st, kmap, vmap, p);
 }
 
 template <typename TQ, int BS>
@@ -32,19 +31,17 @@ static cudaError_t launch_mma(const CUtensorMap& kmap, const CUtensorMap& vmap, 
   auto kern = paged_decode_gqa8_fp8_mma_kernel<TQ, BS>;
   const size_t smem = T::smem_bytes(p.partition_blocks);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(num_kv_heads, p.max_partitions, p.num_seqs);
-  kern<<<grid, 32, smem, st>>>(kmap, vmap, p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(32), smem, st, kmap, vmap, p);
 }
 
 template <typename TQ, int D>
 static cudaError_t launch_reduce(const DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_q_heads;
-  paged_decode_reduce_kernel<TQ, D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(paged_decode_reduce_kernel<TQ, D>, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st,
+                    p);
 }
 
 template <typename TQ, typename TC, int D, int BS>

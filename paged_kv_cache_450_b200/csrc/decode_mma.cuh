@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(32, MINB)
   uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::STAGE_AREA);
   int* ids = reinterpret_cast<int*>(data + T::STAGE_AREA + T::BAR_BYTES);
 
+  pdl_wait_and_release();
   const int hk = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x;
   const int r = lane >> 2, c = lane & 3;  // fragment row / column-pair of this lane
