@@ -193,3 +193,57 @@ def test_launch_count_counts_kernels():
     n0 = pk.launch_count()
     gpu_step(w, partition_tokens=128, validate=False)
     assert pk.launch_count() - n0 == 3   # write, partition pass, reduce
+
+
+def _poison_unused_rows(w):
+    """NaN bit patterns in every cache row no sequence reads: the tail rows of
+    each last block and all free blocks (bf16 0x7FC0, fp8 0x7F, fp32 NaN)."""
+    bs = w.spec.block_size
+    used = torch.zeros(w.num_blocks, bs, dtype=torch.bool, device=w.key_cache.device)
+    for b, c in enumerate(w.ctx_list):
+        n = -(-c // bs)
+        for j in range(n):
+            blk = int(w.block_tables[b, j])
+            used[blk, : min(bs, c - j * bs)] = True
+    for cache in (w.key_cache, w.value_cache):
+        if cache.dtype == torch.float8_e4m3fn:
+            raw = cache.view(torch.uint8)
+            raw[~used] = 0x7F
+        elif cache.dtype == torch.bfloat16:
+            raw = cache.view(torch.int16)
+            raw[~used] = 0x7FC0
+        else:
+            cache[~used] = float("nan")
+
+
+@pytest.mark.parametrize("spec", [W.TINY.with_(new_tokens=False),
+                                  W.LLAMA7B.with_(num_seqs=5, num_q_heads=4, num_kv_heads=4, ctx=("list", (1, 17, 200, 513, 31)),
+                                                  new_tokens=False),
+                                  W.GQA_BATCH.with_(num_seqs=5, ctx=("list", (1, 17, 200, 513, 31)), new_tokens=False),
+                                  W.GQA_BATCH.with_(num_seqs=3, block_size=32, ctx=("list", (5, 33, 70)),
+                                                    new_tokens=False)],
+                         ids=["fp32-mha", "bf16-mha", "fp8-gqa-mma", "fp8-gqa-mma-bs32"])
+def test_rows_past_the_context_are_never_used(spec):
+    w = W.make_decode_workload(spec, seed=12, device=DEV)
+    _poison_unused_rows(w)
+    for pt in (0, 2 * spec.block_size):
+        out = check_step(w, partition_tokens=pt, what=f"poisoned pool pt={pt}")
+        assert torch.isfinite(out.float()).all()
+
+
+def test_tensor_core_kernel_guards_bad_block_ids():
+    w = W.make_decode_workload(W.GQA_BATCH.with_(num_seqs=3, ctx=("list", (40, 300, 7)), new_tokens=False), seed=13,
+                               device=DEV)
+    pk.device_status(clear=True)
+    bad = w.block_tables.clone()
+    bad[1, 3] = -7
+    bad[0, 0] = w.num_blocks
+    out = pk.paged_attention_decode(w.q, w.key_cache, w.value_cache, bad, w.context_lens, w.scale,
+                                    k_scale=w.k_scale, v_scale=w.v_scale, partition_tokens=64)
+    torch.cuda.synchronize()
+    assert pk.device_status(clear=True) & pk.STATUS_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+    # the sequence without bad ids is unaffected
+    rows = np.arange(2 * 64, 3 * 64)
+    _, _, ref = oracle_step(w, rows=rows)
+    assert_close(f64(out).reshape(-1, 128)[rows], ref, *tol_for(w), what="unaffected sequence")
