@@ -258,11 +258,13 @@ def run_gpu(args, rank, world, local_rank):
     host = {k: (getattr(w, k).cpu().pin_memory() if getattr(w, k) is not None else None)
             for k in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens", "copy_pairs")}
     out_h = torch.empty(w.q.shape, dtype=w.q.dtype, pin_memory=True)
+    staging = torch.empty(pk.decode_step_staging_bytes(host["q"], host["new_k"], kc, host["block_tables"],
+                                                       host["copy_pairs"], pt), dtype=torch.uint8, device=dev)
 
     def e2e_step():
         pk.decode_step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
                        host["context_lens"], kc, vc, w.scale, copy_pairs=host["copy_pairs"], k_scale=w.k_scale,
-                       v_scale=w.v_scale, out=out_h, workspace=workspace, partition_tokens=pt, stream=stream)
+                       v_scale=w.v_scale, out=out_h, staging=staging, partition_tokens=pt, stream=stream)
 
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(args.warmup, 10)):
@@ -316,7 +318,7 @@ def run_gpu(args, rank, world, local_rank):
                          "traffic": profile_traffic("paged_decode_" + s.name, s.name)},
             "e2e": {"value": round(total_kv / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": e2e_steps,
                     "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "paged_kv_cache_450_b200.decode_step (pinned host inputs and output)"},
+                    "api": "paged_kv_cache_450_b200.decode_step -> pkv_decode_step_host (pinned host inputs and output)"},
             "gpu_launches": int(launches),
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -243,6 +243,45 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
                       int64_t num_blocks, int64_t block_bytes, int validate, void* stream);
 
 /*
+ * One whole decode step with the per-step inputs and the output in HOST memory.
+ *
+ * Source: the decode step of "vLLM 与 KV Cache", KV Cache：为什么需要缓存 (append
+ * the new token's K,V, then attend over the cache) with the copy-on-write of
+ * "vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点 (copy first, then write).
+ * Enqueued on `stream`, in order: host -> device copies of every per-step
+ * input into `staging`; pkv_kv_block_copy (if num_pairs > 0);
+ * pkv_paged_kv_write (if num_tokens > 0); pkv_paged_attention_decode; the
+ * device -> host copy of the output.  Synchronise `stream` before reading
+ * out_host or reusing the input buffers.  The host buffers should be pinned
+ * (page-locked): pageable buffers make the copies synchronous.
+ *
+ * out_host, q_host      host [num_seqs][num_q_heads][head_dim] of q_dtype.
+ * k_host, v_host,       host [num_tokens][num_kv_heads][head_dim] of q_dtype and
+ * slot_mapping_host     host int64 [num_tokens] (see pkv_paged_kv_write).
+ * block_tables_host,    host int32 [num_seqs][max_blocks_per_seq], [num_seqs].
+ * context_lens_host
+ * copy_pairs_host       host int64 [num_pairs][2] (may be NULL when num_pairs == 0).
+ * key_cache, value_cache  device caches (layout above).
+ * staging               device scratch of at least pkv_decode_step_staging_bytes(...)
+ *                       bytes, 256-byte aligned, caller-owned; holds the copied
+ *                       inputs, the output and the decode workspace.
+ * Other arguments and errors: as pkv_paged_attention_decode / pkv_paged_kv_write /
+ * pkv_kv_block_copy (without validation).  A negative code means nothing was enqueued.
+ */
+int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
+                         const int64_t* slot_mapping_host, int64_t num_tokens, const int32_t* block_tables_host,
+                         const int32_t* context_lens_host, const int64_t* copy_pairs_host, int64_t num_pairs,
+                         void* key_cache, void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads,
+                         int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                         float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                         void* staging, size_t staging_bytes, void* stream);
+
+/* Staging bytes pkv_decode_step_host needs for these arguments. */
+size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                     int max_blocks_per_seq, int q_dtype, int cache_dtype, int partition_tokens,
+                                     int64_t num_tokens, int64_t num_pairs);
+
+/*
  * Reads the current device's status word (PKV_STATUS_* bits) into *status,
  * after synchronising `stream`; clears it if `clear` != 0.
  */

@@ -30,7 +30,8 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_step", "decode_workspace_bytes",
+__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_step", "decode_step_staging_bytes",
+           "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
            "library_path"]
 
@@ -199,38 +200,63 @@ def launch_count() -> int:
     return int(_lib.load().pkv_launch_count())
 
 
+def decode_step_staging_bytes(q, new_k, key_cache, block_tables, copy_pairs=None, partition_tokens: int = 0) -> int:
+    """Device staging bytes decode_step needs for host inputs of these shapes."""
+    B, Hq, d = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    T = 0 if new_k is None else new_k.shape[0]
+    n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+    return int(_lib.load().pkv_decode_step_staging_bytes(B, Hq, Hkv, d, bs, block_tables.shape[1], _dtype(q),
+                                                         _dtype(key_cache), partition_tokens, T, n_pairs))
+
+
 def decode_step(q, new_k, new_v, slot_mapping, block_tables, context_lens, key_cache, value_cache, scale: float, *,
                 copy_pairs=None, k_scale: float = 1.0, v_scale: float = 1.0, out=None, workspace=None,
-                partition_tokens: int = 0, stream=None):
+                staging=None, partition_tokens: int = 0, stream=None):
     """One decode step of one attention layer over a device-resident paged cache.
 
     Order: copy-on-write block copies (``copy_pairs``, if any), the new-token
     write (``new_k``/``new_v`` at ``slot_mapping``), then decode attention over
-    ``context_lens`` (which include the new token).  The per-step inputs may be
-    host tensors (pinned memory makes the copies asynchronous): they are copied
-    to the cache's device on the stream, and the result is copied back into
-    ``out`` (a host tensor, allocated pinned when not given).  With device
-    inputs everything stays on the device.  Returns the output."""
+    ``context_lens`` (which include the new token).
+
+    Host inputs (CPU tensors; pinned memory keeps the copies asynchronous): a
+    single library call (pkv_decode_step_host) enqueues the copies in, the
+    step and the copy of the output into ``out`` (a host tensor, allocated
+    pinned when not given); ``staging`` is the device scratch it uses
+    (allocated when not given, see decode_step_staging_bytes).  Synchronise
+    the stream before reading ``out``.  Device inputs: everything stays on the
+    device and the device output is returned."""
     dev = key_cache.device
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    host = q.device.type == "cpu"
-
-    def to_dev(t):
-        return t.to(dev, non_blocking=True) if t is not None and t.device != dev else t
-
+    if q.device.type == "cpu":
+        host = [t for t in (q, new_k, new_v, slot_mapping, block_tables, context_lens, copy_pairs) if t is not None]
+        if any(t.device.type != "cpu" or not t.is_contiguous() for t in host):
+            raise ValueError("host inputs must all be contiguous CPU tensors")
+        _cuda(key_cache, value_cache)
+        B, Hq, d = q.shape
+        NB, bs, Hkv, _ = key_cache.shape
+        T = 0 if new_k is None else new_k.shape[0]
+        n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+        need = decode_step_staging_bytes(q, new_k, key_cache, block_tables, copy_pairs, partition_tokens)
+        if staging is None:
+            staging = torch.empty(need, dtype=torch.uint8, device=dev)
+        if out is None:
+            out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        with torch.cuda.device(dev):
+            _check(_lib.load().pkv_decode_step_host(
+                out.data_ptr(), q.data_ptr(), ptr(new_k), ptr(new_v), ptr(slot_mapping), T, block_tables.data_ptr(),
+                context_lens.data_ptr(), ptr(copy_pairs), n_pairs, key_cache.data_ptr(), value_cache.data_ptr(), B, Hq,
+                Hkv, d, bs, block_tables.shape[1], NB, float(scale), float(k_scale), float(v_scale), _dtype(q),
+                _dtype(key_cache), int(partition_tokens), staging.data_ptr(),
+                staging.numel() * staging.element_size(), ctypes.c_void_p(st.cuda_stream)), "decode_step")
+        return out
     with torch.cuda.device(dev), torch.cuda.stream(st):
-        qd, kd, vd, sd, td, ld, pd = (to_dev(t) for t in (q, new_k, new_v, slot_mapping, block_tables,
-                                                           context_lens, copy_pairs))
-        if pd is not None and pd.numel():
-            kv_block_copy(pd, key_cache, value_cache, stream=st)
-        if kd is not None:
-            paged_kv_write(kd, vd, sd, key_cache, value_cache, k_scale=k_scale, v_scale=v_scale, stream=st)
-        res = paged_attention_decode(qd, key_cache, value_cache, td, ld, scale, k_scale=k_scale, v_scale=v_scale,
-                                     out=None if host else out, workspace=workspace,
-                                     partition_tokens=partition_tokens, stream=st)
-        if host:
-            if out is None:
-                out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
-            out.copy_(res, non_blocking=True)
-            return out
-        return res
+        if copy_pairs is not None and copy_pairs.numel():
+            kv_block_copy(copy_pairs, key_cache, value_cache, stream=st)
+        if new_k is not None:
+            paged_kv_write(new_k, new_v, slot_mapping, key_cache, value_cache, k_scale=k_scale, v_scale=v_scale,
+                           stream=st)
+        return paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens, scale, k_scale=k_scale,
+                                      v_scale=v_scale, out=out, workspace=workspace,
+                                      partition_tokens=partition_tokens, stream=st)

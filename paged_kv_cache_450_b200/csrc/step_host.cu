@@ -1,0 +1,140 @@
+// step_host.cu -- one decode step whose per-step inputs and output live in
+// host memory: the copies in, the three operations and the copy out, all
+// enqueued on the caller's stream by one call (for serving loops that keep
+// the KV cache on the device and everything else on the host).
+#include <cuda_runtime.h>
+
+#include "../../include/pagedkv.h"
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t dtype_bytes(int dtype) {
+  switch (dtype) {
+    case PKV_DTYPE_F32: return 4;
+    case PKV_DTYPE_BF16: return 2;
+    case PKV_DTYPE_FP8_E4M3: return 1;
+    default: return 0;
+  }
+}
+
+// Offsets of the staged pieces inside the staging buffer.
+struct StagingLayout {
+  size_t q, out, k, v, slots, tables, lens, pairs, workspace, workspace_bytes, total;
+};
+
+bool layout(StagingLayout* L, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+            int max_blocks_per_seq, int q_dtype, int cache_dtype, int partition_tokens, int64_t num_tokens,
+            int64_t num_pairs) {
+  const size_t es = dtype_bytes(q_dtype);
+  if (!es || num_seqs < 0 || num_tokens < 0 || num_pairs < 0 || max_blocks_per_seq <= 0) return false;
+  const size_t qb = static_cast<size_t>(num_seqs) * num_q_heads * head_dim * es;
+  const size_t kb = static_cast<size_t>(num_tokens) * num_kv_heads * head_dim * es;
+  size_t off = 0;
+  L->q = off;
+  off = align256(off + qb);
+  L->out = off;
+  off = align256(off + qb);
+  L->k = off;
+  off = align256(off + kb);
+  L->v = off;
+  off = align256(off + kb);
+  L->slots = off;
+  off = align256(off + static_cast<size_t>(num_tokens) * sizeof(int64_t));
+  L->tables = off;
+  off = align256(off + static_cast<size_t>(num_seqs) * max_blocks_per_seq * sizeof(int32_t));
+  L->lens = off;
+  off = align256(off + static_cast<size_t>(num_seqs) * sizeof(int32_t));
+  L->pairs = off;
+  off = align256(off + static_cast<size_t>(num_pairs) * 2 * sizeof(int64_t));
+  L->workspace = off;
+  L->workspace_bytes = num_seqs > 0 ? pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                                 block_size, max_blocks_per_seq, cache_dtype,
+                                                                 partition_tokens)
+                                    : 0;
+  L->total = align256(off + L->workspace_bytes);
+  return true;
+}
+
+bool h2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return true;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                int block_size, int max_blocks_per_seq, int q_dtype, int cache_dtype,
+                                                int partition_tokens, int64_t num_tokens, int64_t num_pairs) {
+  StagingLayout L;
+  if (!layout(&L, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, q_dtype,
+              cache_dtype, partition_tokens, num_tokens, num_pairs))
+    return 0;
+  return L.total;
+}
+
+extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
+                                    const int64_t* slot_mapping_host, int64_t num_tokens,
+                                    const int32_t* block_tables_host, const int32_t* context_lens_host,
+                                    const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
+                                    void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                                    float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                                    void* staging, size_t staging_bytes, void* stream) {
+  if (num_seqs < 0 || num_tokens < 0 || num_pairs < 0) return PKV_ERR_BAD_SHAPE;
+  if (num_seqs == 0 && num_tokens == 0 && num_pairs == 0) return PKV_OK;
+  if (!staging || !key_cache || !value_cache) return PKV_ERR_NULL_POINTER;
+  if (num_seqs > 0 && (!out_host || !q_host || !block_tables_host || !context_lens_host)) return PKV_ERR_NULL_POINTER;
+  if (num_tokens > 0 && (!k_host || !v_host || !slot_mapping_host)) return PKV_ERR_NULL_POINTER;
+  if (num_pairs > 0 && !copy_pairs_host) return PKV_ERR_NULL_POINTER;
+  if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  const int pt = num_seqs > 0 ? pkv_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                            max_blocks_per_seq, cache_dtype, partition_tokens)
+                              : 0;
+  if (pt < 0) return pt;
+  StagingLayout L;
+  if (!layout(&L, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, q_dtype, cache_dtype,
+              partition_tokens, num_tokens, num_pairs))
+    return PKV_ERR_BAD_DTYPE;
+  if (staging_bytes < L.total) return PKV_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t es = dtype_bytes(q_dtype);
+  const size_t qb = static_cast<size_t>(num_seqs) * num_q_heads * head_dim * es;
+  const size_t kb = static_cast<size_t>(num_tokens) * num_kv_heads * head_dim * es;
+  // Copies in.
+  if (!h2d(base + L.q, q_host, qb, st) || !h2d(base + L.k, k_host, kb, st) || !h2d(base + L.v, v_host, kb, st) ||
+      !h2d(base + L.slots, slot_mapping_host, static_cast<size_t>(num_tokens) * sizeof(int64_t), st) ||
+      !h2d(base + L.tables, block_tables_host,
+           static_cast<size_t>(num_seqs) * max_blocks_per_seq * sizeof(int32_t), st) ||
+      !h2d(base + L.lens, context_lens_host, static_cast<size_t>(num_seqs) * sizeof(int32_t), st) ||
+      !h2d(base + L.pairs, copy_pairs_host, static_cast<size_t>(num_pairs) * 2 * sizeof(int64_t), st))
+    return PKV_ERR_CUDA;
+  int rc;
+  if (num_pairs > 0) {
+    const int64_t block_bytes =
+        static_cast<int64_t>(block_size) * num_kv_heads * head_dim * static_cast<int64_t>(dtype_bytes(cache_dtype));
+    rc = pkv_kv_block_copy(reinterpret_cast<const int64_t*>(base + L.pairs), num_pairs, key_cache, value_cache,
+                           num_blocks, block_bytes, 0, stream);
+    if (rc) return rc;
+  }
+  if (num_tokens > 0) {
+    rc = pkv_paged_kv_write(base + L.k, base + L.v, reinterpret_cast<const int64_t*>(base + L.slots), num_tokens,
+                            key_cache, value_cache, num_blocks, block_size, num_kv_heads, head_dim, q_dtype,
+                            cache_dtype, k_scale, v_scale, 0, stream);
+    if (rc) return rc;
+  }
+  if (num_seqs > 0) {
+    rc = pkv_paged_attention_decode(base + L.out, base + L.q, key_cache, value_cache,
+                                    reinterpret_cast<const int32_t*>(base + L.tables),
+                                    reinterpret_cast<const int32_t*>(base + L.lens), num_seqs, num_q_heads,
+                                    num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale,
+                                    v_scale, q_dtype, cache_dtype, pt, base + L.workspace, L.workspace_bytes, 0,
+                                    stream);
+    if (rc) return rc;
+    // Copy out.
+    if (cudaMemcpyAsync(out_host, base + L.out, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ERR_CUDA;
+  }
+  return PKV_OK;
+}

@@ -247,3 +247,25 @@ def test_tensor_core_kernel_guards_bad_block_ids():
     rows = np.arange(2 * 64, 3 * 64)
     _, _, ref = oracle_step(w, rows=rows)
     assert_close(f64(out).reshape(-1, 128)[rows], ref, *tol_for(w), what="unaffected sequence")
+
+
+@pytest.mark.parametrize("spec", [W.PARALLEL_SAMPLING.with_(num_seqs=8, num_q_heads=8, num_kv_heads=8,
+                                                            sampling=(2, 4, 100, 1, 30)),
+                                  W.GQA_BATCH.with_(num_seqs=4, ctx=("list", (1, 100, 700, 33)))],
+                         ids=["bf16-cow", "fp8-gqa"])
+def test_host_buffer_step_matches_device_step_and_oracle(spec):
+    """pkv_decode_step_host: host inputs, one call (copies in, block copy,
+    write, decode, copy out) -- same bytes as the device-side step."""
+    w = W.make_decode_workload(spec, seed=14, device=DEV)
+    kc_d, vc_d, out_d = gpu_step(w, validate=False)
+    kc_h, vc_h = w.key_cache.clone(), w.value_cache.clone()
+    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+    out_h = pk.decode_step(pin(w.q), pin(w.new_k), pin(w.new_v), pin(w.slot_mapping), pin(w.block_tables),
+                           pin(w.context_lens), kc_h, vc_h, w.scale, copy_pairs=pin(w.copy_pairs),
+                           k_scale=w.k_scale, v_scale=w.v_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, out_d.cpu())
+    assert torch.equal(kc_h, kc_d) and torch.equal(vc_h, vc_d)
+    rk, rv, ref = oracle_step(w)
+    assert_cache_equal(kc_h, rk, "host-step key_cache")
+    assert_close(out_h.float().numpy().astype(np.float64), ref, *tol_for(w), what="host step")
