@@ -172,7 +172,7 @@ def profile_traffic(kernel_file: str, workload: str):
 def kernel_source_hash() -> str:
     d = os.path.join(ROOT, "paged_kv_cache_450_b200", "csrc")
     hsh = hashlib.sha256()
-    for name in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_launch.cuh"):
+    for name in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_mma_bf16.cuh", "decode_launch.cuh"):
         with open(os.path.join(d, name), "rb") as f:
             hsh.update(f.read())
     return hsh.hexdigest()

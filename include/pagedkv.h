@@ -139,7 +139,9 @@ int pkv_paged_kv_write(const void* k, const void* v, const int64_t* slot_mapping
  * workspace       device scratch of at least pkv_decode_workspace_bytes(...)
  *                 bytes (same arguments); not read before it is written.
  *                 Layout, with P = pkv_decode_max_partitions(...):
- *                 float ml[num_seqs][num_q_heads][P][2]  (max logit, exp-sum)
+ *                 float ml[num_seqs][num_q_heads][P][2] = (m, l): a reference
+ *                 logit m (natural units, at most the partition's max) and
+ *                 l = sum e^{s - m}, so m + ln l is the partition's log-sum-exp;
  *                 then float o[num_seqs][num_q_heads][P][head_dim] (normalised
  *                 partial outputs), starting at a 256-byte aligned offset.
  * Supported: head_dim in {64, 128}, block_size in {8, 16, 32}, query heads

@@ -67,7 +67,7 @@ static EncodeTiledFn encode_tiled() {
 // Tensor map of one cache [NB][BS][Hkv][D] seen as a 4-D tensor
 // (D, Hkv, BS, NB) innermost first; the box is one (block, kv head) tile.
 // With `swizzle128` the tile lands in shared memory with the 128-byte swizzle
-// (16-byte chunk q of row t at chunk q ^ (t % 8)); the row must be 128 bytes.
+// (16-byte chunk q of row t at chunk q ^ (t % 8)); rows must be a multiple of 128 bytes.
 static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blocks, int block_size, int num_kv_heads,
                              int head_dim, int dtype, bool swizzle128) {
   EncodeTiledFn fn = encode_tiled();
@@ -84,9 +84,12 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blo
                               static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
   const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * es;
   const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1, static_cast<cuuint32_t>(block_size), 1};
+  // Swizzled maps move one 128-byte segment of a row per box (a whole fp8
+  // row, half a bf16 row); the kernels issue one box per segment.
+  const cuuint32_t box0 = swizzle128 ? static_cast<cuuint32_t>(128 / es) : static_cast<cuuint32_t>(head_dim);
+  const cuuint32_t box[4] = {box0, 1, static_cast<cuuint32_t>(block_size), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  if (swizzle128 && row != 128) return false;
+  if (swizzle128 && (row % 128) != 0) return false;
   return fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -109,8 +112,9 @@ constexpr int kMaxPartitionTokens = 16384;
 // Resident CTAs per SM of the decode kernel that serves these arguments
 // (from the kernels' shared-memory and register budgets on B200).
 static int decode_ctas_per_sm(int cache_dtype, int head_dim, int group, int block_size) {
-  if (decode_uses_mma(cache_dtype, head_dim, group, block_size)) return 16;  // one warp, 13 KB
-  return 6;                                                                  // four warps, ~34 KB
+  if (decode_uses_mma(cache_dtype, head_dim, group, block_size))
+    return cache_dtype == PKV_DTYPE_FP8_E4M3 ? 16 : 8;  // one warp, 13 KB / 25 KB of stages
+  return 6;                                            // four warps, ~34 KB
 }
 
 // Automatic split-context partition length (see pkv_decode_partition_tokens).

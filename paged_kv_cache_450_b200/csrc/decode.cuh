@@ -41,7 +41,7 @@ struct DecodeParams {
   const void* q;                // [B][Hq][D] of TQ
   const int32_t* block_tables;  // [B][max_blocks_per_seq]
   const int32_t* context_lens;  // [B]
-  float* ws_ml;                 // [B][Hq][P][2]: max logit (natural units), exp-sum
+  float* ws_ml;                 // [B][Hq][P][2]: reference logit m (natural units), l = sum e^{s-m}
   float* ws_o;                  // [B][Hq][P][D]: normalised partial outputs
   unsigned* status;
   int num_seqs;

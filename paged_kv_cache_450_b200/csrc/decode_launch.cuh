@@ -7,6 +7,7 @@
 
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_mma_bf16.cuh"
 #include "launch.h"
 
 namespace pkv {
@@ -37,6 +38,19 @@ static cudaError_t launch_mma(const CUtensorMap& kmap, const CUtensorMap& vmap, 
   return launch_pdl(kern, grid, dim3(32), smem, st, kmap, vmap, p);
 }
 
+template <int BS, int G>
+static cudaError_t launch_mma_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                                   int num_kv_heads, cudaStream_t st) {
+  using T = MmaBf16Traits<BS>;
+  auto kern = paged_decode_mma_bf16_kernel<BS, G>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  dim3 grid(num_kv_heads, p.max_partitions, p.num_seqs);
+  return launch_pdl(kern, grid, dim3(32), smem, st, kmap, vmap, p);
+}
+
 template <typename TQ, int D>
 static cudaError_t launch_reduce(const DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_q_heads;
@@ -50,6 +64,17 @@ static cudaError_t dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vm
   if constexpr (std::is_same_v<TC, __nv_fp8_e4m3> && D == 128 && (BS == 16 || BS == 32)) {
     if (group == 8) return launch_mma<TQ, BS>(kmap, vmap, p, num_kv_heads, st);
   }
+  if constexpr (std::is_same_v<TC, __nv_bfloat16> && std::is_same_v<TQ, __nv_bfloat16> && D == 128 &&
+                (BS == 16 || BS == 32)) {
+    switch (group) {
+      case 1: break;  // MHA: CUDA-core kernel below
+      case 2: return launch_mma_bf16<BS, 2>(kmap, vmap, p, num_kv_heads, st);
+      case 4: return launch_mma_bf16<BS, 4>(kmap, vmap, p, num_kv_heads, st);
+      case 8: return launch_mma_bf16<BS, 8>(kmap, vmap, p, num_kv_heads, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  // (decode_uses_mma() in launch.h makes the same choice for the tensor maps.)
   switch (group) {
     case 1: return launch_partition<TQ, TC, D, BS, 1>(kmap, vmap, p, num_kv_heads, st);
     case 2: return launch_partition<TQ, TC, D, BS, 2>(kmap, vmap, p, num_kv_heads, st);

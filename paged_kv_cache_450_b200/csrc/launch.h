@@ -57,12 +57,18 @@ cudaError_t launch_kv_write(const KvWriteArgs& a, cudaStream_t st);
 cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, void* kc, void* vc, int64_t num_blocks,
                               int64_t block_bytes, unsigned* status, cudaStream_t st);
 
-// The tensor-core decode kernel serves fp8 caches with head_dim 128, 8 query
-// heads per KV head and 16- or 32-token blocks; its cache tensor maps use the
-// 128-byte swizzle.  Everything else runs on the CUDA-core kernel.
+// The tensor-core decode kernels serve head_dim 128 with 16- or 32-token
+// blocks: fp8 caches with 8 query heads per KV head, and bf16 caches with 2,
+// 4 or 8 (grouped-query attention, where CUDA-core work grows with the
+// group).  Their cache tensor maps use the 128-byte swizzle (boxes of one
+// 128-byte row segment).  Everything else -- MHA included, which is at the
+// memory limit on CUDA cores and measured slightly faster there (more warps
+// per SM keep more loads in flight) -- runs on the CUDA-core kernel.
 inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_size) {
-  return cache_dtype == 2 /* PKV_DTYPE_FP8_E4M3 */ && head_dim == 128 && group == 8 &&
-         (block_size == 16 || block_size == 32);
+  if (head_dim != 128 || (block_size != 16 && block_size != 32)) return false;
+  if (cache_dtype == 2 /* PKV_DTYPE_FP8_E4M3 */) return group == 8;
+  if (cache_dtype == 1 /* PKV_DTYPE_BF16 */) return group == 2 || group == 4 || group == 8;
+  return false;
 }
 
 // Decode launchers, one per (q dtype, cache dtype); each dispatches on

@@ -78,9 +78,12 @@ GQA_LONG = DecodeSpec("gqa70b_fp8_b16_ctx32k", 16, 64, 8, 128, 16, torch.bfloat1
 GQA_BATCH = DecodeSpec("gqa70b_fp8_b128_ctx8k", 128, 64, 8, 128, 16, torch.bfloat16, FP8,
                        ("fixed", 8192), ("slack", 1.0))
 
+# Extra (not one of the five families): the 70B-GQA shape with a bf16 cache.
+GQA_BATCH_BF16 = GQA_BATCH.with_(name="gqa70b_bf16_b128_ctx8k", cache_dtype=torch.bfloat16)
+
 SPECS = {s.name: s for s in (TINY, LLAMA7B, LLAMA13B, LLAMA13B.with_(name="llama13b_decode_b256_bf16_bs32",
                                                                       block_size=32),
-                             PARALLEL_SAMPLING, GQA_LONG, GQA_BATCH)}
+                             PARALLEL_SAMPLING, GQA_LONG, GQA_BATCH, GQA_BATCH_BF16)}
 
 
 @dataclass
