@@ -182,6 +182,17 @@ def kernel_source_hash() -> str:
 # the GPU arm
 # --------------------------------------------------------------------------- #
 
+def kernel_name(spec) -> str:
+    """The decode partition kernel that serves this workload (mirrors the library's dispatch)."""
+    g = spec.num_q_heads // spec.num_kv_heads
+    if spec.head_dim == 128 and spec.block_size in (16, 32):
+        if spec.cache_dtype == torch.float8_e4m3fn and g == 8:
+            return "paged_decode_gqa8_fp8_mma_kernel"
+        if spec.cache_dtype == torch.bfloat16 and g in (2, 4, 8):
+            return "paged_decode_mma_bf16_kernel"
+    return "paged_decode_partition_kernel"
+
+
 def step_inputs_bytes(w) -> tuple[int, int]:
     """Bytes of one step's per-step inputs (host -> device) and result (device -> host)."""
     ts = [w.q, w.new_k, w.new_v, w.slot_mapping, w.block_tables, w.context_lens, w.copy_pairs]
@@ -208,17 +219,26 @@ def run_gpu(args, rank, world, local_rank):
     kc, vc = w.key_cache, w.value_cache
     stream = torch.cuda.current_stream(dev)
 
+    fused = w.new_k is not None and not args.unfused
+
     def step(ev_mid=None, ev_end=None):
         if w.copy_pairs is not None and len(w.copy_pairs):
             pk.kv_block_copy(w.copy_pairs, kc, vc, stream=stream)
-        if w.new_k is not None:
-            pk.paged_kv_write(w.new_k, w.new_v, w.slot_mapping, kc, vc, k_scale=w.k_scale, v_scale=w.v_scale,
-                              stream=stream)
-        if ev_mid is not None:
-            ev_mid.record(stream)
-        pk.paged_attention_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, k_scale=w.k_scale,
-                                  v_scale=w.v_scale, out=out, workspace=workspace, partition_tokens=pt,
+        if fused:  # the new token (one per sequence, at ctx - 1) is written inside the decode launch
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, w.block_tables, w.context_lens, w.scale,
+                                   k_scale=w.k_scale, v_scale=w.v_scale, out=out, workspace=workspace,
+                                   partition_tokens=pt, stream=stream)
+        else:
+            if w.new_k is not None:
+                pk.paged_kv_write(w.new_k, w.new_v, w.slot_mapping, kc, vc, k_scale=w.k_scale, v_scale=w.v_scale,
                                   stream=stream)
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            pk.paged_attention_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, k_scale=w.k_scale,
+                                      v_scale=w.v_scale, out=out, workspace=workspace, partition_tokens=pt,
+                                      stream=stream)
         if ev_end is not None:
             ev_end.record(stream)
 
@@ -304,13 +324,14 @@ def run_gpu(args, rank, world, local_rank):
                        "context_lens": list(s.ctx), "pool": list(s.pool),
                        "kv_bytes_per_step_per_gpu": kv_bytes, "partition_tokens": pt,
                        "new_tokens_per_step": 0 if w.new_k is None else int(w.new_k.shape[0]),
+                       "new_token_write": "fused into the decode launch" if fused else "separate launch",
                        "cow_pairs_per_step": 0 if w.copy_pairs is None else int(len(w.copy_pairs)),
                        "l2": "inputs larger than L2 (KV stream per step > 126 MB); no flush",
                        "parallelism": f"dp{world} (independent batch per GPU, no collective)"},
             "pct_of_hbm_peak": {"measured_copy": round(100 * value / peak, 2) if peak_kind == "measured" else None,
                                 "spec_8tbs": round(100 * value / SPEC_HBM_GBS, 2)},
             "tokens_per_s_per_layer": round(total_seqs / (step_ms * 1e-3), 1),
-            "roofline": {"kernel": "paged_decode_partition_kernel + paged_decode_reduce_kernel",
+            "roofline": {"kernel": kernel_name(s) + " + paged_decode_reduce_kernel",
                          "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "peak_kind": f"{peak_kind} (burst copy bandwidth)", "frac": round(achieved / peak, 4),
                          "algorithmic_bytes_per_launch": kv_bytes, "decode_ms": round(decode_ms, 5),
@@ -462,6 +483,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=1000)
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="write the new tokens with a separate paged_kv_write launch instead of inside the decode")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch (a smaller case of the same shape, for profiling)")
     return ap.parse_args(argv)

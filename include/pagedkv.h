@@ -158,6 +158,31 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
                                void* workspace, size_t workspace_bytes, int validate, void* stream);
 
 /*
+ * Decode step with the new-token write fused in: append, then attend.
+ *
+ * Source: "vLLM 与 KV Cache", KV Cache：为什么需要缓存 -- each decode step
+ * computes the new token's K,V, appends them to the cache and attends over
+ * all cached tokens.  For every sequence b with context_lens[b] >= 1, the
+ * new token k_new[b] / v_new[b] is written to logical position
+ * context_lens[b] - 1, i.e. row (ctx-1) % block_size of physical block
+ * block_tables[b][(ctx-1) / block_size] (that block must be allocated), with
+ * the same bytes pkv_paged_kv_write would store for that slot; then the
+ * result equals pkv_paged_attention_decode's.  One kernel launch (plus the
+ * split-context merge) instead of two: the CTA that reads the sequence's last
+ * block writes its KV head's slice of the new token first.
+ *
+ * k_new, v_new   device [num_seqs][num_kv_heads][head_dim] of q_dtype, 16-byte aligned.
+ * Other arguments and errors: as pkv_paged_attention_decode (key_cache and
+ * value_cache are written).
+ */
+int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const void* v_new, void* key_cache,
+                            void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale, float v_scale,
+                            int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                            size_t workspace_bytes, int validate, void* stream);
+
+/*
  * Paged decode attention that allocates nothing and takes no workspace.
  *
  * The PagedAttention pages have no counterpart of this call; it is a

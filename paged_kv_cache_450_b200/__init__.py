@@ -30,7 +30,7 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "kv_block_copy", "decode_step", "decode_step_staging_bytes",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
            "library_path"]
@@ -166,6 +166,38 @@ def paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens
             context_lens.data_ptr(), B, Hq, Hkv, d, bs, MB, NB, float(scale), float(k_scale), float(v_scale),
             _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr, ws_bytes, int(validate),
             _stream(dev, stream)), "paged_attention_decode")
+    return out
+
+
+def paged_decode_append(q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale: float, *,
+                        k_scale: float = 1.0, v_scale: float = 1.0, out=None, workspace=None,
+                        partition_tokens: int = 0, validate: bool = False, stream=None):
+    """Append each sequence's new token (k_new/v_new [B, Hkv, d], q's dtype) at
+    logical position context_lens[b] - 1, then run decode attention -- one
+    fused launch.  Returns out [B, Hq, d]."""
+    dev = _cuda(q, k_new, v_new, key_cache, value_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, Hq, d = q.shape
+    NB, bs, Hkv, d2 = key_cache.shape
+    if k_new.shape != (B, Hkv, d) or v_new.shape != k_new.shape or k_new.dtype != q.dtype or d2 != d:
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] in q's dtype")
+    if value_cache.shape != key_cache.shape or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    MB = block_tables.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, MB, key_cache.dtype, partition_tokens) if B else 0
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_paged_decode_append(
+            out.data_ptr(), q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), key_cache.data_ptr(),
+            value_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(), B, Hq, Hkv, d, bs, MB, NB,
+            float(scale), float(k_scale), float(v_scale), _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr,
+            ws_bytes, int(validate), _stream(dev, stream)), "paged_decode_append")
     return out
 
 

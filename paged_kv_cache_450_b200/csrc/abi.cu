@@ -250,16 +250,22 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_head
   return align256(rows * 2 * sizeof(float)) + rows * head_dim * sizeof(float);
 }
 
-int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
-                               const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
-                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                               int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
-                               float v_scale, int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
-                               size_t workspace_bytes, int validate, void* stream) {
+}  // extern "C"
+
+// Decode, optionally with the fused append of one new token per sequence
+// (k_new / v_new non-NULL).
+static int decode_impl(void* out, const void* q, const void* k_new, const void* v_new, const void* key_cache,
+                       const void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                       int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale, float v_scale,
+                       int q_dtype, int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                       int validate, void* stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
     return PKV_ERR_BAD_SHAPE;
   if (num_seqs == 0) return PKV_OK;
   if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_ERR_NULL_POINTER;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PKV_ERR_NULL_POINTER;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PKV_ERR_MISALIGNED;
   if (q_dtype != PKV_DTYPE_F32 && q_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
   if (cache_dtype != q_dtype && cache_dtype != PKV_DTYPE_FP8_E4M3) return PKV_ERR_BAD_DTYPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_HEAD_DIM;
@@ -327,6 +333,12 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
   const bool fp8 = cache_dtype == PKV_DTYPE_FP8_E4M3;
   p.q_scale = scale * kLog2e * (fp8 ? k_scale : 1.0f);
   p.out_scale = fp8 ? v_scale : 1.0f;
+  p.new_k = k_new;
+  p.new_v = v_new;
+  p.key_cache = const_cast<void*>(key_cache);
+  p.value_cache = const_cast<void*>(value_cache);
+  p.k_inv = fp8 ? 1.0f / k_scale : 1.0f;  // rounded once to fp32 on the host, as for pkv_paged_kv_write
+  p.v_inv = fp8 ? 1.0f / v_scale : 1.0f;
   const bool reduce = P > 1;
 
   cudaError_t e;
@@ -339,6 +351,32 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, 
   else
     e = launch_decode_bf16_fp8(kmap, vmap, p, head_dim, group, num_kv_heads, reduce, st);
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+extern "C" {
+
+int pkv_paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                               float v_scale, int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                               size_t workspace_bytes, int validate, void* stream) {
+  return decode_impl(out, q, nullptr, nullptr, key_cache, value_cache, block_tables, context_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale,
+                     v_scale, q_dtype, cache_dtype, partition_tokens, workspace, workspace_bytes, validate, stream);
+}
+
+int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const void* v_new, void* key_cache,
+                            void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale, float v_scale,
+                            int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                            size_t workspace_bytes, int validate, void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return PKV_ERR_NULL_POINTER;
+  if (cache_dtype == PKV_DTYPE_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_BAD_SHAPE;
+  return decode_impl(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale,
+                     v_scale, q_dtype, cache_dtype, partition_tokens, workspace, workspace_bytes, validate, stream);
 }
 
 int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key_cache, void* value_cache,

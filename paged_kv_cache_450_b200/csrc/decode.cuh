@@ -54,7 +54,65 @@ struct DecodeParams {
   int max_partitions;
   float q_scale;    // scale * log2(e) * (fp8 ? k_scale : 1)
   float out_scale;  // fp8 ? v_scale : 1
+  // Fused append (pkv_paged_decode_append): new_k/new_v [B][Hkv][D] in q's
+  // dtype, written to logical position context_lens[b] - 1 before it is read.
+  // NULL for plain decode.
+  const void* new_k;
+  const void* new_v;
+  void* key_cache;
+  void* value_cache;
+  float k_inv;  // fp8 caches: 1/k_scale and 1/v_scale rounded to fp32
+  float v_inv;
 };
+
+// Fused append: the CTA that reads the last block of sequence b writes that
+// sequence's new token for its kv head (row (ctx-1) % BS of physical block
+// block_tables[b][(ctx-1) / BS]) -- a copy, or for fp8 one fp32 multiply and
+// a round-to-nearest saturating E4M3 encode, exactly as paged_kv_write_kernel
+// -- and fences the generic writes against the TMA reads that follow.  An id
+// outside the pool writes nothing (the partition pass reports it).
+template <typename TQ, typename TC, int D, int BS>
+__device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int hk, int ctx, int tid,
+                                                 int nthreads) {
+  const int t = ctx - 1;
+  const int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + t / BS];
+  if (id < 0 || id >= p.num_blocks) return;
+  const int64_t dst = ((static_cast<int64_t>(id) * BS + t % BS) * p.num_kv_heads + hk) * D;
+  const int64_t src = (static_cast<int64_t>(b) * p.num_kv_heads + hk) * D;
+  const TQ* kin = static_cast<const TQ*>(p.new_k) + src;
+  const TQ* vin = static_cast<const TQ*>(p.new_v) + src;
+  for (int c8 = tid; c8 < D / 8; c8 += nthreads) {
+    if constexpr (sizeof(TQ) == sizeof(TC)) {
+      constexpr int kVec = 8 * sizeof(TQ) / 16;
+      const uint4* ks = reinterpret_cast<const uint4*>(kin + 8 * c8);
+      const uint4* vs = reinterpret_cast<const uint4*>(vin + 8 * c8);
+      uint4* kd = reinterpret_cast<uint4*>(static_cast<TC*>(p.key_cache) + dst + 8 * c8);
+      uint4* vd = reinterpret_cast<uint4*>(static_cast<TC*>(p.value_cache) + dst + 8 * c8);
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+      }
+    } else {
+      uint8_t kb[8], vb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        kb[e] = __nv_cvt_float_to_fp8(__fmul_rn(Elem<TQ>::to_float(kin[8 * c8 + e]), p.k_inv), __NV_SATFINITE,
+                                      __NV_E4M3);
+        vb[e] = __nv_cvt_float_to_fp8(__fmul_rn(Elem<TQ>::to_float(vin[8 * c8 + e]), p.v_inv), __NV_SATFINITE,
+                                      __NV_E4M3);
+      }
+      uint2 kw, vw;
+      kw.x = kb[0] | (kb[1] << 8) | (kb[2] << 16) | (uint32_t(kb[3]) << 24);
+      kw.y = kb[4] | (kb[5] << 8) | (kb[6] << 16) | (uint32_t(kb[7]) << 24);
+      vw.x = vb[0] | (vb[1] << 8) | (vb[2] << 16) | (uint32_t(vb[3]) << 24);
+      vw.y = vb[4] | (vb[5] << 8) | (vb[6] << 16) | (uint32_t(vb[7]) << 24);
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.key_cache) + dst + 8 * c8) = kw;
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.value_cache) + dst + 8 * c8) = vw;
+    }
+  }
+  fence_proxy_async_global();
+}
 
 // NW warps per CTA, each with a private pipeline of NS stages (0: about 8 KB of
 // stages per warp).  Small CTAs win: with ~34 KB of shared memory per CTA six
@@ -200,12 +258,15 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   // q of the G heads, pre-scaled into the base-2 logit domain.
   for (int i = threadIdx.x; i < G * D; i += blockDim.x)
     q_s[i] = Elem<TQ>::to_float(static_cast<const TQ*>(p.q)[out_row0 * D + i]) * p.q_scale;
+  const bool append = p.new_k != nullptr && part == nparts - 1;
+  if (append) append_new_token<TQ, TC, D, BS>(p, b, hk, ctx, threadIdx.x, blockDim.x);
   const uint32_t bar0 = smem_u32(bars) + warp * T::NS * 8;
   if (lane == 0) {
     for (int s = 0; s < T::NS; ++s) mbar_init(bar0 + 8 * s, 1);
     fence_barrier_init();
   }
   __syncthreads();
+  if (append && lane == 0) fence_proxy_async_global();
 
   const int n_w = nb > warp ? (nb - warp + T::NW - 1) / T::NW : 0;  // blocks of this warp
   const uint32_t stage0 = smem_u32(data) + warp * T::NS * T::STAGE_BYTES;

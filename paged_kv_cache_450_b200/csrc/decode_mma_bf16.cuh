@@ -121,10 +121,13 @@ __global__ void __launch_bounds__(32, MINB)
     }
     ids[i] = id;
   }
+  const bool append = p.new_k != nullptr && part == nparts - 1;
+  if (append) append_new_token<__nv_bfloat16, __nv_bfloat16, D, BS>(p, b, hk, ctx, lane, 32);
   const uint32_t bar0 = smem_u32(bars);
   if (lane == 0) {
     for (int s = 0; s < T::NS; ++s) mbar_init(bar0 + 8 * s, 1);
     fence_barrier_init();
+    if (append) fence_proxy_async_global();
   }
   __syncwarp();
 

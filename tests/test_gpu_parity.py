@@ -278,3 +278,33 @@ def test_host_buffer_step_matches_device_step_and_oracle(spec):
 def test_full_size_bf16_gqa_sampled():
     w = W.make_decode_workload(W.SPECS["gqa70b_bf16_b128_ctx8k"], seed=0, device=DEV)
     check_step(w, rows=sample_rows(w, 512), what="gqa70b_bf16_b128_ctx8k")
+
+
+APPEND_SPECS = [W.TINY, W.LLAMA7B.with_(num_seqs=6, num_q_heads=4, num_kv_heads=4, ctx=("list", (1, 16, 17, 700, 513, 0))),
+                W.LLAMA7B.with_(num_seqs=4, num_q_heads=16, num_kv_heads=2, ctx=("list", (1, 33, 300, 64))),
+                W.GQA_BATCH.with_(num_seqs=4, ctx=("list", (1, 100, 700, 33))),
+                W.GQA_BATCH.with_(num_seqs=3, num_q_heads=16, num_kv_heads=4, ctx=("list", (5, 48, 200))),
+                W.GQA_BATCH.with_(num_seqs=3, block_size=32, ctx=("list", (5, 33, 300)))]
+
+
+@pytest.mark.parametrize("spec", APPEND_SPECS, ids=["fp32-mha", "bf16-mha", "bf16-gqa8-mma", "fp8-gqa8-mma",
+                                                     "fp8-gqa4-cudacore", "fp8-gqa8-mma-bs32"])
+def test_fused_append_equals_write_then_decode(spec):
+    """pkv_paged_decode_append writes the same cache bytes as the separate
+    write at slot (ctx-1) and gives the same attention output (bit-identical:
+    the same kernels compute it), which the oracle confirms."""
+    w = W.make_decode_workload(spec, seed=15, device=DEV)
+    kc_ref, vc_ref, out_ref = gpu_step(w, partition_tokens=2 * spec.block_size)
+    kc, vc = w.key_cache.clone(), w.value_cache.clone()
+    # sequences with an empty context have no position to write: their k_new row is ignored
+    out = pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, w.block_tables, w.context_lens, w.scale,
+                                 k_scale=w.k_scale, v_scale=w.v_scale, partition_tokens=2 * spec.block_size,
+                                 validate=True)
+    torch.cuda.synchronize()
+    assert torch.equal(kc.view(torch.uint8), kc_ref.view(torch.uint8))
+    assert torch.equal(vc.view(torch.uint8), vc_ref.view(torch.uint8))
+    assert torch.equal(out, out_ref)
+    rk, rv, ref = oracle_step(w)
+    assert_cache_equal(kc, rk, "append key_cache")
+    assert_close(f64(out), ref, *tol_for(w), what="fused append")
+    assert pk.device_status(clear=True) == 0
