@@ -270,6 +270,48 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
                       int64_t num_blocks, int64_t block_bytes, int validate, void* stream);
 
 /*
+ * Per-tensor fp8 scale on the device: *scale = amax(|x|) / 448 (one fp32
+ * division; 1.0 when x is all zeros), the scale that maps the largest
+ * magnitude onto the largest finite E4M3 value.
+ *
+ * Source: the "--kv-cache-dtype fp8" option of "vLLM KV Cache 实现机制", 2.3;
+ * the pages give no calibration rule -- amax / 448 per tensor is this
+ * library's reading.  Pass the value as k_scale / v_scale of the other calls
+ * (copy it to the host first).
+ *
+ * x       device, n elements of dtype (F32 or BF16), 16-byte aligned.
+ * scale   device float, written on `stream` (its previous content is ignored).
+ * NaN elements are ignored (fmax semantics).  Errors: PKV_ERR_NULL_POINTER, _BAD_DTYPE,
+ * _BAD_SHAPE, _MISALIGNED, _CUDA.
+ */
+int pkv_fp8_scale_from_amax(const void* x, int64_t n, int dtype, float* scale, void* stream);
+
+/*
+ * Block swap between two pools (device <-> pinned host, or any two pools).
+ *
+ * Source: "vLLM KV Cache 实现机制", 1.2 (blocks migrate between GPU memory and
+ * CPU RAM block by block when GPU memory runs short) and 2.1 (CPU offloading
+ * tier); "vLLM — 把操作系统的分页搬进 GPU KV cache", 实践案例 3 (SWAP: copy the
+ * blocks to CPU memory and back when needed).
+ * Each (src, dst) pair of src_dst_pairs copies block src of the source pool
+ * (src_key / src_value) onto block dst of the destination pool (dst_key /
+ * dst_value), byte for byte, in ONE kernel launch for all pairs.  Either pool
+ * may live in page-locked host memory allocated with cudaHostAlloc /
+ * cudaMallocHost (or registered with cudaHostRegister): the kernel reads or
+ * writes it directly through unified addressing.  Pageable host memory is not
+ * supported.  Both pools use the cache layout above with the same block_bytes.
+ *
+ * src_dst_pairs   device int64 [num_pairs][2] (src block id, dst block id).
+ *                 Destinations must be distinct (and, within one pool, never a
+ *                 source); validate checks this.
+ * Errors: PKV_ERR_NULL_POINTER, _BAD_SHAPE, _MISALIGNED, _OUT_OF_RANGE /
+ * _BAD_COPY_PAIRS (validate), _CUDA.  num_pairs == 0 launches nothing.
+ */
+int pkv_swap_blocks(const int64_t* src_dst_pairs, int64_t num_pairs, const void* src_key, const void* src_value,
+                    int64_t src_num_blocks, void* dst_key, void* dst_value, int64_t dst_num_blocks,
+                    int64_t block_bytes, int validate, void* stream);
+
+/*
  * One whole decode step with the per-step inputs and the output in HOST memory.
  *
  * Source: the decode step of "vLLM 与 KV Cache", KV Cache：为什么需要缓存 (append

@@ -74,6 +74,10 @@ def _load():
     lib.orc_paged_kv_write.restype = I
     lib.orc_kv_block_copy.argtypes = [P, I64, P, P, I64, I64]
     lib.orc_kv_block_copy.restype = I
+    lib.orc_swap_blocks.argtypes = [P, I64, P, P, I64, P, P, I64, I64]
+    lib.orc_swap_blocks.restype = I
+    lib.orc_fp8_scale.argtypes = [P, I64, I]
+    lib.orc_fp8_scale.restype = F
     lib.orc_e4m3_encode_array.argtypes = [P, P, I64]
     lib.orc_e4m3_encode_array.restype = None
     _lib = lib
@@ -222,3 +226,22 @@ def kv_block_copy(pairs, key_cache, value_cache):
     rc = lib.orc_kv_block_copy(_ptr(pairs), pairs.shape[0], _ptr(key_cache), _ptr(value_cache), NB,
                                block_bytes)
     _check(rc, "kv_block_copy")
+
+
+def swap_blocks(pairs, src_key, src_value, dst_key, dst_value):
+    """Copy block src of the source pool onto block dst of the destination pool IN PLACE."""
+    lib = _load()
+    pairs = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
+    for a in (src_key, src_value, dst_key, dst_value):
+        assert a.flags["C_CONTIGUOUS"]
+    assert src_key.shape[1:] == dst_key.shape[1:] and src_key.dtype == dst_key.dtype
+    block_bytes = src_key[0].nbytes if src_key.shape[0] else 1
+    rc = lib.orc_swap_blocks(_ptr(pairs), pairs.shape[0], _ptr(src_key), _ptr(src_value), src_key.shape[0],
+                             _ptr(dst_key), _ptr(dst_value), dst_key.shape[0], block_bytes)
+    _check(rc, "swap_blocks")
+
+
+def fp8_scale(x, dtype=None) -> float:
+    """amax(|x|) / 448 as an fp32 value (1.0 for all zeros)."""
+    x = np.ascontiguousarray(x)
+    return float(np.float32(_load().orc_fp8_scale(_ptr(x), x.size, _dtype_code(x, dtype))))

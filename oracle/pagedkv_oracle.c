@@ -432,3 +432,47 @@ int orc_kv_block_copy(const int64_t* pairs, int64_t num_pairs, void* key_cache, 
 void orc_e4m3_encode_array(const float* x, uint8_t* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_float(x[i]);
 }
+
+/* ---------- block swap between two pools ------------------------------------ */
+
+/*
+ * Block swap ("vLLM KV Cache 实现机制", 1.2 and 2.1; "vLLM — 把操作系统的分页搬进
+ * GPU KV cache", 实践案例 3): block src of the source pool is copied onto block
+ * dst of the destination pool, in both caches, byte for byte.  Destinations
+ * must be distinct and in range (sources in range); otherwise nothing is
+ * written and ORC_ERANGE / ORC_EINVAL is returned.
+ */
+int orc_swap_blocks(const int64_t* pairs, int64_t num_pairs, const void* src_k, const void* src_v,
+                    int64_t src_blocks, void* dst_k, void* dst_v, int64_t dst_blocks, int64_t block_bytes) {
+  if (num_pairs < 0 || src_blocks < 0 || dst_blocks < 0 || block_bytes <= 0) return ORC_EINVAL;
+  for (int64_t i = 0; i < num_pairs; ++i) {
+    int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) return ORC_ERANGE;
+    for (int64_t j = 0; j < i; ++j)
+      if (pairs[2 * j + 1] == d) return ORC_EINVAL;
+  }
+  for (int64_t i = 0; i < num_pairs; ++i) {
+    int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    memcpy((char*)dst_k + d * block_bytes, (const char*)src_k + s * block_bytes, (size_t)block_bytes);
+    memcpy((char*)dst_v + d * block_bytes, (const char*)src_v + s * block_bytes, (size_t)block_bytes);
+  }
+  return ORC_OK;
+}
+
+/* ---------- per-tensor fp8 scale ---------------------------------------------- */
+
+/* amax(|x|) over n elements (exact in fp64), then amax / 448 as one binary32
+ * division (the largest finite E4M3 value is 448); 1 when amax is 0.  The
+ * calibration rule is this library's reading: the pages name fp8 KV caches
+ * ("vLLM KV Cache 实现机制", 2.3) without one. */
+float orc_fp8_scale(const void* x, int64_t n, int dtype) {
+  double amax = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    double a = fabs(load_elem(x, i, dtype, 1.0));
+    if (a > amax) amax = a;
+  }
+  if (!(amax > 0.0)) return 1.0f;
+  volatile float af = (float)amax; /* exact: amax is one of the inputs */
+  volatile float s = af / 448.0f;
+  return s;
+}

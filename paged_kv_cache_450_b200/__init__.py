@@ -30,7 +30,7 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "decode_step", "decode_step_staging_bytes",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
            "library_path"]
@@ -216,6 +216,46 @@ def kv_block_copy(src_dst_pairs, key_cache, value_cache, *, validate: bool = Fal
         _check(lib.pkv_kv_block_copy(src_dst_pairs.data_ptr(), src_dst_pairs.shape[0], key_cache.data_ptr(),
                                      value_cache.data_ptr(), NB, block_bytes, int(validate),
                                      _stream(dev, stream)), "kv_block_copy")
+
+
+def fp8_scale_from_amax(x, *, out=None, stream=None):
+    """Per-tensor fp8 scale amax(|x|) / 448 computed on the device (float32
+    tensor of one element; 1.0 for an all-zero x)."""
+    dev = _cuda(x)
+    if out is None:
+        out = torch.empty((1,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_fp8_scale_from_amax(x.data_ptr(), x.numel(), _dtype(x), out.data_ptr(),
+                                                   _stream(dev, stream)), "fp8_scale_from_amax")
+    return out
+
+
+def swap_blocks(src_dst_pairs, src_key, src_value, dst_key, dst_value, *, validate: bool = False, stream=None):
+    """Copy block src of (src_key, src_value) onto block dst of (dst_key,
+    dst_value) for every row of src_dst_pairs (int64 [n, 2], on the device), in
+    one kernel launch.  Either pool may be pinned host memory (a CPU tensor
+    from pin_memory()); the other must be on the device."""
+    pools = (src_key, src_value, dst_key, dst_value)
+    devs = [t for t in pools if t.device.type == "cuda"]
+    if not devs:
+        raise ValueError("at least one pool must be on the device")
+    for t in pools:
+        if t.device.type == "cpu" and not t.is_pinned():
+            raise ValueError("host pools must be page-locked (pin_memory())")
+        if not t.is_contiguous():
+            raise ValueError("pools must be contiguous")
+    dev = _cuda(src_dst_pairs, *devs)
+    if src_dst_pairs.dtype != torch.int64 or src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be int64 [n, 2]")
+    if src_key.shape[1:] != dst_key.shape[1:] or src_key.dtype != dst_key.dtype or \
+            src_value.shape != src_key.shape or dst_value.shape != dst_key.shape:
+        raise ValueError("pools must share the block shape and dtype")
+    block_bytes = src_key[0].numel() * src_key.element_size()
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_swap_blocks(src_dst_pairs.data_ptr(), src_dst_pairs.shape[0], src_key.data_ptr(),
+                                           src_value.data_ptr(), src_key.shape[0], dst_key.data_ptr(),
+                                           dst_value.data_ptr(), dst_key.shape[0], block_bytes, int(validate),
+                                           _stream(dev, stream)), "swap_blocks")
 
 
 def device_status(clear: bool = True, device=None, stream=None) -> int:

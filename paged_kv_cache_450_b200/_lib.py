@@ -31,6 +31,8 @@ SIGNATURES = {
     "pkv_decode_max_partitions": (I, [I, I, I, I, I, I, I, I]),
     "pkv_decode_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),
     "pkv_kv_block_copy": (I, [P, I64, P, P, I64, I64, I, P]),
+    "pkv_fp8_scale_from_amax": (I, [P, I64, I, P, P]),
+    "pkv_swap_blocks": (I, [P, I64, P, P, I64, P, P, I64, I64, I, P]),
     "pkv_device_status": (I, [ctypes.POINTER(ctypes.c_uint), I, P]),
     "pkv_launch_count": (U64, []),
 }

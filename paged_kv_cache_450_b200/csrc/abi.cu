@@ -379,6 +379,29 @@ int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const v
                      v_scale, q_dtype, cache_dtype, partition_tokens, workspace, workspace_bytes, validate, stream);
 }
 
+// Host-side check of copy pairs (validate): ids in range; destinations distinct
+// and, when both sides are one pool, never also a source.
+static int check_pairs(const int64_t* pairs, int64_t num_pairs, int64_t src_blocks, int64_t dst_blocks, bool same_pool,
+                       cudaStream_t st) {
+  std::vector<int64_t> h;
+  if (!copy_to_host(h, pairs, static_cast<size_t>(num_pairs) * 2, st)) return PKV_ERR_CUDA;
+  std::vector<int64_t> dsts, srcs;
+  for (int64_t i = 0; i < num_pairs; ++i) {
+    const int64_t s = h[2 * i], d = h[2 * i + 1];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) return PKV_ERR_OUT_OF_RANGE;
+    srcs.push_back(s);
+    dsts.push_back(d);
+  }
+  std::sort(dsts.begin(), dsts.end());
+  std::sort(srcs.begin(), srcs.end());
+  for (size_t i = 1; i < dsts.size(); ++i)
+    if (dsts[i] == dsts[i - 1]) return PKV_ERR_BAD_COPY_PAIRS;
+  if (same_pool)
+    for (int64_t d : dsts)
+      if (std::binary_search(srcs.begin(), srcs.end(), d)) return PKV_ERR_BAD_COPY_PAIRS;
+  return PKV_OK;
+}
+
 int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key_cache, void* value_cache,
                       int64_t num_blocks, int64_t block_bytes, int validate, void* stream) {
   if (num_pairs < 0 || num_blocks <= 0 || block_bytes <= 0 || block_bytes % 16 != 0) return PKV_ERR_BAD_SHAPE;
@@ -387,26 +410,45 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
   if (!aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (validate) {
-    std::vector<int64_t> h;
-    if (!copy_to_host(h, src_dst_pairs, static_cast<size_t>(num_pairs) * 2, st)) return PKV_ERR_CUDA;
-    std::vector<int64_t> dsts, srcs;
-    for (int64_t i = 0; i < num_pairs; ++i) {
-      const int64_t s = h[2 * i], d = h[2 * i + 1];
-      if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PKV_ERR_OUT_OF_RANGE;
-      srcs.push_back(s);
-      dsts.push_back(d);
-    }
-    std::sort(dsts.begin(), dsts.end());
-    std::sort(srcs.begin(), srcs.end());
-    for (size_t i = 1; i < dsts.size(); ++i)
-      if (dsts[i] == dsts[i - 1]) return PKV_ERR_BAD_COPY_PAIRS;
-    for (int64_t d : dsts)
-      if (std::binary_search(srcs.begin(), srcs.end(), d)) return PKV_ERR_BAD_COPY_PAIRS;
+    const int rc = check_pairs(src_dst_pairs, num_pairs, num_blocks, num_blocks, true, st);
+    if (rc) return rc;
   }
   unsigned* status = status_word();
   if (!status) return PKV_ERR_CUDA;
-  return launch_block_copy(src_dst_pairs, num_pairs, key_cache, value_cache, num_blocks, block_bytes, status, st) ==
-                 cudaSuccess
+  return launch_block_copy(src_dst_pairs, num_pairs, key_cache, value_cache, num_blocks, key_cache, value_cache,
+                           num_blocks, block_bytes, status, st) == cudaSuccess
+             ? PKV_OK
+             : PKV_ERR_CUDA;
+}
+
+int pkv_fp8_scale_from_amax(const void* x, int64_t n, int dtype, float* scale, void* stream) {
+  if (n < 0) return PKV_ERR_BAD_SHAPE;
+  if (!x || !scale) return PKV_ERR_NULL_POINTER;
+  if (dtype != PKV_DTYPE_F32 && dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0) return PKV_ERR_MISALIGNED;
+  return launch_fp8_scale(x, n, dtype, scale, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK
+                                                                                                  : PKV_ERR_CUDA;
+}
+
+int pkv_swap_blocks(const int64_t* src_dst_pairs, int64_t num_pairs, const void* src_key, const void* src_value,
+                    int64_t src_num_blocks, void* dst_key, void* dst_value, int64_t dst_num_blocks,
+                    int64_t block_bytes, int validate, void* stream) {
+  if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 || block_bytes <= 0 || block_bytes % 16 != 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_pairs == 0) return PKV_OK;
+  if (!src_dst_pairs || !src_key || !src_value || !dst_key || !dst_value) return PKV_ERR_NULL_POINTER;
+  if (!aligned16(src_key) || !aligned16(src_value) || !aligned16(dst_key) || !aligned16(dst_value))
+    return PKV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    const bool same = src_key == dst_key || src_value == dst_value;
+    const int rc = check_pairs(src_dst_pairs, num_pairs, src_num_blocks, dst_num_blocks, same, st);
+    if (rc) return rc;
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  return launch_block_copy(src_dst_pairs, num_pairs, src_key, src_value, src_num_blocks, dst_key, dst_value,
+                           dst_num_blocks, block_bytes, status, st) == cudaSuccess
              ? PKV_OK
              : PKV_ERR_CUDA;
 }

@@ -54,8 +54,10 @@ struct KvWriteArgs {
 };
 
 cudaError_t launch_kv_write(const KvWriteArgs& a, cudaStream_t st);
-cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, void* kc, void* vc, int64_t num_blocks,
-                              int64_t block_bytes, unsigned* status, cudaStream_t st);
+cudaError_t launch_fp8_scale(const void* x, int64_t n, int dtype, float* scale, cudaStream_t st);
+cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, const void* src_k, const void* src_v,
+                              int64_t src_blocks, void* dst_k, void* dst_v, int64_t dst_blocks, int64_t block_bytes,
+                              unsigned* status, cudaStream_t st);
 
 // The tensor-core decode kernels serve head_dim 128 with 16- or 32-token
 // blocks: fp8 caches with 8 query heads per KV head, and bf16 caches with 2,

@@ -308,3 +308,43 @@ def test_fused_append_equals_write_then_decode(spec):
     assert_cache_equal(kc, rk, "append key_cache")
     assert_close(f64(out), ref, *tol_for(w), what="fused append")
     assert pk.device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, FP8])
+def test_swap_out_and_in_through_pinned_host_memory(dtype):
+    """One launch moves blocks device -> pinned host (swap out) and back (swap
+    in), byte-exact against the oracle's copies."""
+    spec = W.LLAMA7B.with_(num_seqs=4, num_q_heads=8, num_kv_heads=8, cache_dtype=dtype,
+                           ctx=("list", (40, 300, 17, 129)), new_tokens=False)
+    w = W.make_decode_workload(spec, seed=16, device=DEV)
+    NB = w.num_blocks
+    host_k = torch.zeros((7,) + tuple(w.key_cache.shape[1:]), dtype=dtype).pin_memory()
+    host_v = torch.zeros_like(host_k).pin_memory()
+    out_pairs = torch.tensor([[NB - 1, 0], [3, 6], [0, 2], [5, 1]], dtype=torch.int64)
+    pk.swap_blocks(out_pairs.to(DEV), w.key_cache, w.value_cache, host_k, host_v, validate=True)
+    torch.cuda.synchronize()
+    hk = to_np(torch.zeros_like(host_k)).copy()
+    hv = hk.copy()
+    oracle.swap_blocks(out_pairs.numpy(), to_np(w.key_cache), to_np(w.value_cache), hk, hv)
+    assert np.array_equal(to_np(host_k), hk) and np.array_equal(to_np(host_v), hv)
+    # swap back in to other device blocks
+    kc, vc = w.key_cache.clone(), w.value_cache.clone()
+    in_pairs = torch.tensor([[0, 8], [6, 9], [2, 3]], dtype=torch.int64)
+    pk.swap_blocks(in_pairs.to(DEV), host_k, host_v, kc, vc, validate=True)
+    torch.cuda.synchronize()
+    ek, ev = to_np(w.key_cache).copy(), to_np(w.value_cache).copy()
+    oracle.swap_blocks(in_pairs.numpy(), hk, hv, ek, ev)
+    assert_cache_equal(kc, ek, "swap-in key_cache")
+    assert_cache_equal(vc, ev, "swap-in value_cache")
+    assert pk.device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("dtype,n", [(torch.bfloat16, 1 << 20), (torch.bfloat16, 1003), (torch.float32, 77777),
+                                     (torch.float32, 5)])
+def test_fp8_scale_on_device_matches_oracle(dtype, n):
+    g = torch.Generator(device=DEV).manual_seed(n)
+    x = torch.randn(n, generator=g, device=DEV, dtype=torch.float32).to(dtype)
+    x[n // 3] = -7.5
+    s = pk.fp8_scale_from_amax(x)
+    assert float(s.item()) == oracle.fp8_scale(to_np(x), ocode(dtype))
+    assert float(pk.fp8_scale_from_amax(torch.zeros(64, dtype=dtype, device=DEV)).item()) == 1.0

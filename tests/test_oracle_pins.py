@@ -463,3 +463,35 @@ def test_parallel_sampling_first_step_copies_golden():
     assert spec.sampling[1] == g["n"]
     assert info["ref_count_prompt"] == g["prompt_ref_count"]
     assert len(pairs) == prompts * g["copies_per_prompt_first_step"] == 96
+
+
+def test_swap_blocks_between_pools_byte_exact():
+    rng = np.random.default_rng(19)
+    dev_k = rng.integers(0, 256, (12, 16, 2, 64)).astype(np.uint8)
+    dev_v = rng.integers(0, 256, (12, 16, 2, 64)).astype(np.uint8)
+    host_k = rng.integers(0, 256, (5, 16, 2, 64)).astype(np.uint8)
+    host_v = rng.integers(0, 256, (5, 16, 2, 64)).astype(np.uint8)
+    hk0, hv0 = host_k.copy(), host_v.copy()
+    pairs = np.array([[11, 0], [3, 4], [3, 2]], np.int64)     # a source may be copied twice
+    oracle.swap_blocks(pairs, dev_k, dev_v, host_k, host_v)
+    ek, ev = hk0.copy(), hv0.copy()
+    for s_, d_ in pairs:
+        ek[d_], ev[d_] = dev_k[s_], dev_v[s_]
+    assert np.array_equal(host_k, ek) and np.array_equal(host_v, ev)
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(np.array([[0, 5]]), dev_k, dev_v, host_k, host_v)       # dst past the host pool
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(np.array([[0, 1], [2, 1]]), dev_k, dev_v, host_k, host_v)  # repeated destination
+
+
+def test_fp8_scale_is_amax_over_448():
+    rng = np.random.default_rng(20)
+    x = rng.standard_normal(1001).astype(np.float32)
+    x[417] = -9.75                                   # the largest magnitude is negative
+    assert oracle.fp8_scale(x) == np.float32(np.float32(9.75) / np.float32(448.0))
+    assert oracle.fp8_scale(np.zeros(10, np.float32)) == 1.0
+    b = bf16_bits(x)
+    assert oracle.fp8_scale(b, oracle.BF16) == np.float32(np.abs(bf16_value(b)).max().astype(np.float32) / np.float32(448))
+    # the scale maps the amax onto the largest finite code
+    s = oracle.fp8_scale(x)
+    assert oracle.e4m3_from_float(np.float32(np.float32(9.75) * (np.float32(1) / np.float32(s)))) in (0x7E, 0xFE)
