@@ -351,6 +351,54 @@ size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, int num_kv_h
                                      int64_t num_tokens, int64_t num_pairs);
 
 /*
+ * Prefix caching by hash chain (host side; no device work).
+ *
+ * Source: "vLLM KV Cache 实现机制", 4.2 -- a full block is identified by a hash
+ * of (the parent block's hash, the exact tokens in the block, an extra hash
+ * for multimodal inputs), and requests whose prompts share a prefix reuse the
+ * cached blocks; 3.2 -- reference counts keep shared blocks from eviction,
+ * which is least-recently-used.  The hash is FNV-1a 64 over the little-endian
+ * bytes of (parent hash, the block's int32 tokens, extra_hash); the first
+ * block's parent hash is 0.  Only full blocks are hashed or cached.  Every
+ * cache hit also compares the stored tokens, parent and extra hash, so two
+ * blocks with colliding hashes are never shared.  The cache maps blocks to the
+ * caller's physical block ids; it never allocates or frees device blocks.
+ * The functions of one cache are thread-safe.
+ *
+ * pkv_prefix_block_hashes: hashes of the num_tokens / block_size full blocks
+ *   (chained from parent_hash) into hashes_out; returns that count.
+ * pkv_prefix_cache_create / _destroy: a cache of at most capacity_blocks
+ *   entries for blocks of block_size tokens (NULL on bad arguments).
+ * pkv_prefix_cache_match: the longest cached prefix of `tokens` (at most
+ *   max_blocks blocks): writes its physical block ids, takes one reference
+ *   on each and marks them recently used; returns the number of blocks.
+ * pkv_prefix_cache_insert: registers the first num_blocks full blocks of
+ *   `tokens` with physical ids block_ids (one reference each, held by the
+ *   caller); blocks already cached get one more reference instead.  Returns
+ *   the number of new entries, or PKV_ERR_OUT_OF_RANGE (inserting nothing)
+ *   when they would exceed the capacity -- evict first.
+ * pkv_prefix_cache_release: drops one reference from each of the first
+ *   num_blocks cached blocks of `tokens`; returns how many were released.
+ * pkv_prefix_cache_evict: removes up to max_evict unreferenced entries, least
+ *   recently used first, writing their physical ids (now free for the
+ *   caller's pool); returns the count.
+ * pkv_prefix_cache_size: number of entries.
+ * Errors: PKV_ERR_NULL_POINTER, PKV_ERR_BAD_SHAPE, PKV_ERR_OUT_OF_RANGE.
+ */
+int64_t pkv_prefix_block_hashes(const int32_t* tokens, int64_t num_tokens, int block_size, uint64_t parent_hash,
+                                uint64_t extra_hash, uint64_t* hashes_out);
+void* pkv_prefix_cache_create(int block_size, int64_t capacity_blocks);
+void pkv_prefix_cache_destroy(void* cache);
+int64_t pkv_prefix_cache_size(void* cache);
+int64_t pkv_prefix_cache_match(void* cache, const int32_t* tokens, int64_t num_tokens, uint64_t extra_hash,
+                               int32_t* block_ids_out, int64_t max_blocks);
+int64_t pkv_prefix_cache_insert(void* cache, const int32_t* tokens, int64_t num_tokens, uint64_t extra_hash,
+                                const int32_t* block_ids, int64_t num_blocks);
+int64_t pkv_prefix_cache_release(void* cache, const int32_t* tokens, int64_t num_tokens, uint64_t extra_hash,
+                                 int64_t num_blocks);
+int64_t pkv_prefix_cache_evict(void* cache, int64_t max_evict, int32_t* evicted_ids_out);
+
+/*
  * Reads the current device's status word (PKV_STATUS_* bits) into *status,
  * after synchronising `stream`; clears it if `clear` != 0.
  */

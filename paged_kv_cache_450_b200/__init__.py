@@ -30,7 +30,8 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax", "decode_step", "decode_step_staging_bytes",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
+           "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
            "library_path"]
@@ -332,3 +333,74 @@ def decode_step(q, new_k, new_v, slot_mapping, block_tables, context_lens, key_c
         return paged_attention_decode(q, key_cache, value_cache, block_tables, context_lens, scale, k_scale=k_scale,
                                       v_scale=v_scale, out=out, workspace=workspace,
                                       partition_tokens=partition_tokens, stream=st)
+
+
+# --------------------------------------------------------------------------- #
+# prefix caching by hash chain (host side)
+# --------------------------------------------------------------------------- #
+
+def _i32(tokens):
+    import numpy as np
+    return np.ascontiguousarray(tokens, dtype=np.int32)
+
+
+def prefix_block_hashes(tokens, block_size: int, parent_hash: int = 0, extra_hash: int = 0):
+    """Chained FNV-1a 64 hashes of the full blocks of `tokens` (numpy uint64)."""
+    import numpy as np
+    t = _i32(tokens)
+    out = np.zeros(max(1, t.size // block_size), np.uint64)
+    n = _lib.load().pkv_prefix_block_hashes(t.ctypes.data, t.size, block_size, parent_hash, extra_hash,
+                                            out.ctypes.data)
+    _check(min(n, 0), "prefix_block_hashes")
+    return out[:n]
+
+
+class PrefixCache:
+    """Hash-chain prefix cache mapping full token blocks to physical block ids
+    (reference counted, LRU eviction of unreferenced entries).  Host only."""
+
+    def __init__(self, block_size: int, capacity_blocks: int):
+        self.block_size = block_size
+        self._lib = _lib.load()
+        self._h = self._lib.pkv_prefix_cache_create(block_size, capacity_blocks)
+        if not self._h:
+            raise ValueError("bad prefix cache arguments")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pkv_prefix_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def __len__(self):
+        return int(self._lib.pkv_prefix_cache_size(self._h))
+
+    def match(self, tokens, extra_hash: int = 0, max_blocks: int | None = None) -> list:
+        import numpy as np
+        t = _i32(tokens)
+        cap = t.size // self.block_size if max_blocks is None else max_blocks
+        ids = np.zeros(max(1, cap), np.int32)
+        n = self._lib.pkv_prefix_cache_match(self._h, t.ctypes.data, t.size, extra_hash, ids.ctypes.data, cap)
+        _check(min(n, 0), "prefix_cache_match")
+        return ids[:n].tolist()
+
+    def insert(self, tokens, block_ids, extra_hash: int = 0) -> int:
+        t, ids = _i32(tokens), _i32(block_ids)
+        n = self._lib.pkv_prefix_cache_insert(self._h, t.ctypes.data, t.size, extra_hash, ids.ctypes.data, ids.size)
+        _check(min(n, 0), "prefix_cache_insert")
+        return int(n)
+
+    def release(self, tokens, num_blocks: int, extra_hash: int = 0) -> int:
+        t = _i32(tokens)
+        n = self._lib.pkv_prefix_cache_release(self._h, t.ctypes.data, t.size, extra_hash, num_blocks)
+        _check(min(n, 0), "prefix_cache_release")
+        return int(n)
+
+    def evict(self, max_evict: int) -> list:
+        import numpy as np
+        ids = np.zeros(max(1, max_evict), np.int32)
+        n = self._lib.pkv_prefix_cache_evict(self._h, max_evict, ids.ctypes.data)
+        _check(min(n, 0), "prefix_cache_evict")
+        return ids[:n].tolist()

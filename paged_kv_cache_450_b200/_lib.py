@@ -33,6 +33,14 @@ SIGNATURES = {
     "pkv_kv_block_copy": (I, [P, I64, P, P, I64, I64, I, P]),
     "pkv_fp8_scale_from_amax": (I, [P, I64, I, P, P]),
     "pkv_swap_blocks": (I, [P, I64, P, P, I64, P, P, I64, I64, I, P]),
+    "pkv_prefix_block_hashes": (I64, [P, I64, I, U64, U64, P]),
+    "pkv_prefix_cache_create": (P, [I, I64]),
+    "pkv_prefix_cache_destroy": (None, [P]),
+    "pkv_prefix_cache_size": (I64, [P]),
+    "pkv_prefix_cache_match": (I64, [P, P, I64, U64, P, I64]),
+    "pkv_prefix_cache_insert": (I64, [P, P, I64, U64, P, I64]),
+    "pkv_prefix_cache_release": (I64, [P, P, I64, U64, I64]),
+    "pkv_prefix_cache_evict": (I64, [P, I64, P]),
     "pkv_device_status": (I, [ctypes.POINTER(ctypes.c_uint), I, P]),
     "pkv_launch_count": (U64, []),
 }

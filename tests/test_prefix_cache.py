@@ -1,0 +1,88 @@
+"""Prefix caching by hash chain: the reference (oracle/prefix.py) pinned to
+the chain's defining properties, then the library's native implementation
+checked against it operation by operation (host only, no GPU)."""
+import numpy as np
+import pytest
+
+import paged_kv_cache_450_b200 as pk
+from oracle import prefix as ref
+
+
+def test_fnv1a_definition_cases():
+    assert ref.fnv1a(b"") == ref.FNV_OFFSET                                   # no input: the offset basis
+    assert ref.fnv1a(b"\x00") == (ref.FNV_OFFSET * ref.FNV_PRIME) % 2 ** 64   # xor with 0 leaves h
+    assert ref.fnv1a(b"\x01") != ref.fnv1a(b"\x00")
+
+
+def test_chain_properties():
+    rng = np.random.default_rng(0)
+    toks = rng.integers(0, 50000, 16 * 6).tolist()
+    h = ref.block_hashes(toks, 16)
+    assert len(h) == 6 and len(set(h)) == 6
+    assert ref.block_hashes(toks + [1, 2, 3], 16) == h                        # partial blocks are not hashed
+    for i in range(6):                                                        # a token change in block i
+        t2 = list(toks)
+        t2[16 * i + 5] += 1
+        h2 = ref.block_hashes(t2, 16)
+        assert h2[:i] == h[:i] and all(a != b for a, b in zip(h2[i:], h[i:]))
+    assert all(a != b for a, b in zip(ref.block_hashes(toks, 16, extra=7), h))   # the extra hash
+    assert all(a != b for a, b in zip(ref.block_hashes(toks, 16, parent=1), h))  # the parent
+
+
+def test_reference_cache_semantics():
+    c = ref.RefPrefixCache(4, capacity=6)
+    sys_prompt = [9, 8, 7, 6, 5, 4, 3, 2]
+    a = sys_prompt + [1, 1, 1, 1]
+    b = sys_prompt + [2, 2, 2, 2, 0]
+    assert c.match(a) == []
+    assert c.insert(a, [10, 11, 12]) == 3
+    assert c.match(b) == [10, 11]                 # the shared prefix, whole blocks only
+    assert c.match(a, extra=5) == []              # another multimodal extra hash: no reuse
+    assert c.insert(b, [10, 11, 13]) == 1         # two blocks already cached
+    assert c.evict(10) == []                      # everything is referenced
+    assert c.release(a, 3) == 3 and c.release(b, 3) == 3
+    assert c.evict(1) == [12]                     # least recently used unreferenced entry first
+    assert c.insert([0] * 16, [20, 21, 22, 23]) is None   # 4 new > capacity 6 - 4: nothing inserted
+
+
+def test_native_hashes_match_reference():
+    rng = np.random.default_rng(1)
+    for bs in (8, 16, 32):
+        toks = rng.integers(-5, 2 ** 31 - 1, bs * 9 + 3).astype(np.int32)
+        for parent, extra in ((0, 0), (12345, 0), (0, 2 ** 63 + 7)):
+            got = pk.prefix_block_hashes(toks, bs, parent, extra)
+            assert [int(x) for x in got] == ref.block_hashes(toks.tolist(), bs, parent, extra)
+
+
+def test_native_cache_matches_reference_on_random_operations():
+    rng = np.random.default_rng(2)
+    bs = 4
+    native, oracle_cache = pk.PrefixCache(bs, 24), ref.RefPrefixCache(bs, 24)
+    prompts = [rng.integers(0, 6, bs * rng.integers(1, 7)).tolist() for _ in range(12)]
+    for p in prompts[6:]:                      # share prefixes between some prompts
+        p[:bs * 2] = prompts[0][:bs * 2] if len(prompts[0]) >= 2 * bs else p[:bs * 2]
+    next_id = 100
+    for step in range(400):
+        op = rng.integers(0, 4)
+        p = prompts[rng.integers(len(prompts))]
+        extra = int(rng.integers(0, 2))
+        if op == 0:
+            assert native.match(p, extra) == oracle_cache.match(p, extra), step
+        elif op == 1:
+            n = len(p) // bs
+            ids = list(range(next_id, next_id + n))
+            next_id += n
+            r = oracle_cache.insert(p, ids, extra)
+            if r is None:
+                with pytest.raises(pk.PagedKVError):
+                    native.insert(p, ids, extra)
+            else:
+                assert native.insert(p, ids, extra) == r, step
+        elif op == 2:
+            n = int(rng.integers(0, len(p) // bs + 1))
+            assert native.release(p, n, extra) == oracle_cache.release(p, n, extra), step
+        else:
+            k = int(rng.integers(0, 4))
+            assert native.evict(k) == oracle_cache.evict(k), step
+        assert len(native) == len(oracle_cache)
+    native.close()
