@@ -76,6 +76,9 @@ def _load():
     lib.orc_kv_block_copy.restype = I
     lib.orc_swap_blocks.argtypes = [P, I64, P, P, I64, P, P, I64, I64]
     lib.orc_swap_blocks.restype = I
+    lib.orc_paged_attention_multiquery.argtypes = [P, P, I, P, P, P, I, P, P, I64, I, I, I, I, I64, I64, F, F, F,
+                                                   P, I64, I]
+    lib.orc_paged_attention_multiquery.restype = I
     lib.orc_fp8_scale.argtypes = [P, I64, I]
     lib.orc_fp8_scale.restype = F
     lib.orc_e4m3_encode_array.argtypes = [P, P, I64]
@@ -245,3 +248,34 @@ def fp8_scale(x, dtype=None) -> float:
     """amax(|x|) / 448 as an fp32 value (1.0 for all zeros)."""
     x = np.ascontiguousarray(x)
     return float(np.float32(_load().orc_fp8_scale(_ptr(x), x.size, _dtype_code(x, dtype))))
+
+
+def paged_attention_multiquery(q, query_start_loc, key_cache, value_cache, block_tables, context_lens, *, scale,
+                               q_dtype=None, cache_dtype=None, k_scale=1.0, v_scale=1.0, rows=None,
+                               num_threads=None):
+    """Causal multi-query attention over the paged cache, fp64.
+
+    q: [total_q, Hq, d]; query_start_loc int32 [B + 1]; the queries of sequence
+    b are its last q_len_b positions.  Returns float64 [total_q, Hq, d] (or
+    [len(rows), d] for selected flat rows token * Hq + hq)."""
+    lib = _load()
+    q = np.ascontiguousarray(q)
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    key_cache = np.ascontiguousarray(key_cache)
+    value_cache = np.ascontiguousarray(value_cache)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    T, Hq, d = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    B = context_lens.shape[0]
+    MB = block_tables.shape[1]
+    sel = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = T * Hq if sel is None else sel.shape[0]
+    out = np.zeros((max(n, 1), d), np.float64)
+    rc = lib.orc_paged_attention_multiquery(
+        _ptr(out), _ptr(q), _dtype_code(q, q_dtype), _ptr(qsl), _ptr(key_cache), _ptr(value_cache),
+        _dtype_code(key_cache, cache_dtype), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, d, bs, MB, NB, scale,
+        k_scale, v_scale, _ptr(sel), n, num_threads or default_threads())
+    _check(rc, "paged_attention_multiquery")
+    out = out[:n]
+    return out.reshape(T, Hq, d) if sel is None else out

@@ -476,3 +476,70 @@ float orc_fp8_scale(const void* x, int64_t n, int dtype) {
   volatile float s = af / 448.0f;
   return s;
 }
+
+/* ---------- multi-query paged attention (chunked prefill, speculative verify) -- */
+
+/*
+ * Several new query tokens per sequence over the paged cache, each attending
+ * causally: the q_len_b = query_start_loc[b+1] - query_start_loc[b] queries of
+ * sequence b are the last q_len_b positions of its context, so query i sits
+ * at position p = context_lens[b] - q_len_b + i and attends the logical
+ * tokens 0..p ("vLLM 与 KV Cache", KV Cache：为什么需要缓存: every new token
+ * attends all earlier ones; the paged addressing is the decode path's).  The
+ * pages describe only one new token per step; the several-token case is this
+ * library's extension (prefill chunks and draft-token verification).
+ * q and out: [total_q][num_q_heads][head_dim]; rows are q-token * Hq + hq.
+ * A query whose position is negative (q_len_b > context_lens[b]) attends
+ * nothing and gives zeros.  Everything in fp64; sel selects flat rows (NULL: all).
+ */
+int orc_paged_attention_multiquery(double* out, const void* q, int q_dtype, const int32_t* query_start_loc,
+                                   const void* key_cache, const void* value_cache, int cache_dtype,
+                                   const int32_t* block_tables, const int32_t* context_lens, int64_t num_seqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int64_t max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                                   float v_scale, const int64_t* sel, int64_t n_sel, int num_threads) {
+  if (q_dtype != ORC_F32 && q_dtype != ORC_BF16) return ORC_EINVAL;
+  if (!elem_size(cache_dtype)) return ORC_EINVAL;
+  int rc = check_decode_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                               num_blocks, block_tables, context_lens);
+  if (rc) return rc;
+  if (query_start_loc[0] != 0) return ORC_EINVAL;
+  for (int64_t b = 0; b < num_seqs; ++b)
+    if (query_start_loc[b + 1] < query_start_loc[b]) return ORC_EINVAL;
+  const int64_t total_q = query_start_loc[num_seqs];
+  const int64_t rows = total_q * num_q_heads;
+  int64_t n = sel ? n_sel : rows;
+  for (int64_t r = 0; r < n; ++r) {
+    int64_t row = sel ? sel[r] : r;
+    if (row < 0 || row >= rows) return ORC_ERANGE;
+  }
+  const int group = num_q_heads / num_kv_heads;
+  if (num_threads < 1) num_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+  for (int64_t r = 0; r < n; ++r) {
+    int64_t row = sel ? sel[r] : r;
+    int64_t tok = row / num_q_heads;
+    int hq = (int)(row % num_q_heads);
+    int64_t b = 0;
+    while (query_start_loc[b + 1] <= tok) ++b; /* the sequence owning query token tok */
+    int64_t q_len = query_start_loc[b + 1] - query_start_loc[b];
+    int64_t ctx = context_lens[b];
+    int64_t pos = ctx - q_len + (tok - query_start_loc[b]);
+    double* o = out + r * head_dim;
+    double* qv = (double*)malloc(sizeof(double) * head_dim);
+    int64_t nk = pos + 1 > 0 ? pos + 1 : 0;
+    double* K = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * head_dim);
+    double* V = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * head_dim);
+    for (int i = 0; i < head_dim; ++i) qv[i] = load_elem(q, row * head_dim + i, q_dtype, 1.0);
+    gather_logical(K, key_cache, cache_dtype, (double)k_scale, block_tables, max_blocks_per_seq, b, nk, block_size,
+                   num_kv_heads, head_dim, hq / group);
+    gather_logical(V, value_cache, cache_dtype, (double)v_scale, block_tables, max_blocks_per_seq, b, nk, block_size,
+                   num_kv_heads, head_dim, hq / group);
+    double m, l;
+    attend_range(o, &m, &l, qv, K, V, 0, nk, head_dim, (double)scale);
+    free(qv);
+    free(K);
+    free(V);
+  }
+  return ORC_OK;
+}

@@ -495,3 +495,63 @@ def test_fp8_scale_is_amax_over_448():
     # the scale maps the amax onto the largest finite code
     s = oracle.fp8_scale(x)
     assert oracle.e4m3_from_float(np.float32(np.float32(9.75) * (np.float32(1) / np.float32(s)))) in (0x7E, 0xFE)
+
+
+# --------------------------------------------------------------------------- #
+# multi-query (chunked prefill / verification) attention
+# --------------------------------------------------------------------------- #
+
+def test_multiquery_equals_sdpa_with_bottom_right_causal_mask():
+    rng = np.random.default_rng(21)
+    ctxs, qlens = [9, 40, 100, 17], [3, 40, 7, 1]
+    Hq, Hkv, d, bs = 4, 2, 64, 16
+    ks, vs = logical_seqs(rng, ctxs, Hkv, d), logical_seqs(rng, ctxs, Hkv, d)
+    order = rng.permutation(20)
+    tk, kp = page_logical(ks, bs, rng, num_blocks=20, order=order)
+    _, vp = page_logical(vs, bs, rng, num_blocks=20, order=order)
+    qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = rng.standard_normal((int(qsl[-1]), Hq, d)).astype(np.float32)
+    out = oracle.paged_attention_multiquery(q, qsl, kp, vp, tk, np.array(ctxs, np.int32), scale=0.125)
+    g = Hq // Hkv
+    for b, (c, n) in enumerate(zip(ctxs, qlens)):
+        qb = torch.from_numpy(q[qsl[b]:qsl[b + 1]].astype(np.float64)).permute(1, 0, 2)        # [Hq, n, d]
+        kb = torch.from_numpy(ks[b].astype(np.float64)).repeat_interleave(g, 1).permute(1, 0, 2)  # [Hq, c, d]
+        vb = torch.from_numpy(vs[b].astype(np.float64)).repeat_interleave(g, 1).permute(1, 0, 2)
+        # query i (position c - n + i) sees keys 0 .. c - n + i: a bottom-right aligned causal mask
+        mask = torch.arange(c)[None, :] <= (c - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=0.125)
+        np.testing.assert_allclose(out[qsl[b]:qsl[b + 1]], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_multiquery_with_one_query_per_sequence_is_decode():
+    rng = np.random.default_rng(22)
+    ctxs = [1, 33, 70]
+    ks, vs = logical_seqs(rng, ctxs, 2, 64), logical_seqs(rng, ctxs, 2, 64)
+    order = rng.permutation(12)
+    tk, kp = page_logical(ks, 16, rng, num_blocks=12, order=order)
+    _, vp = page_logical(vs, 16, rng, num_blocks=12, order=order)
+    q = rng.standard_normal((3, 8, 64)).astype(np.float32)
+    cl = np.array(ctxs, np.int32)
+    mq = oracle.paged_attention_multiquery(q, np.arange(4, dtype=np.int32), kp, vp, tk, cl, scale=0.2)
+    dec = oracle.paged_attention_decode(q, kp, vp, tk, cl, scale=0.2)
+    assert np.array_equal(mq, dec)
+
+
+def test_multiquery_chunked_prefill_is_consistent():
+    """Prefilling a prompt in two chunks (the second chunk's queries see the
+    first chunk's keys) gives the same rows as one causal pass."""
+    rng = np.random.default_rng(23)
+    n = 50
+    ks, vs = logical_seqs(rng, [n], 1, 64), logical_seqs(rng, [n], 1, 64)
+    tk, kp = page_logical(ks, 16, rng, num_blocks=5, order=rng.permutation(5))
+    vp = np.zeros_like(kp)
+    for t in range(n):
+        vp[tk[0, t // 16], t % 16] = vs[0][t]
+    q = rng.standard_normal((n, 1, 64)).astype(np.float32)
+    whole = oracle.paged_attention_multiquery(q, np.array([0, n], np.int32), kp, vp, tk, np.array([n], np.int32),
+                                              scale=0.125)
+    first = oracle.paged_attention_multiquery(q[:30], np.array([0, 30], np.int32), kp, vp, tk,
+                                              np.array([30], np.int32), scale=0.125)
+    second = oracle.paged_attention_multiquery(q[30:], np.array([0, 20], np.int32), kp, vp, tk,
+                                               np.array([n], np.int32), scale=0.125)
+    np.testing.assert_allclose(np.concatenate([first, second]), whole, rtol=1e-13, atol=1e-14)
