@@ -476,7 +476,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.SPECS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.SPECS) + sorted(W.MQ_SPECS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition-tokens", type=int, default=0)
@@ -488,6 +488,81 @@ def parse_args(argv=None):
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch (a smaller case of the same shape, for profiling)")
     return ap.parse_args(argv)
+
+
+def run_multiquery(args, rank, world, local_rank):
+    """Multi-query attention (draft verification / chunked prefill) timed alone."""
+    import paged_kv_cache_450_b200 as pk
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    spec, n = W.MQ_SPECS[args.workload]
+    mw = W.make_multiquery_workload(spec, [n] * spec.num_seqs, seed=rank_seed(args.seed, rank), device=dev)
+    w = mw.base
+    s = spec
+    kv_bytes = w.kv_bytes()
+    flops = mw.flops()
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(mw.q)
+    MB = w.block_tables.shape[1]
+    lib = pk._lib.load()
+    T = int(mw.query_start_loc[-1])
+    need = int(lib.pkv_multiquery_workspace_bytes(s.num_seqs, T, n, s.num_q_heads, s.num_kv_heads, s.head_dim,
+                                                  s.block_size, MB, args.partition_tokens))
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                      mw.query_start_loc, w.scale, max_q_len=n, out=out, workspace=ws,
+                                      partition_tokens=args.partition_tokens, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    launches0 = pk.launch_count()
+    t0.record(stream)
+    for _ in range(args.steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = pk.launch_count() - launches0
+    clk = clocks.stop()
+    step_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    total_kv = sum_over_ranks(kv_bytes, dev)
+    total_flops = sum_over_ranks(flops, dev)
+    if rank != 0:
+        return None
+    peak_gbs, peak_kind = hbm_peak()
+    gbs = kv_bytes / (step_ms * 1e-3) / 1e9
+    tflops = flops / (step_ms * 1e-3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak_tf = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        peak_tf = 1590.0
+    tensor_bound = flops / max(kv_bytes, 1) > peak_tf * 1e12 / (peak_gbs * 1e9)
+    return {
+        "metric": METRIC, "value": round(total_kv / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": s.name, "op": "paged_attention_multiquery (causal, queries = last q_len positions)",
+                   "num_seqs_per_gpu": s.num_seqs, "q_len": n, "num_q_heads": s.num_q_heads,
+                   "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
+                   "context_lens": list(s.ctx), "kv_bytes_per_step_per_gpu": kv_bytes, "flops_per_step": flops},
+        "tflops": round(total_flops / (step_ms * 1e-3) / 1e12, 2),
+        "roofline": {"kernel": "paged_multiquery_bf16_kernel" + (" + paged_multiquery_reduce_kernel" if need else ""),
+                     "bound": "tensor" if tensor_bound else "hbm",
+                     "achieved": round(tflops if tensor_bound else gbs, 2),
+                     "peak": peak_tf if tensor_bound else peak_gbs,
+                     "unit": "TFLOP/s" if tensor_bound else "GB/s",
+                     "frac": round((tflops / peak_tf) if tensor_bound else (gbs / peak_gbs), 4),
+                     "traffic": None},
+        "gpu_launches": int(launches), "clocks": clk, "cpu_baseline": None,
+    }
 
 
 def main(argv=None):
@@ -510,7 +585,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res = run_gpu(args, rank, world, local_rank)
+        if args.workload in W.MQ_SPECS:
+            res = run_multiquery(args, rank, world, local_rank)
+        else:
+            res = run_gpu(args, rank, world, local_rank)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

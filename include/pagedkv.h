@@ -270,6 +270,47 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
                       int64_t num_blocks, int64_t block_bytes, int validate, void* stream);
 
 /*
+ * Multi-query paged attention: several new query tokens per sequence
+ * (chunked prefill, speculative-decoding verification), causal over the
+ * paged cache.
+ *
+ * Source: the decode step's attention ("vLLM — 把操作系统的分页搬进 GPU KV
+ * cache", 核心要点; "vLLM 与 KV Cache", KV Cache：为什么需要缓存) with several
+ * new tokens per step -- an extension of this library; the pages describe one
+ * new token per step.  The q_len_b = query_start_loc[b+1] - query_start_loc[b]
+ * queries of sequence b are its LAST q_len_b positions (their K/V already in
+ * the cache, written with pkv_paged_kv_write): query i sits at position
+ * p = context_lens[b] - q_len_b + i and attends the logical tokens 0..p.
+ *
+ * out, q            device [total_q][num_q_heads][head_dim] bf16; rows of
+ *                   sequence b are query_start_loc[b] .. query_start_loc[b+1]-1.
+ * query_start_loc   device int32 [num_seqs + 1], non-decreasing, starting at 0,
+ *                   ending at total_q; every q_len_b <= max_q_len and
+ *                   <= context_lens[b] (validate checks all of this).
+ * workspace         device scratch of pkv_multiquery_workspace_bytes(...) bytes
+ *                   (same arguments; 0 when no split is needed), 256-byte aligned.
+ * Supported: bf16 q and caches, head_dim 128, block_size 16 or 32, 1/2/4/8
+ * query heads per KV head (tensor cores, mma.sync m16n8k16).  Other arguments
+ * and errors: as pkv_paged_attention_decode.
+ */
+int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cache, const void* value_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   const int32_t* query_start_loc, int num_seqs, int total_q, int max_q_len,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int64_t num_blocks, float scale, int q_dtype,
+                                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                                   int validate, void* stream);
+
+/* Split-context partition length pkv_paged_attention_multiquery uses (partition_tokens
+ * if non-zero, else automatic); negative PKV_ERR_* for unsupported arguments. */
+int pkv_multiquery_partition_tokens(int num_seqs, int max_q_len, int num_q_heads, int num_kv_heads, int block_size,
+                                    int max_blocks_per_seq, int partition_tokens);
+
+/* Workspace bytes pkv_paged_attention_multiquery needs. */
+size_t pkv_multiquery_workspace_bytes(int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int max_blocks_per_seq, int partition_tokens);
+
+/*
  * Per-tensor fp8 scale on the device: *scale = amax(|x|) / 448 (one fp32
  * division; 1.0 when x is all zeros), the scale that maps the largest
  * magnitude onto the largest finite E4M3 value.

@@ -30,7 +30,7 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_multiquery", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
@@ -199,6 +199,42 @@ def paged_decode_append(q, k_new, v_new, key_cache, value_cache, block_tables, c
             value_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(), B, Hq, Hkv, d, bs, MB, NB,
             float(scale), float(k_scale), float(v_scale), _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr,
             ws_bytes, int(validate), _stream(dev, stream)), "paged_decode_append")
+    return out
+
+
+def paged_attention_multiquery(q, key_cache, value_cache, block_tables, context_lens, query_start_loc,
+                                scale: float, *, max_q_len: int | None = None, out=None, workspace=None,
+                                partition_tokens: int = 0, validate: bool = False, stream=None):
+    """Causal attention of several new query tokens per sequence over the paged
+    cache (chunked prefill, speculative verification).  q: [total_q, Hq, d]
+    bf16; query_start_loc int32 [B + 1]; the queries of sequence b are its
+    last q_len_b positions (their K/V already written).  Returns [total_q, Hq, d]."""
+    dev = _cuda(q, key_cache, value_cache, block_tables, context_lens, query_start_loc)
+    for t in (block_tables, context_lens, query_start_loc):
+        if t.dtype != torch.int32:
+            raise TypeError("block_tables, context_lens and query_start_loc must be int32")
+    T, Hq, d = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    B = context_lens.shape[0]
+    if query_start_loc.shape != (B + 1,) or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    MB = block_tables.shape[1]
+    if max_q_len is None:
+        max_q_len = int((query_start_loc[1:] - query_start_loc[:-1]).max().item()) if B else 0
+    if out is None:
+        out = torch.empty_like(q)
+    lib = _lib.load()
+    need = int(lib.pkv_multiquery_workspace_bytes(B, T, max_q_len, Hq, Hkv, d, bs, MB, partition_tokens)) if B else 0
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        _check(lib.pkv_paged_attention_multiquery(
+            out.data_ptr(), q.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), block_tables.data_ptr(),
+            context_lens.data_ptr(), query_start_loc.data_ptr(), B, T, max_q_len, Hq, Hkv, d, bs, MB, NB,
+            float(scale), _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr, ws_bytes, int(validate),
+            _stream(dev, stream)), "paged_attention_multiquery")
     return out
 
 

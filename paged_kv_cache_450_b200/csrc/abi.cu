@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "launch.h"
+#include "multiquery_params.h"
 
 namespace pkv {
 
@@ -419,6 +420,132 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
                            num_blocks, block_bytes, status, st) == cudaSuccess
              ? PKV_OK
              : PKV_ERR_CUDA;
+}
+
+// Split-context partition length of the multi-query kernel: one partition
+// when (sequences x KV heads x 64-row query tiles) already gives two waves of
+// two CTAs per SM, else the context split so that it does (multiples of 256).
+static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int max_q_len, int block_size,
+                               int max_blocks_per_seq, int partition_tokens) {
+  if (partition_tokens != 0) {
+    if (partition_tokens < 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
+      return PKV_ERR_PARTITION;
+    return partition_tokens;
+  }
+  const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(static_cast<int64_t>(max_q_len) * group, 64);
+  const int64_t want = 4LL * sm_count();
+  int64_t P = units >= want ? 1 : cdiv64(want, units > 0 ? units : 1);
+  int64_t pt = cdiv64(max_ctx, P);
+  pt = cdiv64(pt, 256) * 256;
+  if (pt < 256) pt = 256;
+  if (pt >= max_ctx) pt = cdiv64(max_ctx, block_size) * block_size;
+  if (pt > kMaxPartitionTokens) pt = kMaxPartitionTokens;
+  return static_cast<int>(pt);
+}
+
+int pkv_multiquery_partition_tokens(int num_seqs, int max_q_len, int num_q_heads, int num_kv_heads, int block_size,
+                                    int max_blocks_per_seq, int partition_tokens) {
+  if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (num_seqs < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
+  return mq_partition_tokens(num_seqs, num_kv_heads, num_q_heads / num_kv_heads, max_q_len, block_size,
+                             max_blocks_per_seq, partition_tokens);
+}
+
+size_t pkv_multiquery_workspace_bytes(int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int max_blocks_per_seq, int partition_tokens) {
+  const int pt = pkv_multiquery_partition_tokens(num_seqs, max_q_len, num_q_heads, num_kv_heads, block_size,
+                                                 max_blocks_per_seq, partition_tokens);
+  if (pt < 0 || total_q <= 0 || head_dim <= 0) return 0;
+  const int64_t P = cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt);
+  if (P <= 1) return 0;
+  const size_t rows = static_cast<size_t>(total_q) * num_q_heads * P;
+  return align256(rows * 2 * sizeof(float)) + rows * head_dim * sizeof(float);
+}
+
+int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cache, const void* value_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   const int32_t* query_start_loc, int num_seqs, int total_q, int max_q_len,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int64_t num_blocks, float scale, int q_dtype,
+                                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                                   int validate, void* stream) {
+  if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_seqs == 0 || total_q == 0) return PKV_OK;
+  if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens || !query_start_loc)
+    return PKV_ERR_NULL_POINTER;
+  if (q_dtype != PKV_DTYPE_BF16 || cache_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (head_dim != 128) return PKV_ERR_HEAD_DIM;
+  if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_HEAD_GROUPING;
+  if (num_blocks > 0x7fffffffLL || num_seqs > 65535) return PKV_ERR_BAD_SHAPE;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
+  const int pt = mq_partition_tokens(num_seqs, num_kv_heads, group, max_q_len, block_size, max_blocks_per_seq,
+                                     partition_tokens);
+  if (pt < 0) return pt;
+  const int P = static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
+  if (P > 65535) return PKV_ERR_PARTITION;
+  const size_t need = pkv_multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads,
+                                                     head_dim, block_size, max_blocks_per_seq, partition_tokens);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    std::vector<int32_t> lens, tables, qsl;
+    if (!copy_to_host(lens, context_lens, static_cast<size_t>(num_seqs), st) ||
+        !copy_to_host(qsl, query_start_loc, static_cast<size_t>(num_seqs) + 1, st) ||
+        !copy_to_host(tables, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st))
+      return PKV_ERR_CUDA;
+    if (qsl[0] != 0 || qsl[num_seqs] != total_q) return PKV_ERR_OUT_OF_RANGE;
+    for (int b = 0; b < num_seqs; ++b) {
+      const int64_t ctx = lens[b], ql = static_cast<int64_t>(qsl[b + 1]) - qsl[b];
+      if (ql < 0 || ql > max_q_len || ctx < ql || ctx > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+        return PKV_ERR_OUT_OF_RANGE;
+      for (int64_t j = 0; j < cdiv64(ctx, block_size); ++j) {
+        const int64_t id = tables[static_cast<size_t>(b) * max_blocks_per_seq + j];
+        if (id < 0 || id >= num_blocks) return PKV_ERR_OUT_OF_RANGE;
+      }
+    }
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, true) ||
+      !encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, true))
+    return PKV_ERR_TENSOR_MAP;
+  MultiQueryParams p;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.query_start_loc = query_start_loc;
+  p.ws_ml = nullptr;
+  p.ws_o = nullptr;
+  if (need > 0) {
+    const size_t rows = static_cast<size_t>(total_q) * num_q_heads * P;
+    p.ws_ml = static_cast<float*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * 2 * sizeof(float)));
+  }
+  p.status = status;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = static_cast<int>(num_blocks);
+  p.block_size = block_size;
+  p.partition_blocks = pt / block_size;
+  p.max_partitions = P;
+  p.total_q = total_q;
+  p.q_scale = scale * kLog2e;
+  const int n_qtiles = static_cast<int>(cdiv64(static_cast<int64_t>(max_q_len) * group, 64));
+  if (n_qtiles <= 0) return PKV_OK;
+  return launch_multiquery_bf16(kmap, vmap, p, group, n_qtiles, P > 1, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 int pkv_fp8_scale_from_amax(const void* x, int64_t n, int dtype, float* scale, void* stream) {

@@ -11,6 +11,7 @@
 namespace pkv {
 
 struct DecodeParams;
+struct MultiQueryParams;
 
 // Counts one kernel launch (pkv_launch_count()).
 void count_launch();
@@ -72,6 +73,10 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
   if (cache_dtype == 1 /* PKV_DTYPE_BF16 */) return group == 2 || group == 4 || group == 8;
   return false;
 }
+
+// Multi-query (prefill / verification) attention: bf16, head_dim 128, bs 16/32.
+cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                                   int group, int n_qtiles, bool reduce, cudaStream_t st);
 
 // Decode launchers, one per (q dtype, cache dtype); each dispatches on
 // head_dim, block_size and the query-head group.  `reduce` adds the merge

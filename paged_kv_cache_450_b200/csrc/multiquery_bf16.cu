@@ -1,0 +1,43 @@
+// multiquery_bf16.cu -- launcher of the multi-query paged attention kernels.
+#include "launch.h"
+#include "multiquery.cuh"
+
+namespace pkv {
+
+template <int BS, int G>
+static cudaError_t launch_mq(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                             int n_qtiles, bool reduce, cudaStream_t st) {
+  using T = MqTraits<BS>;
+  auto kern = paged_multiquery_bf16_kernel<BS, G>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(p.num_kv_heads) * n_qtiles, p.max_partitions, p.num_seqs);
+  e = launch_pdl(kern, grid, dim3(T::THREADS), smem, st, kmap, vmap, p);
+  if (e != cudaSuccess || !reduce) return e;
+  const int64_t rows = static_cast<int64_t>(p.total_q) * p.num_q_heads;
+  return launch_pdl(paged_multiquery_reduce_kernel, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st, p);
+}
+
+template <int BS>
+static cudaError_t dispatch_mq_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                                     int group, int n_qtiles, bool reduce, cudaStream_t st) {
+  switch (group) {
+    case 1: return launch_mq<BS, 1>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 2: return launch_mq<BS, 2>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 4: return launch_mq<BS, 4>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 8: return launch_mq<BS, 8>(kmap, vmap, p, n_qtiles, reduce, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                                   int group, int n_qtiles, bool reduce, cudaStream_t st) {
+  switch (p.block_size) {
+    case 16: return dispatch_mq_group<16>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 32: return dispatch_mq_group<32>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace pkv

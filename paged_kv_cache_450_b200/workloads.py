@@ -293,3 +293,53 @@ def make_decode_workload(spec: DecodeSpec, seed: int = 0, device: str | torch.de
         new_k=new_k, new_v=new_v, slot_mapping=slot,
         copy_pairs=None if pairs is None else torch.from_numpy(pairs).to(device),
         info=info)
+
+
+@dataclass
+class MultiQueryWorkload:
+    """A decode-style pool plus several query tokens per sequence: the queries
+    of sequence b are its last q_len_b positions (their K/V are already in the
+    pool, as after a paged_kv_write of those tokens)."""
+    base: DecodeWorkload
+    q: torch.Tensor                 # [total_q, Hq, d]
+    query_start_loc: torch.Tensor   # int32 [B + 1]
+    q_lens: list
+
+    def flops(self) -> int:
+        """4 * d flops per (query, visible key, query head) pair."""
+        s = self.base.spec
+        ctx = self.base.ctx_list
+        pairs = 0
+        for c, n in zip(ctx, self.q_lens):
+            for i in range(n):
+                pairs += max(0, c - n + i + 1)
+        return 4 * s.head_dim * s.num_q_heads * pairs
+
+
+def make_multiquery_workload(spec: DecodeSpec, q_lens, seed: int = 0,
+                             device: str | torch.device = "cpu") -> MultiQueryWorkload:
+    """q_lens: one query count per sequence (each <= its context length).
+    The q tensor is drawn after the decode workload's tensors (same seed)."""
+    base = make_decode_workload(spec.with_(new_tokens=False), seed=seed, device=device)
+    q_lens = [int(n) for n in q_lens]
+    assert len(q_lens) == spec.num_seqs
+    for c, n in zip(base.ctx_list, q_lens):
+        if n > c:
+            raise ValueError("a sequence cannot have more queries than context tokens")
+    qsl = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    gen = torch.Generator(device=str(device))
+    gen.manual_seed(seed + 7919)
+    q = _randn((int(qsl[-1]), spec.num_q_heads, spec.head_dim), gen, str(device), spec.q_dtype)
+    return MultiQueryWorkload(base=base, q=q, query_start_loc=torch.from_numpy(qsl).to(device), q_lens=q_lens)
+
+
+# Multi-query workload families: draft verification (4 draft tokens + the
+# accepted one per sequence) and chunked prefill (512-token chunks after a
+# prefix), on the LLaMA-7B and 70B-GQA (bf16) shapes.
+MQ_SPECS = {
+    "llama7b_verify_b64_q5": (LLAMA7B.with_(name="llama7b_verify_b64_q5"), 5),
+    "llama7b_prefill_b8_chunk512": (LLAMA7B.with_(name="llama7b_prefill_b8_chunk512", num_seqs=8,
+                                                  ctx=("uniform", 512, 2048)), 512),
+    "gqa70b_bf16_verify_b64_q5": (GQA_BATCH_BF16.with_(name="gqa70b_bf16_verify_b64_q5", num_seqs=64,
+                                                        ctx=("uniform", 1024, 8192)), 5),
+}

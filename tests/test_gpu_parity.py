@@ -348,3 +348,65 @@ def test_fp8_scale_on_device_matches_oracle(dtype, n):
     s = pk.fp8_scale_from_amax(x)
     assert float(s.item()) == oracle.fp8_scale(to_np(x), ocode(dtype))
     assert float(pk.fp8_scale_from_amax(torch.zeros(64, dtype=dtype, device=DEV)).item()) == 1.0
+
+
+def _mq_check(mw, partition_tokens=0, rows=None, what=""):
+    w = mw.base
+    s = w.spec
+    out = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                        mw.query_start_loc, w.scale, partition_tokens=partition_tokens,
+                                        validate=True)
+    torch.cuda.synchronize()
+    ref = oracle.paged_attention_multiquery(to_np(mw.q), to_np(mw.query_start_loc), to_np(w.key_cache),
+                                            to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
+                                            scale=w.scale, q_dtype=oracle.BF16, cache_dtype=oracle.BF16, rows=rows)
+    got = f64(out)
+    if rows is not None:
+        got = got.reshape(-1, s.head_dim)[rows]
+    assert_close(got, ref, *TOL_BF16, what=what)
+    assert pk.device_status(clear=True) == 0
+    return out
+
+
+TOL_BF16 = (2e-3, 1e-2)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 2)])
+def test_multiquery_small(bs, hq, hkv):
+    ctxs = (1, 20, 700, 129, 33, 64)
+    q_lens = (1, 5, 8, 129, 0, 17)            # a full prefill from scratch (129 of 129), an empty query set
+    spec = W.DecodeSpec("mq", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs + hq, device=DEV)
+    for pt in (0, 2 * bs, 256):
+        _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
+
+
+def test_multiquery_prefill_chunk_after_prefix():
+    spec = W.LLAMA7B.with_(num_seqs=3, num_q_heads=8, num_kv_heads=8, ctx=("list", (600, 300, 1030)))
+    mw = W.make_multiquery_workload(spec, (300, 300, 512), seed=3, device=DEV)
+    for pt in (0, 128):
+        _mq_check(mw, partition_tokens=pt, what=f"prefill chunk pt={pt}")
+
+
+@pytest.mark.parametrize("name", sorted(W.MQ_SPECS))
+def test_multiquery_full_size_sampled(name):
+    spec, n = W.MQ_SPECS[name]
+    rng = np.random.default_rng(0)
+    mw = W.make_multiquery_workload(spec, [n] * spec.num_seqs, seed=0, device=DEV)
+    T = int(mw.query_start_loc[-1])
+    rows = np.unique(np.concatenate([rng.choice(T * spec.num_q_heads, 400, replace=False),
+                                     np.arange(spec.num_q_heads), T * spec.num_q_heads - 1 - np.arange(spec.num_q_heads)]))
+    _mq_check(mw, rows=rows, what=name)
+
+
+def test_multiquery_one_query_per_sequence_matches_decode():
+    spec = W.LLAMA7B.with_(num_seqs=5, num_q_heads=16, num_kv_heads=2, ctx=("list", (1, 40, 300, 17, 1000)))
+    mw = W.make_multiquery_workload(spec, (1,) * 5, seed=4, device=DEV)
+    w = mw.base
+    mq = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                       mw.query_start_loc, w.scale)
+    dec = pk.paged_attention_decode(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, w.scale)
+    torch.cuda.synchronize()
+    assert_close(f64(mq), f64(dec), *TOL_BF16, what="multi-query vs decode")
