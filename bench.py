@@ -497,6 +497,8 @@ def run_multiquery(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     spec, n = W.MQ_SPECS[args.workload]
+    if args.num_seqs:
+        spec = spec.with_(name=f"{spec.name}@b{args.num_seqs}", num_seqs=args.num_seqs)
     mw = W.make_multiquery_workload(spec, [n] * spec.num_seqs, seed=rank_seed(args.seed, rank), device=dev)
     w = mw.base
     s = spec

@@ -423,8 +423,9 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
 }
 
 // Split-context partition length of the multi-query kernel: one partition
-// when (sequences x KV heads x 64-row query tiles) already gives two waves of
-// two CTAs per SM, else the context split so that it does (multiples of 256).
+// when (sequences x KV heads x query-row tiles) already gives about two waves
+// of the kernel's resident CTAs, else the context split so that it does
+// (multiples of 256 tokens).
 static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int max_q_len, int block_size,
                                int max_blocks_per_seq, int partition_tokens) {
   if (partition_tokens != 0) {
@@ -433,8 +434,10 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
     return partition_tokens;
   }
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
-  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(static_cast<int64_t>(max_q_len) * group, 64);
-  const int64_t want = 4LL * sm_count();
+  const int64_t rows = static_cast<int64_t>(max_q_len) * group;
+  const bool small = rows <= 16;  // one-warp CTAs, ~6 per SM; else four-warp CTAs, 2 per SM
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(rows, small ? 16 : 64);
+  const int64_t want = (small ? 12LL : 4LL) * sm_count();
   int64_t P = units >= want ? 1 : cdiv64(want, units > 0 ? units : 1);
   int64_t pt = cdiv64(max_ctx, P);
   pt = cdiv64(pt, 256) * 256;
@@ -543,9 +546,9 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   p.max_partitions = P;
   p.total_q = total_q;
   p.q_scale = scale * kLog2e;
-  const int n_qtiles = static_cast<int>(cdiv64(static_cast<int64_t>(max_q_len) * group, 64));
-  if (n_qtiles <= 0) return PKV_OK;
-  return launch_multiquery_bf16(kmap, vmap, p, group, n_qtiles, P > 1, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  const int rows_per_seq = max_q_len * group;
+  if (rows_per_seq <= 0) return PKV_OK;
+  return launch_multiquery_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 int pkv_fp8_scale_from_amax(const void* x, int64_t n, int dtype, float* scale, void* stream) {

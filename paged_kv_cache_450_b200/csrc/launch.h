@@ -76,7 +76,7 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
 
 // Multi-query (prefill / verification) attention: bf16, head_dim 128, bs 16/32.
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
-                                   int group, int n_qtiles, bool reduce, cudaStream_t st);
+                                   int group, int rows_per_seq, bool reduce, cudaStream_t st);
 
 // Decode launchers, one per (q dtype, cache dtype); each dispatches on
 // head_dim, block_size and the query-head group.  `reduce` adds the merge

@@ -4,13 +4,14 @@
 // and query i (position p = ctx - q_len + i) attends the logical tokens 0..p.
 //
 // FlashAttention-2 style on the tensor cores (mma.sync m16n8k16, bf16
-// operands, fp32 accumulation).  One CTA = 64 query rows x one KV head x one
+// operands, fp32 accumulation).  One CTA = 64 query rows (16 when a sequence
+// has at most 16 rows per KV head, as in verification) x one KV head x one
 // split-context partition of one sequence; rows are (query i, query head g)
 // with g fastest, so grouped-query heads share every K/V tile.  A producer
 // warp streams the partition's blocks through a ring of TMA stages (K and V
 // tiles as two 128-byte half rows with the 128-byte swizzle, as the decode
-// kernels); four compute warps of 16 rows each consume every stage and
-// release it through an "empty" mbarrier.  Per 16-token tile and warp:
+// kernels); the compute warps (16 rows each) holding at least one valid row
+// consume every stage and release it through an "empty" mbarrier.  Per 16-token tile and warp:
 //   S = Q . K^T   M = 16 rows, N = 16 tokens, K = 128  (16 MMAs; K via ldmatrix)
 //   O += P . V    M = 16 rows, N = 128 dims,  K = 16   (2 x 16 MMAs; V via
 //                 ldmatrix.trans; P as bf16 hi + lo, ~16 bits per weight)
@@ -25,29 +26,30 @@
 
 namespace pkv {
 
-
-
-template <int BS, int NS_ = 0>
+// NWC_ compute warps of 16 rows each (4 for prefill-sized row counts, 1 for
+// verification-sized ones, so that small CTAs fill the SM).
+template <int BS, int NWC_ = 4, int NS_ = 0>
 struct MqTraits {
   static constexpr int D = 128;
-  static constexpr int NWC = 4;                      // compute warps (16 rows each)
+  static constexpr int NWC = NWC_;                   // compute warps (16 rows each)
   static constexpr int ROWS = 16 * NWC;              // query rows per CTA
   static constexpr int THREADS = 32 * (NWC + 1);     // + one producer warp
   static constexpr int HALF_BYTES = BS * 128;
   static constexpr int TILE_BYTES = 2 * HALF_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NS = NS_ > 0 ? NS_ : 4;
+  static constexpr int NS = NS_ > 0 ? NS_ : (NWC_ == 1 ? 3 : 4);
+  static constexpr int MIN_BLOCKS = NWC_ == 1 ? 6 : 2;
   static constexpr int NT = BS / 16;
   static constexpr int STAGE_AREA = NS * STAGE_BYTES;
   static constexpr int BAR_BYTES = 2 * NS * 8;
   static constexpr size_t smem_bytes(int pb) { return 1024 + STAGE_AREA + BAR_BYTES + static_cast<size_t>(pb) * 4; }
 };
 
-template <int BS, int G>
-__global__ void __launch_bounds__(MqTraits<BS>::THREADS, 2)
+template <int BS, int G, int NWC>
+__global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>::MIN_BLOCKS)
     paged_multiquery_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                                  const MultiQueryParams p) {
-  using T = MqTraits<BS>;
+  using T = MqTraits<BS, NWC>;
   constexpr int D = T::D;
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
@@ -74,7 +76,7 @@ __global__ void __launch_bounds__(MqTraits<BS>::THREADS, 2)
   const int Hq = p.num_q_heads;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   const int base_pos = ctx - q_len;  // position of query 0
-  // rows of this CTA: row = qt*64 + m, query i = row / G, head g = row % G
+  // rows of this CTA: row = qt*ROWS + m, query i = row / G, head g = row % G
   const int row_last = min(rows_total, (qt + 1) * T::ROWS) - 1;
   const int pos_last = base_pos + row_last / G;
   if (nparts == 0 || pos_last < 0) {  // nothing to attend: zero rows (partition 0 writes them)
@@ -100,15 +102,18 @@ __global__ void __launch_bounds__(MqTraits<BS>::THREADS, 2)
     }
     ids[i] = id;
   }
+  // compute warps holding at least one row of this CTA (the others leave now)
+  const int n_active = min(T::NWC, (min(rows_total - qt * T::ROWS, T::ROWS) + 15) / 16);
   const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * T::NS;
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, T::NWC);
+      mbar_init(empty0 + 8 * s, n_active);
     }
     fence_barrier_init();
   }
   __syncthreads();
+  if (warp < T::NWC && warp >= n_active) return;
   const uint32_t stage0 = smem_u32(data);
 
   if (warp == T::NWC) {  // ---------------- producer warp ----------------------

@@ -4,11 +4,11 @@
 
 namespace pkv {
 
-template <int BS, int G>
+template <int BS, int G, int NWC>
 static cudaError_t launch_mq(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                              int n_qtiles, bool reduce, cudaStream_t st) {
-  using T = MqTraits<BS>;
-  auto kern = paged_multiquery_bf16_kernel<BS, G>;
+  using T = MqTraits<BS, NWC>;
+  auto kern = paged_multiquery_bf16_kernel<BS, G, NWC>;
   const size_t smem = T::smem_bytes(p.partition_blocks);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -19,23 +19,30 @@ static cudaError_t launch_mq(const CUtensorMap& kmap, const CUtensorMap& vmap, c
   return launch_pdl(paged_multiquery_reduce_kernel, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st, p);
 }
 
-template <int BS>
+template <int BS, int NWC>
 static cudaError_t dispatch_mq_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                                      int group, int n_qtiles, bool reduce, cudaStream_t st) {
   switch (group) {
-    case 1: return launch_mq<BS, 1>(kmap, vmap, p, n_qtiles, reduce, st);
-    case 2: return launch_mq<BS, 2>(kmap, vmap, p, n_qtiles, reduce, st);
-    case 4: return launch_mq<BS, 4>(kmap, vmap, p, n_qtiles, reduce, st);
-    case 8: return launch_mq<BS, 8>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 1: return launch_mq<BS, 1, NWC>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 2: return launch_mq<BS, 2, NWC>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 4: return launch_mq<BS, 4, NWC>(kmap, vmap, p, n_qtiles, reduce, st);
+    case 8: return launch_mq<BS, 8, NWC>(kmap, vmap, p, n_qtiles, reduce, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
-                                   int group, int n_qtiles, bool reduce, cudaStream_t st) {
+                                   int group, int rows_per_seq, bool reduce, cudaStream_t st) {
+  // <= 16 rows per (sequence, kv head): one compute warp per CTA (16-row tiles)
+  const bool small = rows_per_seq <= 16;
+  const int n_qtiles = (rows_per_seq + (small ? 15 : 63)) / (small ? 16 : 64);
   switch (p.block_size) {
-    case 16: return dispatch_mq_group<16>(kmap, vmap, p, group, n_qtiles, reduce, st);
-    case 32: return dispatch_mq_group<32>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 16:
+      return small ? dispatch_mq_group<16, 1>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                   : dispatch_mq_group<16, 4>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 32:
+      return small ? dispatch_mq_group<32, 1>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                   : dispatch_mq_group<32, 4>(kmap, vmap, p, group, n_qtiles, reduce, st);
     default: return cudaErrorInvalidValue;
   }
 }

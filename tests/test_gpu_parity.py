@@ -383,6 +383,19 @@ def test_multiquery_small(bs, hq, hkv):
         _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
 
 
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv,q_lens", [(4, 4, (1, 5, 16, 0, 3, 7)), (8, 4, (8, 1, 0, 5, 2, 8)),
+                                           (16, 2, (2, 1, 0, 2, 1, 2))])
+def test_multiquery_verify_sized(bs, hq, hkv, q_lens):
+    # at most 16 rows per (sequence, KV head): the 16-row tile kernel
+    ctxs = (9, 20, 700, 129, 2100, 64)
+    spec = W.DecodeSpec("mqv", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs * hq, device=DEV)
+    for pt in (0, bs, 512):
+        _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
+
+
 def test_multiquery_prefill_chunk_after_prefix():
     spec = W.LLAMA7B.with_(num_seqs=3, num_q_heads=8, num_kv_heads=8, ctx=("list", (600, 300, 1030)))
     mw = W.make_multiquery_workload(spec, (300, 300, 512), seed=3, device=DEV)
