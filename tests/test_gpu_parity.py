@@ -396,6 +396,21 @@ def test_multiquery_verify_sized(bs, hq, hkv, q_lens):
         _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
 
 
+def test_multiquery_queries_before_the_context_get_zero_rows():
+    # context_lens shortened below q_len: the leading queries have no position
+    ctxs = (40, 300, 20, 900)
+    spec = W.DecodeSpec("mqneg", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, (20, 5, 20, 100), seed=11, device=DEV)
+    w = mw.base
+    w.context_lens.copy_(torch.tensor([7, 300, 0, 60], dtype=torch.int32, device=DEV))
+    for pt in (0, 16, 32):
+        out = _mq_check(mw, partition_tokens=pt, what=f"negative positions pt={pt}")
+        qsl = mw.query_start_loc.tolist()
+        assert torch.all(out[qsl[0]:qsl[0] + 13] == 0) and torch.all(out[qsl[2]:qsl[3]] == 0)
+        assert torch.all(out[qsl[3]:qsl[3] + 40] == 0)
+
+
 def test_multiquery_prefill_chunk_after_prefix():
     spec = W.LLAMA7B.with_(num_seqs=3, num_q_heads=8, num_kv_heads=8, ctx=("list", (600, 300, 1030)))
     mw = W.make_multiquery_workload(spec, (300, 300, 512), seed=3, device=DEV)

@@ -523,6 +523,23 @@ def test_multiquery_equals_sdpa_with_bottom_right_causal_mask():
         np.testing.assert_allclose(out[qsl[b]:qsl[b + 1]], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
 
 
+def test_multiquery_queries_before_the_context_get_zero_rows():
+    """More queries than context tokens: the first q_len - ctx queries sit at
+    negative positions, see no key and give zero rows; the rest equal a pass
+    over only the queries with a position."""
+    rng = np.random.default_rng(24)
+    ks, vs = logical_seqs(rng, [3], 1, 64), logical_seqs(rng, [3], 1, 64)
+    tk, kp = page_logical(ks, 16, rng, num_blocks=2, order=np.array([1, 0]))
+    vp = np.zeros_like(kp)
+    vp[tk[0, 0], :3] = vs[0]
+    q = rng.standard_normal((5, 2, 64)).astype(np.float32)
+    cl = np.array([3], np.int32)
+    out = oracle.paged_attention_multiquery(q, np.array([0, 5], np.int32), kp, vp, tk, cl, scale=0.125)
+    assert np.all(out[:2] == 0.0)
+    tail = oracle.paged_attention_multiquery(q[2:], np.array([0, 3], np.int32), kp, vp, tk, cl, scale=0.125)
+    assert np.array_equal(out[2:], tail)
+
+
 def test_multiquery_with_one_query_per_sequence_is_decode():
     rng = np.random.default_rng(22)
     ctxs = [1, 33, 70]

@@ -12,6 +12,9 @@ def test_fnv1a_definition_cases():
     assert ref.fnv1a(b"") == ref.FNV_OFFSET                                   # no input: the offset basis
     assert ref.fnv1a(b"\x00") == (ref.FNV_OFFSET * ref.FNV_PRIME) % 2 ** 64   # xor with 0 leaves h
     assert ref.fnv1a(b"\x01") != ref.fnv1a(b"\x00")
+    # published FNV-1a 64 test vectors
+    assert ref.fnv1a(b"a") == 0xaf63dc4c8601ec8c
+    assert ref.fnv1a(b"foobar") == 0x85944171f73967e8
 
 
 def test_chain_properties():
