@@ -286,12 +286,18 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
  *                   sequence b are query_start_loc[b] .. query_start_loc[b+1]-1.
  * query_start_loc   device int32 [num_seqs + 1], non-decreasing, starting at 0,
  *                   ending at total_q; every q_len_b <= max_q_len and
- *                   <= context_lens[b] (validate checks all of this).
+ *                   <= context_lens[b] (validate checks all of this; without
+ *                   validate, the first q_len_b - context_lens[b] queries of a
+ *                   sequence with more queries than context tokens sit at
+ *                   negative positions and get zero rows).
  * workspace         device scratch of pkv_multiquery_workspace_bytes(...) bytes
  *                   (same arguments; 0 when no split is needed), 256-byte aligned.
  * Supported: bf16 q and caches, head_dim 128, block_size 16 or 32, 1/2/4/8
- * query heads per KV head (tensor cores, mma.sync m16n8k16).  Other arguments
- * and errors: as pkv_paged_attention_decode.
+ * query heads per KV head.  Runs on the tensor cores: up to 64 rows per
+ * (sequence, KV head) -- rows = max_q_len x query heads per KV head -- on
+ * mma.sync m16n8k16; more rows (prefill) on tcgen05 with 128-row tiles and
+ * 128-token KV tiles.  Other arguments and errors: as
+ * pkv_paged_attention_decode.
  */
 int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cache, const void* value_cache,
                                    const int32_t* block_tables, const int32_t* context_lens,

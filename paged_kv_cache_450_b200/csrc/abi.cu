@@ -96,6 +96,22 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int64_t num_blo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over the bf16 queries [total_q][num_q_heads][128] of the tcgen05
+// multi-query kernel: one box = 128 / group queries x the group's query heads
+// x one 64-dim half (128 bytes, 128-byte swizzle), i.e. 128 MMA rows ordered
+// (query, head) with the head fastest.  Rows past total_q read as zeros.
+static bool encode_query_map(CUtensorMap* map, const void* q, int total_q, int num_q_heads, int group) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(total_q)};
+  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(num_q_heads) * 128 * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -435,9 +451,13 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
   }
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   const int64_t rows = static_cast<int64_t>(max_q_len) * group;
-  const bool small = rows <= 16;  // one-warp CTAs, ~6 per SM; else four-warp CTAs, 2 per SM
-  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(rows, small ? 16 : 64);
-  const int64_t want = (small ? 12LL : 4LL) * sm_count();
+  // CTAs per (sequence, KV head) and resident CTAs per SM of the kernel that
+  // serves these rows: 16-row one-warp CTAs (~6 per SM), 64-row CTAs (2 per
+  // SM), or 128-row tcgen05 CTAs (1 per SM)
+  const int tile = rows <= 16 ? 16 : (rows <= 64 ? 64 : 128);
+  const int per_sm = rows <= 16 ? 6 : (rows <= 64 ? 2 : 1);
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(rows, tile);
+  const int64_t want = 2LL * per_sm * sm_count();
   int64_t P = units >= want ? 1 : cdiv64(want, units > 0 ? units : 1);
   int64_t pt = cdiv64(max_ctx, P);
   pt = cdiv64(pt, 256) * 256;
@@ -548,6 +568,12 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   p.q_scale = scale * kLog2e;
   const int rows_per_seq = max_q_len * group;
   if (rows_per_seq <= 0) return PKV_OK;
+  if (multiquery_uses_tc(rows_per_seq)) {
+    CUtensorMap qmap;
+    if (!encode_query_map(&qmap, q, total_q, num_q_heads, group)) return PKV_ERR_TENSOR_MAP;
+    return launch_multiquery_tc(qmap, kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
+                                                                                                     : PKV_ERR_CUDA;
+  }
   return launch_multiquery_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -75,8 +75,17 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
 }
 
 // Multi-query (prefill / verification) attention: bf16, head_dim 128, bs 16/32.
+// Up to 64 rows per (sequence, KV head) -- rows = queries x query heads of the
+// group -- run on the mma.sync kernel; more rows (prefill) on the tcgen05
+// kernel with 128-row tiles.
+inline bool multiquery_uses_tc(int rows_per_seq) { return rows_per_seq > 64; }
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                                    int group, int rows_per_seq, bool reduce, cudaStream_t st);
+cudaError_t launch_multiquery_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                 const MultiQueryParams& p, int group, int rows_per_seq, bool reduce,
+                                 cudaStream_t st);
+// The split-context merge of either multi-query kernel.
+cudaError_t launch_multiquery_reduce(const MultiQueryParams& p, cudaStream_t st);
 
 // Decode launchers, one per (q dtype, cache dtype); each dispatches on
 // head_dim, block_size and the query-head group.  `reduce` adds the merge

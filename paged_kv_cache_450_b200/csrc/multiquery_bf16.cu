@@ -15,8 +15,7 @@ static cudaError_t launch_mq(const CUtensorMap& kmap, const CUtensorMap& vmap, c
   dim3 grid(static_cast<unsigned>(p.num_kv_heads) * n_qtiles, p.max_partitions, p.num_seqs);
   e = launch_pdl(kern, grid, dim3(T::THREADS), smem, st, kmap, vmap, p);
   if (e != cudaSuccess || !reduce) return e;
-  const int64_t rows = static_cast<int64_t>(p.total_q) * p.num_q_heads;
-  return launch_pdl(paged_multiquery_reduce_kernel, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st, p);
+  return launch_multiquery_reduce(p, st);
 }
 
 template <int BS, int NWC>
@@ -29,6 +28,11 @@ static cudaError_t dispatch_mq_group(const CUtensorMap& kmap, const CUtensorMap&
     case 8: return launch_mq<BS, 8, NWC>(kmap, vmap, p, n_qtiles, reduce, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_multiquery_reduce(const MultiQueryParams& p, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(p.total_q) * p.num_q_heads;
+  return launch_pdl(paged_multiquery_reduce_kernel, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st, p);
 }
 
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,

@@ -1,0 +1,45 @@
+// multiquery_tc.cu -- launcher of the tcgen05 multi-query attention kernel.
+#include "launch.h"
+#include "multiquery_tc.cuh"
+
+namespace pkv {
+
+template <int BS, int G>
+static cudaError_t launch_mq_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
+  using T = MqTcTraits<BS>;
+  auto kern = paged_multiquery_tc_kernel<BS, G>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(p.num_kv_heads) * n_qtiles, p.max_partitions, p.num_seqs);
+  e = launch_pdl(kern, grid, dim3(T::THREADS), smem, st, qmap, kmap, vmap, p);
+  if (e != cudaSuccess || !reduce) return e;
+  return launch_multiquery_reduce(p, st);
+}
+
+template <int BS>
+static cudaError_t dispatch_mq_tc_group(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                        const MultiQueryParams& p, int group, int n_qtiles, bool reduce,
+                                        cudaStream_t st) {
+  switch (group) {
+    case 1: return launch_mq_tc<BS, 1>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
+    case 2: return launch_mq_tc<BS, 2>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
+    case 4: return launch_mq_tc<BS, 4>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
+    case 8: return launch_mq_tc<BS, 8>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_multiquery_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                 const MultiQueryParams& p, int group, int rows_per_seq, bool reduce,
+                                 cudaStream_t st) {
+  const int n_qtiles = (rows_per_seq + 127) / 128;
+  switch (p.block_size) {
+    case 16: return dispatch_mq_tc_group<16>(qmap, kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 32: return dispatch_mq_tc_group<32>(qmap, kmap, vmap, p, group, n_qtiles, reduce, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace pkv

@@ -350,12 +350,12 @@ def test_fp8_scale_on_device_matches_oracle(dtype, n):
     assert float(pk.fp8_scale_from_amax(torch.zeros(64, dtype=dtype, device=DEV)).item()) == 1.0
 
 
-def _mq_check(mw, partition_tokens=0, rows=None, what=""):
+def _mq_check(mw, partition_tokens=0, rows=None, what="", validate=True):
     w = mw.base
     s = w.spec
     out = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
                                         mw.query_start_loc, w.scale, partition_tokens=partition_tokens,
-                                        validate=True)
+                                        validate=validate)
     torch.cuda.synchronize()
     ref = oracle.paged_attention_multiquery(to_np(mw.q), to_np(mw.query_start_loc), to_np(w.key_cache),
                                             to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
@@ -397,18 +397,68 @@ def test_multiquery_verify_sized(bs, hq, hkv, q_lens):
 
 
 def test_multiquery_queries_before_the_context_get_zero_rows():
-    # context_lens shortened below q_len: the leading queries have no position
+    # context_lens shortened below q_len (which validate rejects): the leading queries have no position
     ctxs = (40, 300, 20, 900)
     spec = W.DecodeSpec("mqneg", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
                         ("slack", 1.2))
     mw = W.make_multiquery_workload(spec, (20, 5, 20, 100), seed=11, device=DEV)
     w = mw.base
     w.context_lens.copy_(torch.tensor([7, 300, 0, 60], dtype=torch.int32, device=DEV))
-    for pt in (0, 16, 32):
-        out = _mq_check(mw, partition_tokens=pt, what=f"negative positions pt={pt}")
+    for pt in (0, 16, 128):
+        out = _mq_check(mw, partition_tokens=pt, what=f"negative positions pt={pt}", validate=False)
         qsl = mw.query_start_loc.tolist()
         assert torch.all(out[qsl[0]:qsl[0] + 13] == 0) and torch.all(out[qsl[2]:qsl[3]] == 0)
         assert torch.all(out[qsl[3]:qsl[3] + 40] == 0)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2)])
+def test_multiquery_prefill_sized_tiles(bs, hq, hkv):
+    # more than 64 rows per (sequence, KV head): the 128-row tcgen05 kernel for
+    # partitions of a multiple of 128 tokens (0 = automatic), mma.sync otherwise
+    ctxs = (70, 500, 30, 1000, 10, 300, 2049)
+    q_lens = (70, 129, 1, 200, 0, 300, 77)
+    spec = W.DecodeSpec("mqp", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs + 3 * hq + hkv, device=DEV)
+    for pt in (0, 128, 384, 2 * bs):
+        _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
+
+
+@pytest.mark.parametrize("q_lens", [(5, 5, 5, 5), (200, 129, 64, 300)], ids=["verify", "prefill"])
+def test_multiquery_rows_past_the_context_are_never_used(q_lens):
+    ctxs = (300, 129, 100, 700)
+    spec = W.DecodeSpec("mqnan", len(ctxs), 8, 4, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=21, device=DEV)
+    _poison_unused_rows(mw.base)
+    for pt in (0, 128, 32):
+        out = _mq_check(mw, partition_tokens=pt, what=f"poisoned pool pt={pt}")
+        assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("q_lens", [(5, 5, 5), (100, 200, 40)], ids=["verify", "prefill"])
+def test_multiquery_guards_bad_block_ids(q_lens):
+    ctxs = (300, 400, 200)
+    spec = W.DecodeSpec("mqbad", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=22, device=DEV)
+    w = mw.base
+    bad = w.block_tables.clone()
+    bad[1, 3] = -7
+    bad[0, 10] = w.num_blocks
+    pk.device_status(clear=True)
+    out = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, bad, w.context_lens, mw.query_start_loc,
+                                        w.scale)
+    torch.cuda.synchronize()
+    assert pk.device_status(clear=True) & pk.STATUS_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+    qsl = mw.query_start_loc.tolist()
+    rows = np.arange(qsl[2] * 8, qsl[3] * 8)  # the sequence without bad ids is unaffected
+    ref = oracle.paged_attention_multiquery(to_np(mw.q), to_np(mw.query_start_loc), to_np(w.key_cache),
+                                            to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
+                                            scale=w.scale, q_dtype=oracle.BF16, cache_dtype=oracle.BF16, rows=rows)
+    assert_close(f64(out).reshape(-1, 128)[rows], ref, *TOL_BF16, what="unaffected sequence")
 
 
 def test_multiquery_prefill_chunk_after_prefix():
