@@ -9,25 +9,35 @@
 //   from the partition's start (a partition that is not a multiple of 128
 //   tokens ends in a partial tile, masked like the context end).
 //   S = Q . K^T      M = 128 rows, N = 128 tokens, K = 128 dims -> TMEM columns [0, 128)
-//   O += P . V       M = 128 rows, N = 128 dims,   K = 128 tokens -> TMEM columns [128, 256)
+//   O_h += P_h . V_h M = 128 rows, N = 128 dims,   K = 64 tokens (half h of the tile)
+//                    -> TMEM columns [128, 256) (h = 0) and [256, 384) (h = 1)
+// (Every MMA is as wide as the operands allow: the single issuing thread pays
+// about the same per instruction for N = 64 as for N = 128.)
 //
 // Q, K and V sit in shared memory in the 128-byte-swizzled layout (two
 // 64-element halves of every 256-byte row) as TMA delivers them; Q and K are
 // K-major operands, V (stored token-major, dims contiguous) is the N-major B
 // operand of P . V, so no transpose is ever made.  P never touches shared
-// memory: it is the TMEM A operand of P . V, split into a bf16 high part
-// (columns [256, 320)) and a bf16 residual (columns [320, 384)) -- two MMAs
-// per k-step -- so each probability keeps ~16 significant bits (a bf16 P
-// alone costs up to ~3e-3 absolute on short contexts).  Six warps:
-//   warps 0-3  softmax: thread t owns row t (TMEM lane t).  It reads its row
-//              of S from TMEM, applies the causal / context mask, keeps a
-//              reference max (the accumulator is rescaled only when a score
-//              passes it by more than 2^8), writes its row of P into TMEM
-//              and, at the end, reads its row of O, divides by the row sum
-//              and stores it (or the split-context partial).
-//   warp 4     TMA producer: Q once, then K and V tiles block by block through
-//              two-stage rings (one 4-D box per block and 64-dim half).
-//   warp 5     MMA issuer: one thread issues S_j as soon as the softmax has
+// memory: it is the TMEM A operand of P . V (columns [384, 512)), split into
+// a bf16 high part and a bf16 residual -- two MMAs per k-step -- so each
+// probability keeps ~16 significant bits (a bf16 P alone costs up to ~3e-3
+// absolute on short contexts).  Eleven warps:
+//   warps 0-7  softmax: warp w serves rows 32 (w & 3) .. +31 (the TMEM lanes
+//              its sub-partition may touch) and half h = w >> 2 of every KV
+//              tile's tokens.  The two halves are independent online
+//              softmaxes -- each with its own running max, row sum and
+//              accumulator O_h -- so the two warps of a sub-partition never
+//              wait for each other and their special-function (exp) and
+//              integer / FMA (P packing) phases interleave; they are merged
+//              once, in the epilogue.  Per tile a thread reads its 64 scores
+//              from TMEM, applies the causal / context mask, keeps a
+//              reference max (O_h is rescaled only when a score passes it by
+//              more than 2^8), and writes its 64 probabilities into P_h.
+//   warp 8     TMA producer of Q (once) and the K tiles (three-stage ring; one
+//              4-D box per block and 64-dim half); owns the TMEM allocation.
+//   warp 10    TMA producer of the V tiles (two-stage ring), so that a K load
+//              never waits behind a V stage that P . V still holds.
+//   warp 9     MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
 // Every wait is bounded (2 s); on a timeout the status bit is set, the loops
@@ -48,17 +58,20 @@ struct MqTcTraits {
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16)
   static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 bf16
-  static constexpr int NSTAGE = 2;           // K ring and V ring depth
+  static constexpr int NSK = 3, NSV = 2;     // K ring and V ring depth
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
-  static constexpr int V_OFF = K_OFF + NSTAGE * TILE;
-  static constexpr int BAR_OFF = V_OFF + NSTAGE * TILE;
-  // mbarriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, s_free, p_full, pv_done, mma_done
-  static constexpr int NBAR = 1 + 4 * NSTAGE + 5;
+  static constexpr int V_OFF = K_OFF + NSK * TILE;
+  static constexpr int BAR_OFF = V_OFF + NSV * TILE;
+  // mbarriers: q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_free, p_full[2], pv_done[2],
+  // mma_done (the pairs: one per token half)
+  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
-  static constexpr int IDS_OFF = SLOT_OFF + 16;
-  static constexpr int THREADS = 192;
-  static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O 128 | P hi 64 | P lo 64 | unused
+  static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [3 slots][2 halves][128 rows]
+  static constexpr int IDS_OFF = XCH_OFF + 3 * 2 * 128 * 4;
+  static constexpr int THREADS = 352;
+  static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
+  static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O_0 128 | O_1 128 | P hi 0,1 (32 + 32), lo 0,1 (32 + 32)
   static constexpr size_t smem_bytes(int pb) { return 1024 + IDS_OFF + static_cast<size_t>(pb) * 4; }
 };
 
@@ -69,6 +82,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
+}
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Bounded wait taken by every lane of a warp; the result is the same on every
@@ -130,39 +150,48 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const int nt = (tok_end - tok_begin + T::TOK - 1) / T::TOK;
   const int nb = (tok_end - tok_begin + BS - 1) / BS;
 
+  int local_bad = 0;
   for (int i = threadIdx.x; i < nb; i += blockDim.x) {
     int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb + i];
     if (id < 0 || id >= p.num_blocks) {
       set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
       id = -1;
+      local_bad = 1;
     }
     ids[i] = id;
   }
+  const bool any_bad = __syncthreads_or(local_bad) != 0;  // (also orders the ids before their use)
   const uint32_t base = smem_u32(data);
   const uint32_t bar0 = base + T::BAR_OFF;
   const uint32_t q_full = bar0;
   auto k_full = [&](int s) { return bar0 + 8 * (1 + s); };
-  auto k_empty = [&](int s) { return bar0 + 8 * (3 + s); };
-  auto v_full = [&](int s) { return bar0 + 8 * (5 + s); };
-  auto v_empty = [&](int s) { return bar0 + 8 * (7 + s); };
-  const uint32_t s_full = bar0 + 8 * 9, s_free = bar0 + 8 * 10, p_full = bar0 + 8 * 11, pv_done = bar0 + 8 * 12,
-                 mma_done = bar0 + 8 * 13;
+  auto k_empty = [&](int s) { return bar0 + 8 * (4 + s); };
+  auto v_full = [&](int s) { return bar0 + 8 * (7 + s); };
+  auto v_empty = [&](int s) { return bar0 + 8 * (9 + s); };
+  // P-full and P.V-done barriers per token half h (each completes once per tile)
+  const uint32_t s_full = bar0 + 8 * 11, s_free = bar0 + 8 * 12, mma_done = bar0 + 8 * 17;
+  auto p_full = [&](int h) { return bar0 + 8 * (13 + h); };
+  auto pv_done = [&](int h) { return bar0 + 8 * (15 + h); };
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < T::NSTAGE; ++s) {
+    for (int s = 0; s < T::NSK; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < T::NSV; ++s) {
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    mbar_init(s_free, 8);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(p_full(h), 4);
+      mbar_init(pv_done(h), 1);
+    }
     mbar_init(mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == T::W_K) {
     __syncwarp();
     tmem_alloc(base + T::SLOT_OFF, T::TMEM_COLS);
     tmem_relinquish();
@@ -171,63 +200,60 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(data + T::SLOT_OFF);
-  const uint32_t tmem_s = tmem, tmem_o = tmem + 128, tmem_phi = tmem + 256, tmem_plo = tmem + 320;
+  const uint32_t tmem_s = tmem;
+  auto tmem_o = [&](int h) { return tmem + 128 + 128 * h; };
+  auto tmem_phi = [&](int h) { return tmem + 384 + 32 * h; };  // tokens 64h .. 64h+63, packed in pairs
+  auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };
 
-  if (warp == 4) {  // ---------------- TMA producer ------------------------------------
+  if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
     if (lane == 0) {
+      const bool is_k = warp == T::W_K;
+      const int ns = is_k ? T::NSK : T::NSV;
+      const CUtensorMap* map = is_k ? &kmap : &vmap;
+      const uint32_t area = base + (is_k ? T::K_OFF : T::V_OFF);
       const uint64_t policy = l2_policy_evict_first();
-      mbar_arrive_expect_tx(q_full, T::TILE);
-      tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
-      tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, hk * G, q0 + qt * QPT);
-      int k_issued = 0, v_issued = 0;
+      if (is_k) {
+        mbar_arrive_expect_tx(q_full, T::TILE);
+        tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
+        tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, hk * G, q0 + qt * QPT);
+      }
+      int issued = 0;
       for (int j = 0; j < nt; ++j) {
-        const int s = j & 1;
+        const int s = j % ns, use = j / ns;
+        const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
         const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
         int nvalid = 0;
         for (int i = i0; i < i1; ++i) nvalid += ids[i] >= 0;
         const uint32_t bytes = static_cast<uint32_t>(nvalid) * 2u * BS * 128u;
-        // K tile j
-        if (j >= T::NSTAGE && !mbar_wait_bounded(k_empty(s), ((j >> 1) - 1) & 1, p.status)) break;
-        if (bytes) mbar_arrive_expect_tx(k_full(s), bytes); else mbar_arrive(k_full(s));
+        if (use > 0 && !mbar_wait_bounded(empty, (use - 1) & 1, p.status)) break;
+        if (bytes) mbar_arrive_expect_tx(full, bytes); else mbar_arrive(full);
         for (int i = i0; i < i1; ++i) {
           const int id = ids[i];
           if (id < 0) continue;
-          const uint32_t dst = base + T::K_OFF + s * T::TILE + (i - i0) * BS * 128;
-          tma_load_4d(dst, &kmap, k_full(s), 0, hk, 0, id, policy);
-          tma_load_4d(dst + T::HALF, &kmap, k_full(s), 64, hk, 0, id, policy);
+          const uint32_t dst = area + s * T::TILE + (i - i0) * BS * 128;
+          tma_load_4d(dst, map, full, 0, hk, 0, id, policy);
+          tma_load_4d(dst + T::HALF, map, full, 64, hk, 0, id, policy);
         }
-        k_issued = j + 1;
-        // V tile j
-        if (j >= T::NSTAGE && !mbar_wait_bounded(v_empty(s), ((j >> 1) - 1) & 1, p.status)) break;
-        if (bytes) mbar_arrive_expect_tx(v_full(s), bytes); else mbar_arrive(v_full(s));
-        for (int i = i0; i < i1; ++i) {
-          const int id = ids[i];
-          if (id < 0) continue;
-          const uint32_t dst = base + T::V_OFF + s * T::TILE + (i - i0) * BS * 128;
-          tma_load_4d(dst, &vmap, v_full(s), 0, hk, 0, id, policy);
-          tma_load_4d(dst + T::HALF, &vmap, v_full(s), 64, hk, 0, id, policy);
-        }
-        v_issued = j + 1;
+        issued = j + 1;
       }
       // drain (bounded): the copies of the last stages have landed before exit
-      mbar_wait_bounded(q_full, 0, p.status);
-      for (int j = max(0, k_issued - T::NSTAGE); j < k_issued; ++j)
-        mbar_wait_bounded(k_full(j & 1), (j >> 1) & 1, p.status);
-      for (int j = max(0, v_issued - T::NSTAGE); j < v_issued; ++j)
-        mbar_wait_bounded(v_full(j & 1), (j >> 1) & 1, p.status);
+      if (is_k) mbar_wait_bounded(q_full, 0, p.status);
+      for (int j = max(0, issued - ns); j < issued; ++j)
+        mbar_wait_bounded(is_k ? k_full(j % ns) : v_full(j % ns), (j / ns) & 1, p.status);
     }
-  } else if (warp == 5) {  // ---------------- MMA issuer ------------------------------
+  } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
       bool ok = mbar_wait_bounded(q_full, 0, p.status);
+      // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1)
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
-          const int s = j & 1;
-          if (!mbar_wait_bounded(k_full(s), (j >> 1) & 1, p.status)) break;
-          if (j > 0 && !mbar_wait_bounded(s_free, (j - 1) & 1, p.status)) break;
+          const int sk = j % T::NSK;
+          if (!(ok = mbar_wait_bounded(k_full(sk), (j / T::NSK) & 1, p.status))) break;
+          if (j > 0 && !(ok = mbar_wait_bounded(s_free, (j - 1) & 1, p.status))) break;
           tc_fence_after();
-          const uint32_t ka = base + T::K_OFF + s * T::TILE;
+          const uint32_t ka = base + T::K_OFF + sk * T::TILE;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * T::HALF + (kk & 3) * 32;
@@ -235,81 +261,100 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
                         idesc_s, kk > 0 ? 1u : 0u);
           }
           tc_commit(s_full);
-          tc_commit(k_empty(s));
+          tc_commit(k_empty(sk));
         }
         if (j > 0) {
-          const int jj = j - 1, s = jj & 1;
-          if (!mbar_wait_bounded(v_full(s), (jj >> 1) & 1, p.status)) break;
-          if (!mbar_wait_bounded(p_full, jj & 1, p.status)) break;
-          tc_fence_after();
-          const uint32_t va = base + T::V_OFF + s * T::TILE;
+          const int jj = j - 1, sv = jj % T::NSV;
+          if (!(ok = mbar_wait_bounded(v_full(sv), (jj / T::NSV) & 1, p.status))) break;
+          const uint32_t va = base + T::V_OFF + sv * T::TILE;
+          for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
+            if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
-            const uint64_t vdesc = smem_desc_sw128(va + kk * 16 * 128, T::HALF, 1024);
-            tc_mma_bf16_tmem_a(tmem_o, tmem_phi + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_bf16_tmem_a(tmem_o, tmem_plo + 8 * kk, vdesc, idesc_pv, 1u);
+            for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
+              const uint64_t vdesc = smem_desc_sw128(va + (64 * h + 16 * kk) * 128, T::HALF, 1024);
+              tc_mma_bf16_tmem_a(tmem_o(h), tmem_phi(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+            }
+            tc_commit(pv_done(h));
           }
-          tc_commit(pv_done);
-          tc_commit(v_empty(s));
+          if (!ok) break;
+          tc_commit(v_empty(sv));
         }
       }
       // drain (bounded): no MMA may still read shared memory or write TMEM at exit
       tc_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, p.status);
     }
-  } else {  // ---------------- softmax warps 0-3: thread t owns row t -------------------------
-    const int r = threadIdx.x;
+  } else {  // ---------------- softmax warps 0-7 ------------------------------------------
+    const int quarter = warp & 3, h = warp >> 2;  // TMEM lane quarter, token half of each tile
+    const int r = 32 * quarter + lane;            // this thread's row (TMEM lane)
     const int row = qt * T::ROWS + r;
     const bool valid = row < rows_total;
     const int pos = valid ? base_pos + row / G : -1;  // an invalid row sees nothing
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float qk = p.q_scale;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // this half's running reference max (log2 units) and row sum
+    // After a timed-out wait the warp stops waiting (every later wait fails at
+    // once) but still runs every iteration, so the two warps of a pair meet at
+    // the epilogue's named barrier; the status bit reports the failure.
     bool ok = true;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+      if (ok) ok = warp_wait_bounded(bar, parity, p.status);
+      return ok;
+    };
     for (int j = 0; j < nt; ++j) {
-      const int t0 = tok_begin + j * T::TOK;
-      if (!warp_wait_bounded(s_full, j & 1, p.status)) {
-        ok = false;
-        break;
-      }
+      const int t0 = tok_begin + j * T::TOK + 64 * h;  // first token of this half of the tile
+      wait(s_full, j & 1);
       tc_fence_after();
-      float sv[128];
+      float sv[64];
+      {
+        uint32_t u[2][32];
+        tmem_ld32(tmem_s + lane_off + 64 * h, u[0]);
+        tmem_ld32(tmem_s + lane_off + 64 * h + 32, u[1]);
+        tmem_ld_wait(u[0]);
+        tmem_ld_wait(u[1]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tmem_s + lane_off + 32 * c, u);
-        tmem_ld_wait(u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[32 * c + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 32; ++e) {
+          sv[e] = __uint_as_float(u[0][e]);
+          sv[32 + e] = __uint_as_float(u[1][e]);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
 
-      // blocks of this tile with a bad id (their tokens are masked, their V rows zeroed)
-      bool bad_tile = false;
-      {
-        const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
-        for (int i = i0; i < i1; ++i) bad_tile |= ids[i] < 0;
+      // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
+      bool bad = false;
+      if (any_bad) {
+        const int i0 = (t0 - tok_begin) / BS, i1 = min(nb, (t0 + 64 - tok_begin) / BS);
+        for (int i = i0; i < i1; ++i) bad |= ids[i] < 0;
       }
-      const bool ragged = t0 + T::TOK > tok_end;  // tokens at or past tok_end in this tile
-      float mx = -INFINITY;
-      if (t0 + T::TOK - 1 > pos || ragged || bad_tile) {
+      const bool ragged = t0 + 64 > tok_end;  // tokens at or past tok_end in this half tile
+      // row max of the raw scores (q_scale > 0 commutes with the max); masked scores -> -inf.
+      // Eight independent partial maxima / sums: instruction-level parallelism hides latency.
+      float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int t = t0 + c;
-          bool masked = t > pos || t >= tok_end;
-          if (bad_tile) masked = masked || ids[(t - tok_begin) / BS] < 0;
-          sv[c] = masked ? -INFINITY : sv[c] * qk;
-          mx = fmaxf(mx, sv[c]);
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+      if (t0 + 63 > pos || ragged || bad) {
+        if (bad) {  // scores of blocks that were not loaded (stale tiles) never reach the max
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (ids[(t0 + c - tok_begin) / BS] < 0) sv[c] = -INFINITY;
+        }
+        // column c is visible iff c <= last (causal position and the end of what is loaded)
+        const int last = min(pos, tok_end - 1) - t0;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          sv[c] = c > last ? -INFINITY : sv[c];
+          mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          sv[c] *= qk;
-          mx = fmaxf(mx, sv[c]);
-        }
+        for (int c = 0; c < 64; c += 2) mx8[(c >> 1) & 7] = fmax3f(mx8[(c >> 1) & 7], sv[c], sv[c + 1]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qk;
       // reference max: move it (and rescale) only when a score passes it by more than 8 (log2 units)
       float alpha = 1.f;
       if (mx > m + 8.f) {
@@ -317,112 +362,129 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         l *= alpha;
         m = mx;
       }
-      float sum = 0.f;
+      const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
+      // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add
+      const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
+      float2 sum4[4];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        sv[c] = m == -INFINITY ? 0.f : fast_exp2(sv[c] - m);
-        sum += sv[c];
+      for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), qk2, nm2);
+        sv[c] = fast_exp2(x.x);
+        sv[c + 1] = fast_exp2(x.y);
+        sum4[(c >> 1) & 3] = __fadd2_rn(sum4[(c >> 1) & 3], make_float2(sv[c], sv[c + 1]));
       }
-      l += sum;
-      // P_{j-1} . V_{j-1} must be complete before P and O are touched
+      const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
+      l += s2.x + s2.y;
+      // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
       if (j > 0) {
-        if (!warp_wait_bounded(pv_done, (j - 1) & 1, p.status)) {
-          ok = false;
-          break;
-        }
+        wait(pv_done(h), (j - 1) & 1);
         tc_fence_after();
-        if (__any_sync(kFullMask, alpha != 1.f)) {
+        if (__any_sync(kFullMask, alpha != 1.f)) {  // a moved reference: rescale this row of O_h
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t u[32];
-            tmem_ld32(tmem_o + lane_off + 32 * c, u);
+            const uint32_t oa = tmem_o(h) + lane_off + 32 * c;
+            tmem_ld32(oa, u);
             tmem_ld_wait(u);
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(tmem_o + lane_off + 32 * c, u);
-          }
-          tmem_st_wait();
-        }
-      }
-      // V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed: 0 * NaN would poison O
-      if (ragged || bad_tile) {
-        if (!warp_wait_bounded(v_full(j & 1), (j >> 1) & 1, p.status)) {
-          ok = false;
-          break;
-        }
-        const int t = t0 + r;
-        if (t >= tok_end || (bad_tile && ids[(t - tok_begin) / BS] < 0)) {
-          uint8_t* vrow = data + T::V_OFF + (j & 1) * T::TILE + r * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(vrow + T::HALF + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+            tmem_st32(oa, u);
           }
         }
       }
-      // row r of P into TMEM lane r: tokens (2k, 2k+1) in column k, high part and residual
+      // V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed: 0 * NaN would
+      // poison O.  The 64 rows of this half: thread (quarter, lane) takes row 16 quarter + lane / 2,
+      // dims half lane & 1.
+      if (ragged || bad) {
+        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
+        const int vr = 64 * h + 16 * quarter + (lane >> 1);
+        const int t = tok_begin + j * T::TOK + vr;
+        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
+          uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
+      }
+      // this half of row r of P into TMEM lane r: tokens (2k, 2k+1) in column k, as a high part (the
+      // top 16 bits of the fp32 value: truncation) and the residual (exact in fp32, then truncated to
+      // its top 16 bits): ~16 significant bits per probability, integer / FMA-pipe work only
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const float a = sv[32 * c + 2 * k], bb = sv[32 * c + 2 * k + 1];
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a, bb);
-          const __nv_bfloat162 lw = __floats2bfloat162_rn(a - __low2float(h), bb - __high2float(h));
-          hi[k] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[k] = *reinterpret_cast<const uint32_t*>(&lw);
+          const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
+          // residual = value - its truncation (the negated truncation is one logic op)
+          const float2 rr = __fadd2_rn(make_float2(a, bb), make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
+                                                                        __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
+          hi[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
+          lo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
         }
-        tmem_st16(tmem_phi + lane_off + 16 * c, hi);
-        tmem_st16(tmem_plo + lane_off + 16 * c, lo);
+        tmem_st16(tmem_phi(h) + lane_off + 16 * c, hi);
+        tmem_st16(tmem_plo(h) + lane_off + 16 * c, lo);
       }
       tmem_st_wait();
-      fence_proxy_async_smem();  // zeroed V rows (if any) before the MMA reads them
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full(h));
     }
-    if (ok && !warp_wait_bounded(pv_done, (nt - 1) & 1, p.status)) ok = false;
+    wait(pv_done(h), (nt - 1) & 1);
     tc_fence_after();
-    // ---- epilogue: row r of O / l ------------------------------------------------------
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 -----
+    float* xch = reinterpret_cast<float*>(data + T::XCH_OFF);  // [m_0, m_1, l_0, l_1][row]
+    xch[h * 128 + r] = m;
+    xch[(2 + h) * 128 + r] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");  // the two warps of this lane quarter
+    const float m_o = xch[(h ^ 1) * 128 + r], l_o = xch[(2 + (h ^ 1)) * 128 + r];
+    const float M = fmaxf(l > 0.f ? m : -INFINITY, l_o > 0.f ? m_o : -INFINITY);
+    const float w_self = l > 0.f ? fast_exp2(m - M) : 0.f, w_oth = l_o > 0.f ? fast_exp2(m_o - M) : 0.f;
+    const float lsum = l * w_self + l_o * w_oth;
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
     const int64_t orow = static_cast<int64_t>(q0 + row / G) * Hq + hk * G + row % G;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t u[32];
-      tmem_ld32(tmem_o + lane_off + 32 * c, u);
-      tmem_ld_wait(u);
+    for (int c = 0; c < 2; ++c) {
+      const int d0 = 64 * h + 32 * c;
+      uint32_t u0[32], u1[32];
+      tmem_ld32(tmem_o(0) + lane_off + d0, u0);
+      tmem_ld32(tmem_o(1) + lane_off + d0, u1);
+      tmem_ld_wait(u0);
+      tmem_ld_wait(u1);
       if (!valid || !ok) continue;
+      float o[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u0[e]) * w0 + __uint_as_float(u1[e]) * w1;
       if (nparts == 1) {
-        __nv_bfloat16* dst = out + orow * D + 32 * c;
+        __nv_bfloat16* dst = out + orow * D + d0;
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
           uint32_t w[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(u[e + 2 * k]) * inv,
-                                                     __uint_as_float(u[e + 2 * k + 1]) * inv);
-            w[k] = *reinterpret_cast<uint32_t*>(&h);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(o[e + 2 * k], o[e + 2 * k + 1]);
+            w[k] = *reinterpret_cast<uint32_t*>(&hv);
           }
           *reinterpret_cast<uint4*>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
-        float* dst = p.ws_o + (orow * p.max_partitions + part) * D + 32 * c;
+        float* dst = p.ws_o + (orow * p.max_partitions + part) * D + d0;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) =
-              make_float4(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv,
-                          __uint_as_float(u[e + 2]) * inv, __uint_as_float(u[e + 3]) * inv);
+        for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
       }
     }
-    if (valid && ok && nparts > 1) {
+    if (valid && ok && nparts > 1 && h == 0) {
       const int64_t srow = orow * p.max_partitions + part;
-      p.ws_ml[srow * 2] = l > 0.f ? m * kLn2 : 0.f;
-      p.ws_ml[srow * 2 + 1] = l;
+      p.ws_ml[srow * 2] = lsum > 0.f ? M * kLn2 : 0.f;
+      p.ws_ml[srow * 2 + 1] = lsum;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == T::W_K) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, T::TMEM_COLS);
