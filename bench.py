@@ -556,7 +556,7 @@ def run_multiquery(args, rank, world, local_rank):
                    "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
                    "context_lens": list(s.ctx), "kv_bytes_per_step_per_gpu": kv_bytes, "flops_per_step": flops},
         "tflops": round(total_flops / (step_ms * 1e-3) / 1e12, 2),
-        "roofline": {"kernel": ("paged_multiquery_tc_kernel" if n * (s.num_q_heads // s.num_kv_heads) > 64
+        "roofline": {"kernel": ("paged_multiquery_tc_kernel" if n * (s.num_q_heads // s.num_kv_heads) > 16
                                 else "paged_multiquery_bf16_kernel")
                                + (" + paged_multiquery_reduce_kernel" if need else ""),
                      "bound": "tensor" if tensor_bound else "hbm",

@@ -452,10 +452,12 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   const int64_t rows = static_cast<int64_t>(max_q_len) * group;
   // CTAs per (sequence, KV head) and resident CTAs per SM of the kernel that
-  // serves these rows: 16-row one-warp CTAs (~6 per SM), 64-row CTAs (2 per
-  // SM), or 128-row tcgen05 CTAs (1 per SM)
-  const int tile = rows <= 16 ? 16 : (rows <= 64 ? 64 : 128);
-  const int per_sm = rows <= 16 ? 6 : (rows <= 64 ? 2 : 1);
+  // serves these rows: 16- to 64-row mma.sync CTAs (6 to 2 per SM), or 128-row
+  // tcgen05 CTAs (1 per SM)
+  const bool tc = multiquery_uses_tc(static_cast<int>(rows > 0x7fffffff ? 0x7fffffff : rows));
+  const int nwc = multiquery_compute_warps(static_cast<int>(rows > 64 ? 64 : rows));
+  const int tile = tc ? 128 : 16 * nwc;
+  const int per_sm = tc ? 1 : multiquery_ctas_per_sm(nwc);
   const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * cdiv64(rows, tile);
   const int64_t want = 2LL * per_sm * sm_count();
   int64_t P = units >= want ? 1 : cdiv64(want, units > 0 ? units : 1);

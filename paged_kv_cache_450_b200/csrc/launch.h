@@ -75,10 +75,25 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
 }
 
 // Multi-query (prefill / verification) attention: bf16, head_dim 128, bs 16/32.
-// Up to 64 rows per (sequence, KV head) -- rows = queries x query heads of the
-// group -- run on the mma.sync kernel; more rows (prefill) on the tcgen05
-// kernel with 128-row tiles.
-inline bool multiquery_uses_tc(int rows_per_seq) { return rows_per_seq > 64; }
+// Up to 16 rows per (sequence, KV head) -- rows = queries x query heads of the
+// group -- run on the mma.sync kernel (one 16-row warp per CTA); more rows on
+// the tcgen05 kernel with 128-row tiles, whose time per KV tile does not
+// depend on how many of the rows are used (measured: 40 rows, 70B-GQA
+// verification, 2.70 TB/s on mma.sync with three 16-row warps, 3.56 TB/s on
+// tcgen05).
+#ifndef PKV_MQ_TC_MIN_ROWS
+#define PKV_MQ_TC_MIN_ROWS 16
+#endif
+inline bool multiquery_uses_tc(int rows_per_seq) { return rows_per_seq > PKV_MQ_TC_MIN_ROWS; }
+// Compute warps (16 rows each) per CTA of the mma.sync kernel, and its
+// resident CTAs per SM.
+inline int multiquery_compute_warps(int rows_per_seq) {
+  const int w = (rows_per_seq + 15) / 16;
+  return w < 1 ? 1 : (w > 4 ? 4 : w);
+}
+inline int multiquery_ctas_per_sm(int compute_warps) {
+  return compute_warps == 1 ? 6 : (compute_warps == 2 ? 4 : (compute_warps == 3 ? 3 : 2));
+}
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                                    int group, int rows_per_seq, bool reduce, cudaStream_t st);
 cudaError_t launch_multiquery_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,

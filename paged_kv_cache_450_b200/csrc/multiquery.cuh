@@ -4,8 +4,8 @@
 // and query i (position p = ctx - q_len + i) attends the logical tokens 0..p.
 //
 // FlashAttention-2 style on the tensor cores (mma.sync m16n8k16, bf16
-// operands, fp32 accumulation).  One CTA = 64 query rows (16 when a sequence
-// has at most 16 rows per KV head, as in verification) x one KV head x one
+// operands, fp32 accumulation).  One CTA = 16, 32, 48 or 64 query rows (the
+// rows of a (sequence, KV head), rounded up to 16, at most 64) x one KV head x one
 // split-context partition of one sequence; rows are (query i, query head g)
 // with g fastest, so grouped-query heads share every K/V tile.  A producer
 // warp streams the partition's blocks through a ring of TMA stages (K and V
@@ -26,8 +26,9 @@
 
 namespace pkv {
 
-// NWC_ compute warps of 16 rows each (4 for prefill-sized row counts, 1 for
-// verification-sized ones, so that small CTAs fill the SM).
+// NWC_ compute warps of 16 rows each: as many as the rows of a (sequence, KV
+// head) need, up to 4, so that CTAs are no larger than the work and more of
+// them fit on an SM.
 template <int BS, int NWC_ = 4, int NS_ = 0>
 struct MqTraits {
   static constexpr int D = 128;
@@ -38,7 +39,8 @@ struct MqTraits {
   static constexpr int TILE_BYTES = 2 * HALF_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int NS = NS_ > 0 ? NS_ : (NWC_ == 1 ? 3 : 4);
-  static constexpr int MIN_BLOCKS = NWC_ == 1 ? 6 : 2;
+  // resident CTAs per SM (registers: ~170 per thread at these counts)
+  static constexpr int MIN_BLOCKS = NWC_ == 1 ? 6 : (NWC_ == 2 ? 4 : (NWC_ == 3 ? 3 : 2));
   static constexpr int NT = BS / 16;
   static constexpr int STAGE_AREA = NS * STAGE_BYTES;
   static constexpr int BAR_BYTES = 2 * NS * 8;

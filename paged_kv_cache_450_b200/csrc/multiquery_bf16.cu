@@ -37,17 +37,20 @@ cudaError_t launch_multiquery_reduce(const MultiQueryParams& p, cudaStream_t st)
 
 cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                                    int group, int rows_per_seq, bool reduce, cudaStream_t st) {
-  // <= 16 rows per (sequence, kv head): one compute warp per CTA (16-row tiles)
-  const bool small = rows_per_seq <= 16;
-  const int n_qtiles = (rows_per_seq + (small ? 15 : 63)) / (small ? 16 : 64);
-  switch (p.block_size) {
-    case 16:
-      return small ? dispatch_mq_group<16, 1>(kmap, vmap, p, group, n_qtiles, reduce, st)
-                   : dispatch_mq_group<16, 4>(kmap, vmap, p, group, n_qtiles, reduce, st);
-    case 32:
-      return small ? dispatch_mq_group<32, 1>(kmap, vmap, p, group, n_qtiles, reduce, st)
-                   : dispatch_mq_group<32, 4>(kmap, vmap, p, group, n_qtiles, reduce, st);
-    default: return cudaErrorInvalidValue;
+  // one compute warp per 16 rows of a (sequence, KV head), at most four
+  const int nwc = multiquery_compute_warps(rows_per_seq);
+  const int n_qtiles = (rows_per_seq + 16 * nwc - 1) / (16 * nwc);
+  if (p.block_size != 16 && p.block_size != 32) return cudaErrorInvalidValue;
+  const bool b16 = p.block_size == 16;
+  switch (nwc) {
+    case 1: return b16 ? dispatch_mq_group<16, 1>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                       : dispatch_mq_group<32, 1>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 2: return b16 ? dispatch_mq_group<16, 2>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                       : dispatch_mq_group<32, 2>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    case 3: return b16 ? dispatch_mq_group<16, 3>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                       : dispatch_mq_group<32, 3>(kmap, vmap, p, group, n_qtiles, reduce, st);
+    default: return b16 ? dispatch_mq_group<16, 4>(kmap, vmap, p, group, n_qtiles, reduce, st)
+                        : dispatch_mq_group<32, 4>(kmap, vmap, p, group, n_qtiles, reduce, st);
   }
 }
 

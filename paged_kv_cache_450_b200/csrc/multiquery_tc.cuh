@@ -58,7 +58,7 @@ struct MqTcTraits {
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16)
   static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 bf16
-  static constexpr int NSK = 3, NSV = 2;     // K ring and V ring depth
+  static constexpr int NSK = 3, NSV = 2;  // K ring and V ring depth (K2 / V3 measured slower)
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
@@ -165,13 +165,14 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const uint32_t bar0 = base + T::BAR_OFF;
   const uint32_t q_full = bar0;
   auto k_full = [&](int s) { return bar0 + 8 * (1 + s); };
-  auto k_empty = [&](int s) { return bar0 + 8 * (4 + s); };
-  auto v_full = [&](int s) { return bar0 + 8 * (7 + s); };
-  auto v_empty = [&](int s) { return bar0 + 8 * (9 + s); };
+  auto k_empty = [&](int s) { return bar0 + 8 * (1 + T::NSK + s); };
+  auto v_full = [&](int s) { return bar0 + 8 * (1 + 2 * T::NSK + s); };
+  auto v_empty = [&](int s) { return bar0 + 8 * (1 + 2 * T::NSK + T::NSV + s); };
   // P-full and P.V-done barriers per token half h (each completes once per tile)
-  const uint32_t s_full = bar0 + 8 * 11, s_free = bar0 + 8 * 12, mma_done = bar0 + 8 * 17;
-  auto p_full = [&](int h) { return bar0 + 8 * (13 + h); };
-  auto pv_done = [&](int h) { return bar0 + 8 * (15 + h); };
+  constexpr int B2 = 1 + 2 * T::NSK + 2 * T::NSV;
+  const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1), mma_done = bar0 + 8 * (B2 + 6);
+  auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
+  auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < T::NSK; ++s) {

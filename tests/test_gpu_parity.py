@@ -412,6 +412,20 @@ def test_multiquery_queries_before_the_context_get_zero_rows():
 
 
 @pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv,q_lens", [(8, 4, (12, 3, 0, 7, 16, 1)), (8, 2, (12, 5, 1, 0, 9, 11)),
+                                           (4, 4, (64, 33, 1, 17, 0, 50)), (16, 2, (6, 5, 1, 2, 0, 3)),
+                                           (16, 2, (8, 7, 8, 1, 4, 2))])
+def test_multiquery_mid_sized_tiles(bs, hq, hkv, q_lens):
+    # 17 to 64 rows per (sequence, KV head): 2, 3 or 4 compute warps per mma.sync CTA
+    ctxs = (300, 40, 700, 2050, 16, 129)
+    spec = W.DecodeSpec("mqm", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs + hq + sum(q_lens), device=DEV)
+    for pt in (0, bs, 256):
+        _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} q_lens={q_lens} pt={pt}")
+
+
+@pytest.mark.parametrize("bs", [16, 32])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2)])
 def test_multiquery_prefill_sized_tiles(bs, hq, hkv):
     # more than 64 rows per (sequence, KV head): the 128-row tcgen05 kernel for
