@@ -277,25 +277,29 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the public API with pinned host buffers ----------
     host = {k: (getattr(w, k).cpu().pin_memory() if getattr(w, k) is not None else None)
             for k in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens", "copy_pairs")}
-    out_h = torch.empty(w.q.shape, dtype=w.q.dtype, pin_memory=True)
-    staging = torch.empty(pk.decode_step_staging_bytes(host["q"], host["new_k"], kc, host["block_tables"],
-                                                       host["copy_pairs"], pt), dtype=torch.uint8, device=dev)
+    # two steps in flight: the copies in of step i+1 overlap the kernels of step i
+    pipe = pk.HostStepPipeline(host["q"], host["new_k"], kc, host["block_tables"], host["copy_pairs"],
+                               partition_tokens=pt, depth=2, compute_stream=stream)
 
     def e2e_step():
-        pk.decode_step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
-                       host["context_lens"], kc, vc, w.scale, copy_pairs=host["copy_pairs"], k_scale=w.k_scale,
-                       v_scale=w.v_scale, out=out_h, staging=staging, partition_tokens=pt, stream=stream)
+        pipe.step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
+                  host["context_lens"], kc, vc, w.scale, copy_pairs=host["copy_pairs"], k_scale=w.k_scale,
+                  v_scale=w.v_scale)
 
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(args.warmup, 10)):
         e2e_step()
+    pipe.synchronize()
     torch.cuda.synchronize(dev)
     barrier(dev)
+    # the timed region opens on the copy-in stream (before the first copy) and closes on the
+    # copy-out stream after the last step's output has landed in host memory
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(pipe.copy_in)
     for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
+    e1.record(pipe.copy_out)
+    e1.synchronize()
     torch.cuda.synchronize(dev)
     barrier(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -339,7 +343,7 @@ def run_gpu(args, rank, world, local_rank):
                          "traffic": profile_traffic("paged_decode_" + s.name, s.name)},
             "e2e": {"value": round(total_kv / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": e2e_steps,
                     "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "paged_kv_cache_450_b200.decode_step -> pkv_decode_step_host (pinned host inputs and output)"},
+                    "api": "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async (pinned host inputs and output every step; two steps in flight: copies in, kernels, copies out on three streams)"},
             "gpu_launches": int(launches),
             "clocks": clk,
             "cpu_baseline": cpu,

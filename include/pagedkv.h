@@ -382,7 +382,8 @@ int pkv_swap_blocks(const int64_t* src_dst_pairs, int64_t num_pairs, const void*
  *                       bytes, 256-byte aligned, caller-owned; holds the copied
  *                       inputs, the output and the decode workspace.
  * Other arguments and errors: as pkv_paged_attention_decode / pkv_paged_kv_write /
- * pkv_kv_block_copy (without validation).  A negative code means nothing was enqueued.
+ * pkv_kv_block_copy (without validation).  Argument errors are returned before
+ * anything is enqueued.
  */
 int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
                          const int64_t* slot_mapping_host, int64_t num_tokens, const int32_t* block_tables_host,
@@ -396,6 +397,36 @@ int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host,
 size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                      int max_blocks_per_seq, int q_dtype, int cache_dtype, int partition_tokens,
                                      int64_t num_tokens, int64_t num_pairs);
+
+/*
+ * pkv_decode_step_host with its three parts on three streams, so that a caller
+ * can keep several steps in flight: the host -> device copies on
+ * copy_in_stream, the kernels on compute_stream (after those copies), the
+ * device -> host copy of the output on copy_out_stream (after the kernels).
+ * The library orders the parts of one step with events of its own; the order
+ * BETWEEN steps is the caller's: the kernels of consecutive steps follow each
+ * other on compute_stream, and a staging buffer (and its host output) may be
+ * reused only after the step that last used it has copied its output out.
+ *
+ * Source: as pkv_decode_step_host (the pages' decode step); the overlap of the
+ * next step's input copies with this step's kernels is this library's.
+ *
+ * staging_free_event  cudaEvent_t or NULL: copy_in_stream waits for it before
+ *                     the copies in (pass the done_event of the step that last
+ *                     used this staging buffer).
+ * done_event          cudaEvent_t or NULL: recorded on copy_out_stream after
+ *                     the copy out; out_host is valid once it has completed.
+ * All other arguments, the order of operations inside the step and the errors:
+ * as pkv_decode_step_host.  The three streams may be the same stream.
+ */
+int pkv_decode_step_host_async(void* out_host, const void* q_host, const void* k_host, const void* v_host,
+                               const int64_t* slot_mapping_host, int64_t num_tokens, const int32_t* block_tables_host,
+                               const int32_t* context_lens_host, const int64_t* copy_pairs_host, int64_t num_pairs,
+                               void* key_cache, void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads,
+                               int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                               float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                               void* staging, size_t staging_bytes, void* copy_in_stream, void* compute_stream,
+                               void* copy_out_stream, void* staging_free_event, void* done_event);
 
 /*
  * Prefix caching by hash chain (host side; no device work).

@@ -371,6 +371,65 @@ def decode_step(q, new_k, new_v, slot_mapping, block_tables, context_lens, key_c
                                       partition_tokens=partition_tokens, stream=st)
 
 
+class HostStepPipeline:
+    """Decode steps with host inputs and outputs, ``depth`` of them in flight
+    (pkv_decode_step_host_async): the copies in of step i+1 overlap the
+    kernels of step i, which run in order on the compute stream.
+
+    ``step(...)`` takes the same host tensors as :func:`decode_step` and
+    returns ``(out, done)``: ``out`` is a pinned host tensor owned by the
+    pipeline that holds the step's output once ``done`` (a CUDA event) has
+    completed, and that is overwritten ``depth`` steps later."""
+
+    def __init__(self, q, new_k, key_cache, block_tables, copy_pairs=None, partition_tokens: int = 0,
+                 depth: int = 2, compute_stream=None):
+        dev = key_cache.device
+        self.depth = int(depth)
+        self.partition_tokens = int(partition_tokens)
+        need = decode_step_staging_bytes(q, new_k, key_cache, block_tables, copy_pairs, partition_tokens)
+        self.staging = [torch.empty(max(need, 1), dtype=torch.uint8, device=dev) for _ in range(self.depth)]
+        self.outs = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(self.depth)]
+        self.compute = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev)
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.done = [torch.cuda.Event() for _ in range(self.depth)]
+        for e in self.done:  # create the events (torch makes them on first record)
+            e.record(self.compute)
+        self.used = [False] * self.depth
+        self.i = 0
+
+    def step(self, q, new_k, new_v, slot_mapping, block_tables, context_lens, key_cache, value_cache, scale: float, *,
+             copy_pairs=None, k_scale: float = 1.0, v_scale: float = 1.0):
+        host = [t for t in (q, new_k, new_v, slot_mapping, block_tables, context_lens, copy_pairs) if t is not None]
+        if any(t.device.type != "cpu" or not t.is_contiguous() for t in host):
+            raise ValueError("host inputs must all be contiguous CPU tensors")
+        _cuda(key_cache, value_cache)
+        k = self.i % self.depth
+        B, Hq, d = q.shape
+        NB, bs, Hkv, _ = key_cache.shape
+        T = 0 if new_k is None else new_k.shape[0]
+        n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+        ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        out, st = self.outs[k], self.staging[k]
+        with torch.cuda.device(key_cache.device):
+            _check(_lib.load().pkv_decode_step_host_async(
+                out.data_ptr(), q.data_ptr(), ptr(new_k), ptr(new_v), ptr(slot_mapping), T, block_tables.data_ptr(),
+                context_lens.data_ptr(), ptr(copy_pairs), n_pairs, key_cache.data_ptr(), value_cache.data_ptr(), B, Hq,
+                Hkv, d, bs, block_tables.shape[1], NB, float(scale), float(k_scale), float(v_scale), _dtype(q),
+                _dtype(key_cache), self.partition_tokens, st.data_ptr(), st.numel(),
+                ctypes.c_void_p(self.copy_in.cuda_stream), ctypes.c_void_p(self.compute.cuda_stream),
+                ctypes.c_void_p(self.copy_out.cuda_stream),
+                ctypes.c_void_p(self.done[k].cuda_event if self.used[k] else 0),
+                ctypes.c_void_p(self.done[k].cuda_event)), "decode_step_pipelined")
+        self.used[k] = True
+        self.i += 1
+        return out, self.done[k]
+
+    def synchronize(self):
+        for e in self.done:
+            e.synchronize()
+
+
 # --------------------------------------------------------------------------- #
 # prefix caching by hash chain (host side)
 # --------------------------------------------------------------------------- #

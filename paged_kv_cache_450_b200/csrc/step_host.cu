@@ -74,14 +74,30 @@ extern "C" size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, i
   return L.total;
 }
 
-extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
-                                    const int64_t* slot_mapping_host, int64_t num_tokens,
-                                    const int32_t* block_tables_host, const int32_t* context_lens_host,
-                                    const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
-                                    void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                                    int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
-                                    float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
-                                    void* staging, size_t staging_bytes, void* stream) {
+namespace {
+
+// Records an event on `from` and makes `to` wait for it (nothing when the
+// streams are the same).  The event is released at once; CUDA keeps it alive
+// until the wait has been satisfied.
+bool order(cudaStream_t from, cudaStream_t to) {
+  if (from == to) return true;
+  cudaEvent_t ev;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return false;
+  const bool ok = cudaEventRecord(ev, from) == cudaSuccess && cudaStreamWaitEvent(to, ev, 0) == cudaSuccess;
+  cudaEventDestroy(ev);
+  return ok;
+}
+
+// The step with its copies in on `in`, kernels on `comp`, copy out on `out`;
+// `wait_ev` (optional) gates the copies in, `done_ev` (optional) is recorded
+// after the copy out.
+int step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
+              const int64_t* slot_mapping_host, int64_t num_tokens, const int32_t* block_tables_host,
+              const int32_t* context_lens_host, const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
+              void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+              int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale, float v_scale, int q_dtype,
+              int cache_dtype, int partition_tokens, void* staging, size_t staging_bytes, cudaStream_t in,
+              cudaStream_t comp, cudaStream_t outs, cudaEvent_t wait_ev, cudaEvent_t done_ev) {
   if (num_seqs < 0 || num_tokens < 0 || num_pairs < 0) return PKV_ERR_BAD_SHAPE;
   if (num_seqs == 0 && num_tokens == 0 && num_pairs == 0) return PKV_OK;
   if (!staging || !key_cache || !value_cache) return PKV_ERR_NULL_POINTER;
@@ -99,11 +115,13 @@ extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const vo
     return PKV_ERR_BAD_DTYPE;
   if (staging_bytes < L.total) return PKV_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(staging);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t st = in;
+  void* stream = static_cast<void*>(comp);  // the kernels' stream
   const size_t es = dtype_bytes(q_dtype);
   const size_t qb = static_cast<size_t>(num_seqs) * num_q_heads * head_dim * es;
   const size_t kb = static_cast<size_t>(num_tokens) * num_kv_heads * head_dim * es;
-  // Copies in.
+  // Copies in (after the caller's event: the previous user of this staging buffer is done).
+  if (wait_ev && cudaStreamWaitEvent(in, wait_ev, 0) != cudaSuccess) return PKV_ERR_CUDA;
   if (!h2d(base + L.q, q_host, qb, st) || !h2d(base + L.k, k_host, kb, st) || !h2d(base + L.v, v_host, kb, st) ||
       !h2d(base + L.slots, slot_mapping_host, static_cast<size_t>(num_tokens) * sizeof(int64_t), st) ||
       !h2d(base + L.tables, block_tables_host,
@@ -111,6 +129,7 @@ extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const vo
       !h2d(base + L.lens, context_lens_host, static_cast<size_t>(num_seqs) * sizeof(int32_t), st) ||
       !h2d(base + L.pairs, copy_pairs_host, static_cast<size_t>(num_pairs) * 2 * sizeof(int64_t), st))
     return PKV_ERR_CUDA;
+  if (!order(in, comp)) return PKV_ERR_CUDA;
   int rc;
   if (num_pairs > 0) {
     const int64_t block_bytes =
@@ -134,7 +153,47 @@ extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const vo
                                     stream);
     if (rc) return rc;
     // Copy out.
-    if (cudaMemcpyAsync(out_host, base + L.out, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ERR_CUDA;
+    if (!order(comp, outs)) return PKV_ERR_CUDA;
+    if (cudaMemcpyAsync(out_host, base + L.out, qb, cudaMemcpyDeviceToHost, outs) != cudaSuccess) return PKV_ERR_CUDA;
+  } else if (!order(comp, outs)) {
+    return PKV_ERR_CUDA;
   }
+  if (done_ev && cudaEventRecord(done_ev, outs) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host, const void* v_host,
+                                    const int64_t* slot_mapping_host, int64_t num_tokens,
+                                    const int32_t* block_tables_host, const int32_t* context_lens_host,
+                                    const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
+                                    void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                                    float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                                    void* staging, size_t staging_bytes, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return step_host(out_host, q_host, k_host, v_host, slot_mapping_host, num_tokens, block_tables_host,
+                   context_lens_host, copy_pairs_host, num_pairs, key_cache, value_cache, num_seqs, num_q_heads,
+                   num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale, v_scale,
+                   q_dtype, cache_dtype, partition_tokens, staging, staging_bytes, st, st, st, nullptr, nullptr);
+}
+
+extern "C" int pkv_decode_step_host_async(void* out_host, const void* q_host, const void* k_host,
+                                          const void* v_host, const int64_t* slot_mapping_host, int64_t num_tokens,
+                                          const int32_t* block_tables_host, const int32_t* context_lens_host,
+                                          const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
+                                          void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads,
+                                          int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                          float scale, float k_scale, float v_scale, int q_dtype, int cache_dtype,
+                                          int partition_tokens, void* staging, size_t staging_bytes,
+                                          void* copy_in_stream, void* compute_stream, void* copy_out_stream,
+                                          void* staging_free_event, void* done_event) {
+  return step_host(out_host, q_host, k_host, v_host, slot_mapping_host, num_tokens, block_tables_host,
+                   context_lens_host, copy_pairs_host, num_pairs, key_cache, value_cache, num_seqs, num_q_heads,
+                   num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale, v_scale,
+                   q_dtype, cache_dtype, partition_tokens, staging, staging_bytes,
+                   static_cast<cudaStream_t>(copy_in_stream), static_cast<cudaStream_t>(compute_stream),
+                   static_cast<cudaStream_t>(copy_out_stream), static_cast<cudaEvent_t>(staging_free_event),
+                   static_cast<cudaEvent_t>(done_event));
 }

@@ -275,6 +275,42 @@ def test_host_buffer_step_matches_device_step_and_oracle(spec):
     assert_close(out_h.float().numpy().astype(np.float64), ref, *tol_for(w), what="host step")
 
 
+@pytest.mark.parametrize("depth", [1, 2, 3])
+def test_host_step_pipeline_matches_device_steps(depth):
+    """pkv_decode_step_host_async through HostStepPipeline: several steps in
+    flight (copies in, kernels and copies out on three streams), each step's
+    output equal to the device-side step on the same inputs."""
+    spec = W.PARALLEL_SAMPLING.with_(num_seqs=8, num_q_heads=8, num_kv_heads=8, sampling=(2, 4, 100, 1, 30))
+    w = W.make_decode_workload(spec, seed=16, device=DEV)
+    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+    steps = 7
+    g = torch.Generator(device="cpu").manual_seed(16)
+    qs = [torch.randn(w.q.shape, generator=g).to(w.q.dtype).pin_memory() for _ in range(steps)]
+    host = {k: pin(getattr(w, k)) for k in ("new_k", "new_v", "slot_mapping", "block_tables", "context_lens",
+                                            "copy_pairs")}
+    kc_h, vc_h = w.key_cache.clone(), w.value_cache.clone()
+    pipe = pk.HostStepPipeline(qs[0], host["new_k"], kc_h, host["block_tables"], host["copy_pairs"], depth=depth)
+    got = []
+    for i in range(steps):
+        out, done = pipe.step(qs[i], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
+                              host["context_lens"], kc_h, vc_h, w.scale, copy_pairs=host["copy_pairs"])
+        if i >= depth - 1:  # the oldest step in flight is complete once its event is
+            j = i - depth + 1
+            pipe.done[j % depth].synchronize()
+            got.append(pipe.outs[j % depth].clone())
+    pipe.synchronize()
+    for j in range(steps - depth + 1, steps):
+        got.append(pipe.outs[j % depth].clone())
+    # the same steps on the device: the copies and the write are idempotent, only q changes
+    kc_d, vc_d = w.key_cache.clone(), w.value_cache.clone()
+    for i in range(steps):
+        ref = pk.decode_step(qs[i].to(DEV), w.new_k, w.new_v, w.slot_mapping, w.block_tables, w.context_lens, kc_d,
+                             vc_d, w.scale, copy_pairs=w.copy_pairs)
+        torch.cuda.synchronize()
+        assert torch.equal(got[i], ref.cpu()), f"step {i}"
+    assert torch.equal(kc_h, kc_d) and torch.equal(vc_h, vc_d)
+
+
 def test_full_size_bf16_gqa_sampled():
     w = W.make_decode_workload(W.SPECS["gqa70b_bf16_b128_ctx8k"], seed=0, device=DEV)
     check_step(w, rows=sample_rows(w, 512), what="gqa70b_bf16_b128_ctx8k")
