@@ -48,6 +48,39 @@ def logical_seqs(rng, ctxs, Hkv, d):
 # paged decode attention == dense attention over the logical K/V
 # --------------------------------------------------------------------------- #
 
+def test_decode_equals_python_double_loop_brute_force():
+    """Tiny cases against plain Python: every score, the max, math.exp and the
+    weighted sum written out element by element over explicitly gathered
+    rows (no library routine at all)."""
+    rng = np.random.default_rng(30)
+    for trial in range(6):
+        B, Hkv, g, d, bs = int(rng.integers(1, 5)), int(rng.integers(1, 3)), int(rng.choice([1, 2])), 8, 4
+        Hq = Hkv * g
+        ctxs = [int(c) for c in rng.integers(1, 41, B)]
+        ks, vs = logical_seqs(rng, ctxs, Hkv, d), logical_seqs(rng, ctxs, Hkv, d)
+        nb = sum(-(-c // bs) for c in ctxs) + 3
+        order = rng.permutation(nb)
+        tk, kp = page_logical(ks, bs, rng, num_blocks=nb, order=order)
+        _, vp = page_logical(vs, bs, rng, num_blocks=nb, order=order)
+        q = rng.standard_normal((B, Hq, d)).astype(np.float32)
+        scale = float(np.float32(0.3))  # the scale crosses the C interface as a float
+        out = oracle.paged_attention_decode(q, kp, vp, tk, np.array(ctxs, np.int32), scale=scale)
+        for b in range(B):
+            for h in range(Hq):
+                kh = h // g
+                rows_k, rows_v = [], []
+                for t in range(ctxs[b]):  # gather through the block table, by hand
+                    blk = int(tk[b, t // bs])
+                    rows_k.append([float(x) for x in kp[blk, t % bs, kh]])
+                    rows_v.append([float(x) for x in vp[blk, t % bs, kh]])
+                sc = [scale * sum(float(q[b, h, i]) * kr[i] for i in range(d)) for kr in rows_k]
+                mx = max(sc)
+                w = [math.exp(x - mx) for x in sc]
+                den = sum(w)
+                ref = [sum(w[t] * rows_v[t][i] for t in range(len(w))) / den for i in range(d)]
+                assert np.allclose(out[b, h], ref, rtol=1e-12, atol=1e-12), (trial, b, h)
+
+
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_decode_equals_dense_sdpa_fp32(bs):
     rng = np.random.default_rng(1)
