@@ -1,5 +1,6 @@
 // multiquery_tc.cuh -- multi-query paged attention on the tcgen05 tensor cores
-// for prefill-sized query counts (more than 64 rows per sequence and KV head).
+// for more than 16 rows (queries x query heads of a group) per sequence and
+// KV head: chunked prefill, grouped-query draft verification.
 //
 // Same operation as multiquery.cuh (causal over the paged cache, queries are
 // the sequence's last q_len positions), written for the Blackwell MMA:
@@ -40,8 +41,9 @@
 //   warp 9     MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
-// Every wait is bounded (2 s); on a timeout the status bit is set, the loops
-// stop, in-flight work is drained with bounded waits and TMEM is freed.
+// Every wait is bounded (2 s); on a timeout the status bit is set, the
+// producer and issuer loops stop, the softmax warps skip their remaining
+// waits, in-flight work is drained with bounded waits and TMEM is freed.
 #pragma once
 
 #include "common.cuh"
@@ -67,8 +69,8 @@ struct MqTcTraits {
   // mma_done (the pairs: one per token half)
   static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
-  static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [3 slots][2 halves][128 rows]
-  static constexpr int IDS_OFF = XCH_OFF + 3 * 2 * 128 * 4;
+  static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [4][128 rows]: m_0, m_1, l_0, l_1
+  static constexpr int IDS_OFF = XCH_OFF + 4 * 128 * 4;
   static constexpr int THREADS = 352;
   static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
   static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O_0 128 | O_1 128 | P hi 0,1 (32 + 32), lo 0,1 (32 + 32)
