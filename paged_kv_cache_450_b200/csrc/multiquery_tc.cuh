@@ -152,17 +152,6 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const int nt = (tok_end - tok_begin + T::TOK - 1) / T::TOK;
   const int nb = (tok_end - tok_begin + BS - 1) / BS;
 
-  int local_bad = 0;
-  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-    int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb + i];
-    if (id < 0 || id >= p.num_blocks) {
-      set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
-      id = -1;
-      local_bad = 1;
-    }
-    ids[i] = id;
-  }
-  const bool any_bad = __syncthreads_or(local_bad) != 0;  // (also orders the ids before their use)
   const uint32_t base = smem_u32(data);
   const uint32_t bar0 = base + T::BAR_OFF;
   const uint32_t q_full = bar0;
@@ -175,25 +164,64 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1), mma_done = bar0 + 8 * (B2 + 6);
   auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
   auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < T::NSK; ++s) {
-      mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
+  const uint64_t policy = l2_policy_evict_first();
+  const int* table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb;
+  if (warp == T::W_K) {
+    // The K producer starts the first loads before the CTA-wide set-up: it
+    // initialises the barriers (no other thread touches them before the
+    // barrier below), then fetches Q and the first K tile itself.
+    if (lane == 0) {
+      mbar_init(q_full, 1);
+      for (int s = 0; s < T::NSK; ++s) {
+        mbar_init(k_full(s), 1);
+        mbar_init(k_empty(s), 1);
+      }
+      for (int s = 0; s < T::NSV; ++s) {
+        mbar_init(v_full(s), 1);
+        mbar_init(v_empty(s), 1);
+      }
+      mbar_init(s_full, 1);
+      mbar_init(s_free, 8);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(p_full(h), 4);
+        mbar_init(pv_done(h), 1);
+      }
+      mbar_init(mma_done, 1);
+      fence_barrier_init();
+      mbar_arrive_expect_tx(q_full, T::TILE);
+      tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
+      tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, hk * G, q0 + qt * QPT);
     }
-    for (int s = 0; s < T::NSV; ++s) {
-      mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
+    // K tile 0: lane i < blocks of the tile reads block id i
+    int id = -1;
+    if (lane < min(nb, T::BPT)) {
+      id = table[lane];
+      if (id < 0 || id >= p.num_blocks) id = -1;  // (reported by the scan below)
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(p_full(h), 4);
-      mbar_init(pv_done(h), 1);
+    const unsigned valid = __ballot_sync(kFullMask, id >= 0);
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(__popc(valid)) * 2u * BS * 128u;
+      if (bytes) mbar_arrive_expect_tx(k_full(0), bytes); else mbar_arrive(k_full(0));
     }
-    mbar_init(mma_done, 1);
-    fence_barrier_init();
+    __syncwarp();
+    if (id >= 0) {
+      const uint32_t dst = base + T::K_OFF + lane * BS * 128;
+      tma_load_4d(dst, &kmap, k_full(0), 0, hk, 0, id, policy);
+      tma_load_4d(dst + T::HALF, &kmap, k_full(0), 64, hk, 0, id, policy);
+    }
   }
+
+  int local_bad = 0;
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    int id = table[i];
+    if (id < 0 || id >= p.num_blocks) {
+      set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
+      id = -1;
+      local_bad = 1;
+    }
+    ids[i] = id;
+  }
+  const bool any_bad = __syncthreads_or(local_bad) != 0;  // (also orders the ids before their use)
   if (warp == T::W_K) {
     __syncwarp();
     tmem_alloc(base + T::SLOT_OFF, T::TMEM_COLS);
@@ -214,14 +242,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
       const int ns = is_k ? T::NSK : T::NSV;
       const CUtensorMap* map = is_k ? &kmap : &vmap;
       const uint32_t area = base + (is_k ? T::K_OFF : T::V_OFF);
-      const uint64_t policy = l2_policy_evict_first();
-      if (is_k) {
-        mbar_arrive_expect_tx(q_full, T::TILE);
-        tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
-        tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, hk * G, q0 + qt * QPT);
-      }
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      int issued = is_k ? 1 : 0;  // Q and K tile 0 were issued in the prologue
+      for (int j = issued; j < nt; ++j) {
         const int s = j % ns, use = j / ns;
         const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
         const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
