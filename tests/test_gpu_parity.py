@@ -511,6 +511,54 @@ def test_multiquery_guards_bad_block_ids(q_lens):
     assert_close(f64(out).reshape(-1, 128)[rows], ref, *TOL_BF16, what="unaffected sequence")
 
 
+def test_multiquery_long_context_largest_partition():
+    # a 16384-token partition (1024 block ids of bs 16 in the tcgen05 kernel's shared memory) and a
+    # context split in two by it
+    ctxs = (20000, 16384, 300)
+    spec = W.DecodeSpec("mqlong", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.05))
+    mw = W.make_multiquery_workload(spec, (40, 17, 300), seed=23, device=DEV)
+    T = int(mw.query_start_loc[-1])
+    rows = np.unique(np.concatenate([np.arange(0, T * 8, 7), [T * 8 - 1]]))
+    for pt in (16384, 0):
+        _mq_check(mw, partition_tokens=pt, rows=rows, what=f"long context pt={pt}")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_multiquery_random_shapes(seed):
+    """Seeded random mixes: head grouping, block size, context and query lengths (zero, one, a few,
+    a full prefill), partition length -- both multi-query kernels."""
+    rng = np.random.default_rng(100 + seed)
+    hkv = int(rng.choice([1, 2, 4]))
+    g = int(rng.choice([1, 2, 4, 8]))
+    bs = int(rng.choice([16, 32]))
+    B = int(rng.integers(1, 7))
+    ctxs = tuple(int(c) for c in rng.integers(1, 1500, B))
+    q_lens = tuple(int(min(c, rng.choice([0, 1, 3, 9, 40, 200, c]))) for c in ctxs)
+    spec = W.DecodeSpec("mqrand", B, hkv * g, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=200 + seed, device=DEV)
+    pt = int(rng.choice([0, bs, 4 * bs, 512]))
+    _mq_check(mw, partition_tokens=pt, what=f"seed={seed} g={g} hkv={hkv} bs={bs} ctxs={ctxs} q_lens={q_lens} pt={pt}")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_multiquery_random_verify_shapes(seed):
+    """Seeded random verification mixes with at most 16 rows per (sequence, KV head): the mma.sync kernel."""
+    rng = np.random.default_rng(300 + seed)
+    hkv = int(rng.choice([1, 2, 4]))
+    g = int(rng.choice([1, 2, 4, 8]))
+    bs = int(rng.choice([16, 32]))
+    B = int(rng.integers(1, 9))
+    ctxs = tuple(int(c) for c in rng.integers(1, 3000, B))
+    q_lens = tuple(int(min(c, rng.integers(0, 16 // g + 1))) for c in ctxs)
+    spec = W.DecodeSpec("mqrandv", B, hkv * g, hkv, 128, bs, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=400 + seed, device=DEV)
+    pt = int(rng.choice([0, bs, 4 * bs, 512]))
+    _mq_check(mw, partition_tokens=pt, what=f"seed={seed} g={g} hkv={hkv} bs={bs} ctxs={ctxs} q_lens={q_lens} pt={pt}")
+
+
 def test_multiquery_prefill_chunk_after_prefix():
     spec = W.LLAMA7B.with_(num_seqs=3, num_q_heads=8, num_kv_heads=8, ctx=("list", (600, 300, 1030)))
     mw = W.make_multiquery_workload(spec, (300, 300, 512), seed=3, device=DEV)
