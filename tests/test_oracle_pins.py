@@ -602,6 +602,42 @@ def test_multiquery_queries_before_the_context_get_zero_rows():
     assert np.array_equal(out[2:], tail)
 
 
+def test_multiquery_equals_python_double_loop_brute_force():
+    """Tiny causal cases against plain Python: for query i of a sequence with
+    q_len queries and context c, the keys 0 .. c - q_len + i, scores, max,
+    math.exp and the weighted sum written out element by element."""
+    rng = np.random.default_rng(31)
+    for trial in range(5):
+        B, Hkv, g, d, bs = int(rng.integers(1, 4)), int(rng.integers(1, 3)), int(rng.choice([1, 2])), 8, 4
+        Hq = Hkv * g
+        ctxs = [int(c) for c in rng.integers(1, 30, B)]
+        qlens = [int(rng.integers(0, c + 1)) for c in ctxs]
+        ks, vs = logical_seqs(rng, ctxs, Hkv, d), logical_seqs(rng, ctxs, Hkv, d)
+        nb = sum(-(-c // bs) for c in ctxs) + 2
+        order = rng.permutation(nb)
+        tk, kp = page_logical(ks, bs, rng, num_blocks=nb, order=order)
+        _, vp = page_logical(vs, bs, rng, num_blocks=nb, order=order)
+        qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+        q = rng.standard_normal((int(qsl[-1]), Hq, d)).astype(np.float32)
+        scale = float(np.float32(0.25))
+        out = oracle.paged_attention_multiquery(q, qsl, kp, vp, tk, np.array(ctxs, np.int32), scale=scale)
+        for b in range(B):
+            for i in range(qlens[b]):
+                pos = ctxs[b] - qlens[b] + i
+                for h in range(Hq):
+                    rows_k, rows_v = [], []
+                    for t in range(pos + 1):
+                        blk = int(tk[b, t // bs])
+                        rows_k.append([float(x) for x in kp[blk, t % bs, h // g]])
+                        rows_v.append([float(x) for x in vp[blk, t % bs, h // g]])
+                    qv = [float(x) for x in q[qsl[b] + i, h]]
+                    sc = [scale * sum(qv[e] * kr[e] for e in range(d)) for kr in rows_k]
+                    mx = max(sc)
+                    w = [math.exp(x - mx) for x in sc]
+                    ref = [sum(w[t] * rows_v[t][e] for t in range(len(w))) / sum(w) for e in range(d)]
+                    assert np.allclose(out[qsl[b] + i, h], ref, rtol=1e-12, atol=1e-12), (trial, b, i, h)
+
+
 def test_multiquery_with_one_query_per_sequence_is_decode():
     rng = np.random.default_rng(22)
     ctxs = [1, 33, 70]
