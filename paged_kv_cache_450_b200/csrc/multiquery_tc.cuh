@@ -388,17 +388,27 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         m = mx;
       }
       const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
-      // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add
+      // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add, and at once the
+      // row's half of P as packed pairs (tokens 2k, 2k+1 in word k): a high part (the top 16 bits of
+      // the fp32 value: truncation) and the residual (exact in fp32, then truncated to its top 16
+      // bits), ~16 significant bits per probability.  One loop, so the special-function unit (ex2)
+      // and the integer / FMA pipes (packing) work side by side; the stores to TMEM wait below.
       const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
       float2 sum4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
+      uint32_t phi[32], plo[32];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), qk2, nm2);
-        sv[c] = fast_exp2(x.x);
-        sv[c + 1] = fast_exp2(x.y);
-        sum4[(c >> 1) & 3] = __fadd2_rn(sum4[(c >> 1) & 3], make_float2(sv[c], sv[c + 1]));
+      for (int k = 0; k < 32; ++k) {
+        const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
+        const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
+        sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
+        const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
+        // residual = value - its truncation (the negated truncation is one logic op)
+        const float2 rr = __fadd2_rn(make_float2(a, bb), make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
+                                                                      __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
+        phi[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
+        plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
       }
       const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
       l += s2.x + s2.y;
@@ -433,21 +443,14 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         }
         fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
       }
-      // this half of row r of P into TMEM lane r: tokens (2k, 2k+1) in column k, as a high part (the
-      // top 16 bits of the fp32 value: truncation) and the residual (exact in fp32, then truncated to
-      // its top 16 bits): ~16 significant bits per probability, integer / FMA-pipe work only
+      // this half of row r of P into TMEM lane r
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float a = sv[32 * c + 2 * k], bb = sv[32 * c + 2 * k + 1];
-          const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
-          // residual = value - its truncation (the negated truncation is one logic op)
-          const float2 rr = __fadd2_rn(make_float2(a, bb), make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
-                                                                        __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
-          hi[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
-          lo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+          hi[k] = phi[16 * c + k];
+          lo[k] = plo[16 * c + k];
         }
         tmem_st16(tmem_phi(h) + lane_off + 16 * c, hi);
         tmem_st16(tmem_plo(h) + lane_off + 16 * c, lo);
