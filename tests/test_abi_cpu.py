@@ -105,6 +105,44 @@ def test_partition_choice_and_workspace_size():
         pk.decode_partition_tokens(1, 1, 1, 128, 16, 100, bf16, 40)
 
 
+def test_multiquery_partition_and_workspace():
+    lib = _lib.load()
+    PT, WS = lib.pkv_multiquery_partition_tokens, lib.pkv_multiquery_workspace_bytes
+    # (num_seqs, max_q_len, Hq, Hkv, bs, max_blocks, partition_tokens)
+    # prefill-sized rows, 1024 tcgen05 CTAs >= two waves: one partition over the longest context
+    assert PT(8, 512, 32, 32, 16, 128, 0) == 2048
+    assert WS(8, 8 * 512, 512, 32, 32, 128, 16, 128, 0) == 0
+    # GQA verification (40 rows per KV head, tcgen05): 64 x 8 = 512 CTAs already fill two waves of
+    # one CTA per SM -> one partition; 8 sequences -> split in 256-token multiples
+    assert PT(64, 5, 64, 8, 16, 512, 0) == 8192
+    assert WS(64, 64 * 5, 5, 64, 8, 128, 16, 512, 0) == 0
+    pt = PT(8, 5, 64, 8, 16, 512, 0)
+    assert pt % 256 == 0 and 256 <= pt < 8192
+    P = -(-512 * 16 // pt)
+    rows = 8 * 5 * 64 * P
+    assert WS(8, 8 * 5, 5, 64, 8, 128, 16, 512, 0) == ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
+    # MHA verification (5 rows): 16-row CTAs, 6 per SM
+    assert PT(64, 5, 32, 32, 16, 128, 0) > 0
+    # explicit partition lengths: a multiple of the block size up to 16384 tokens
+    assert PT(1, 4, 8, 8, 16, 100, 48) == 48
+    ERR_HEAD_DIM, ERR_BAD_DTYPE, ERR_BLOCK_SIZE, ERR_HEAD_GROUPING, ERR_BAD_SHAPE, ERR_PARTITION = -3, -2, -4, -5, -7, -13
+    assert PT(1, 4, 8, 8, 16, 100, 40) == ERR_PARTITION
+    assert PT(1, 4, 8, 8, 16, 100, 16400) == ERR_PARTITION
+    # argument errors
+    assert PT(1, 4, 8, 8, 8, 100, 0) == ERR_BLOCK_SIZE
+    assert PT(1, 4, 8, 3, 16, 100, 0) == ERR_HEAD_GROUPING
+    assert PT(-1, 4, 8, 8, 16, 100, 0) == ERR_BAD_SHAPE
+    # a call with no work launches nothing and needs nothing
+    assert lib.pkv_paged_attention_multiquery(None, None, None, None, None, None, None, 0, 0, 0, 8, 8, 128, 16, 10,
+                                              100, 0.1, pk.DTYPE_BF16, pk.DTYPE_BF16, 0, None, 0, 0, None) == 0
+    # unsupported shapes are refused before anything else happens
+    args = [ctypes.c_void_p(16)] * 7 + [1, 4, 4, 8, 8]
+    assert lib.pkv_paged_attention_multiquery(*args, 64, 16, 10, 100, 0.1, pk.DTYPE_BF16, pk.DTYPE_BF16, 0, None, 0,
+                                              0, None) == ERR_HEAD_DIM
+    assert lib.pkv_paged_attention_multiquery(*args, 128, 16, 10, 100, 0.1, pk.DTYPE_F32, pk.DTYPE_BF16, 0, None,
+                                              0, 0, None) == ERR_BAD_DTYPE
+
+
 def test_ops_refuse_cpu_tensors():
     import torch
     x = torch.zeros(2, 2, 128)
