@@ -232,7 +232,9 @@ int pkv_paged_attention_decode_static(void* out, const void* q, const void* key_
  * splits the longest possible context (max_blocks_per_seq * block_size) into
  * at least 4 partitions and gives at least one CTA per resident slot of the
  * kernel; a single partition when that context is 512 tokens or less.
- * Returns a negative PKV_ERR_* code for unsupported arguments.
+ * Returns a negative PKV_ERR_* code for unsupported arguments.  (This and the
+ * other sizing helpers below are this library's; the pages have no
+ * counterpart: the split-context partition is its design for long contexts.)
  */
 int pkv_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                 int max_blocks_per_seq, int cache_dtype, int partition_tokens);
@@ -307,12 +309,19 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
                                    int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
                                    int validate, void* stream);
 
-/* Split-context partition length pkv_paged_attention_multiquery uses (partition_tokens
- * if non-zero, else automatic); negative PKV_ERR_* for unsupported arguments. */
+/* Split-context partition length pkv_paged_attention_multiquery uses:
+ * partition_tokens if non-zero (a multiple of block_size, at most 16384), else
+ * automatic -- one partition when (sequences x KV heads x query-row tiles of
+ * the kernel that serves these rows) already gives two waves of its resident
+ * CTAs, else the longest context split so that it does, in multiples of 256
+ * tokens.  Negative PKV_ERR_* for unsupported arguments.  A sizing helper of
+ * this library (no counterpart on the pages). */
 int pkv_multiquery_partition_tokens(int num_seqs, int max_q_len, int num_q_heads, int num_kv_heads, int block_size,
                                     int max_blocks_per_seq, int partition_tokens);
 
-/* Workspace bytes pkv_paged_attention_multiquery needs. */
+/* Workspace bytes pkv_paged_attention_multiquery needs (0 when no context is
+ * split): float (m, l) then, at a 256-byte boundary, float o[d] per (query
+ * token, query head, partition).  A sizing helper of this library. */
 size_t pkv_multiquery_workspace_bytes(int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
                                       int head_dim, int block_size, int max_blocks_per_seq, int partition_tokens);
 
@@ -393,7 +402,8 @@ int pkv_decode_step_host(void* out_host, const void* q_host, const void* k_host,
                          float k_scale, float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
                          void* staging, size_t staging_bytes, void* stream);
 
-/* Staging bytes pkv_decode_step_host needs for these arguments. */
+/* Staging bytes pkv_decode_step_host / _async need for these arguments (a
+ * sizing helper of this library). */
 size_t pkv_decode_step_staging_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                      int max_blocks_per_seq, int q_dtype, int cache_dtype, int partition_tokens,
                                      int64_t num_tokens, int64_t num_pairs);
@@ -478,11 +488,14 @@ int64_t pkv_prefix_cache_evict(void* cache, int64_t max_evict, int32_t* evicted_
 
 /*
  * Reads the current device's status word (PKV_STATUS_* bits) into *status,
- * after synchronising `stream`; clears it if `clear` != 0.
+ * after synchronising `stream`; clears it if `clear` != 0.  The library's
+ * failure reporting (in-kernel guards and bounded waits set the bits); the
+ * pages have no counterpart.
  */
 int pkv_device_status(unsigned* status, int clear, void* stream);
 
-/* Number of kernel launches this library issued on this process (all devices). */
+/* Number of kernel launches this library issued on this process (all devices):
+ * the library's own accounting, no counterpart on the pages. */
 uint64_t pkv_launch_count(void);
 
 #ifdef __cplusplus
