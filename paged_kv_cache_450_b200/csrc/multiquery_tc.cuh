@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
+      const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
+      const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
       bool ok = mbar_wait_bounded(q_full, 0, p.status);
       // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1)
       for (int j = 0; ok && j <= nt; ++j) {
@@ -278,12 +280,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
           if (!(ok = mbar_wait_bounded(k_full(sk), (j / T::NSK) & 1, p.status))) break;
           if (j > 0 && !(ok = mbar_wait_bounded(s_free, (j - 1) & 1, p.status))) break;
           tc_fence_after();
-          const uint32_t ka = base + T::K_OFF + sk * T::TILE;
+          // descriptors differ only in the start-address field (address >> 4 in the low bits, all
+          // addresses below 256 KB): the base descriptors plus offsets
+          const uint64_t kd0 = qd0 + ((T::K_OFF - T::Q_OFF + sk * T::TILE) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * T::HALF + (kk & 3) * 32;
-            tc_mma_bf16(tmem_s, smem_desc_sw128(base + T::Q_OFF + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                        idesc_s, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * T::HALF + (kk & 3) * 32) >> 4;
+            tc_mma_bf16(tmem_s, qd0 + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           tc_commit(s_full);
           tc_commit(k_empty(sk));
@@ -291,13 +294,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         if (j > 0) {
           const int jj = j - 1, sv = jj % T::NSV;
           if (!(ok = mbar_wait_bounded(v_full(sv), (jj / T::NSV) & 1, p.status))) break;
-          const uint32_t va = base + T::V_OFF + sv * T::TILE;
+          const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
           for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
             if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
-              const uint64_t vdesc = smem_desc_sw128(va + (64 * h + 16 * kk) * 128, T::HALF, 1024);
+              const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
               tc_mma_bf16_tmem_a(tmem_o(h), tmem_phi(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
               tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
             }
