@@ -17,6 +17,8 @@
 //                 ldmatrix.trans; P as bf16 hi + lo, ~16 bits per weight)
 // The online softmax per row keeps a reference max as in the decode kernels.
 // Partitions write (m, l, o) partials merged by paged_multiquery_reduce_kernel.
+// The dispatch (launch.h) sends it up to 16 rows per (sequence, KV head); more
+// rows go to the tcgen05 kernel (multiquery_tc.cuh).
 #pragma once
 
 #include "decode.cuh"
