@@ -57,10 +57,10 @@ def test_native_hashes_match_reference():
             assert [int(x) for x in got] == ref.block_hashes(toks.tolist(), bs, parent, extra)
 
 
-def test_native_cache_matches_reference_on_random_operations():
-    rng = np.random.default_rng(2)
-    bs = 4
-    native, oracle_cache = pk.PrefixCache(bs, 24), ref.RefPrefixCache(bs, 24)
+@pytest.mark.parametrize("seed,bs,capacity", [(2, 4, 24), (3, 4, 8), (4, 2, 64), (5, 8, 12), (6, 1, 40)])
+def test_native_cache_matches_reference_on_random_operations(seed, bs, capacity):
+    rng = np.random.default_rng(seed)
+    native, oracle_cache = pk.PrefixCache(bs, capacity), ref.RefPrefixCache(bs, capacity)
     prompts = [rng.integers(0, 6, bs * rng.integers(1, 7)).tolist() for _ in range(12)]
     for p in prompts[6:]:                      # share prefixes between some prompts
         p[:bs * 2] = prompts[0][:bs * 2] if len(prompts[0]) >= 2 * bs else p[:bs * 2]
