@@ -71,6 +71,8 @@ extern "C" {
 #define PKV_STATUS_BAD_SLOT 0x4u        /* write met a slot >= num_blocks * block_size */
 #define PKV_STATUS_BAD_COPY_PAIR 0x8u   /* block copy met an id outside [0, num_blocks) */
 #define PKV_STATUS_WAIT_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up */
+#define PKV_STATUS_BAD_QUERY_LOC 0x20u  /* multi-query met query_start_loc entries outside [0, total_q] or a
+                                           q_len above max_q_len: that sequence's rows are left unwritten */
 
 /*
  * Human-readable name of a PKV_* status code (static storage).
@@ -201,9 +203,11 @@ int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const v
  *
  * - Every GPU on which the library's device code is loaded holds that array
  *   until the process exits.
- * - The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make
- *   that first call before any stream capture.
+ * - The first call on each device that needs partials looks up the array's
+ *   device address (cudaGetSymbolAddress, with that device current) and
+ *   caches it; make that first call before any stream capture.  Calls that
+ *   need no partials (pkv_decode_workspace_bytes() == 0, e.g. num_seqs == 0
+ *   or one partition per sequence) do not touch the array.
  * - All calls on a device share the array, and it keeps the partials of the
  *   last call.  Nothing in it has to start at zero.  Calls that may run at
  *   the same time on the GPU (other streams, or host threads without an
@@ -212,7 +216,8 @@ int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const v
  * - A call whose partials need more than PKV_DECODE_STATIC_SCRATCH_BYTES
  *   (pkv_decode_workspace_bytes() for the same call) returns
  *   PKV_ERR_WORKSPACE and launches nothing; a larger partition_tokens lowers
- *   the need.
+ *   the need.  Argument errors take precedence over it, in the order
+ *   pkv_paged_attention_decode checks them.
  * Other errors: as pkv_paged_attention_decode.
  */
 #define PKV_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
@@ -291,7 +296,11 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
  *                   <= context_lens[b] (validate checks all of this; without
  *                   validate, the first q_len_b - context_lens[b] queries of a
  *                   sequence with more queries than context tokens sit at
- *                   negative positions and get zero rows).
+ *                   negative positions and get zero rows).  Independently of
+ *                   validate, the kernels skip a sequence whose rows would fall
+ *                   outside [0, total_q) or whose q_len_b exceeds max_q_len:
+ *                   nothing of it is read or written (its rows of out keep their
+ *                   previous bytes) and PKV_STATUS_BAD_QUERY_LOC is set.
  * workspace         device scratch of pkv_multiquery_workspace_bytes(...) bytes
  *                   (same arguments; 0 when no split is needed), 256-byte aligned.
  * Supported: bf16 q and caches, head_dim 128, block_size 16 or 32, 1/2/4/8

@@ -29,6 +29,7 @@ STATUS_BAD_CONTEXT = 0x2
 STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
+STATUS_BAD_QUERY_LOC = 0x20
 
 __all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_multiquery", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",

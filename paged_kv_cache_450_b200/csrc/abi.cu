@@ -567,6 +567,7 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   p.partition_blocks = pt / block_size;
   p.max_partitions = P;
   p.total_q = total_q;
+  p.max_q_len = max_q_len;
   p.q_scale = scale * kLog2e;
   const int rows_per_seq = max_q_len * group;
   if (rows_per_seq <= 0) return PKV_OK;

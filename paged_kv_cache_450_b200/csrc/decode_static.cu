@@ -58,10 +58,19 @@ extern "C" int pkv_paged_attention_decode_static(void* out, const void* q, const
                                                  int max_blocks_per_seq, int64_t num_blocks, float scale,
                                                  float k_scale, float v_scale, int q_dtype, int cache_dtype,
                                                  int partition_tokens, void* stream) {
-  // Refuse, before touching the device, any call whose partials would not fit.
   const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                                  max_blocks_per_seq, cache_dtype, partition_tokens);
-  if (need > kScratchBytes) return PKV_ERR_WORKSPACE;
+  if (need == 0 || need > kScratchBytes) {
+    // No partials (one partition per sequence, an empty batch or arguments the
+    // decode rejects), or more than the array holds: the workspace entry point
+    // without a workspace gives the same answer -- its argument errors first,
+    // PKV_OK for an empty batch, PKV_ERR_WORKSPACE (nothing launched) when
+    // partials are needed -- and the array's address is not looked up.
+    return pkv_paged_attention_decode(out, q, key_cache, value_cache, block_tables, context_lens, num_seqs,
+                                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                      num_blocks, scale, k_scale, v_scale, q_dtype, cache_dtype, partition_tokens,
+                                      nullptr, 0, /*validate=*/0, stream);
+  }
   int status = PKV_OK;
   void* scratch = scratch_address(&status);
   if (!scratch) return status;

@@ -64,8 +64,11 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
   const int Hkv = p.num_kv_heads;
   const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = p.query_start_loc[b];
-  const int q_len = p.query_start_loc[b + 1] - q0;
+  int q0, q_len;
+  if (!query_rows_ok(p, b, q0, q_len)) {  // before any load or store
+    if (threadIdx.x == 0) set_status(p.status, PKV_STATUS_BAD_QUERY_LOC);
+    return;
+  }
   const int rows_total = q_len * G;
   if (q_len <= 0 || qt * T::ROWS >= rows_total) return;
   const int max_ctx = p.max_blocks_per_seq * BS;
@@ -343,12 +346,13 @@ __global__ void __launch_bounds__(128) paged_multiquery_reduce_kernel(const Mult
     const int mid = (lo + hi + 1) / 2;
     if (p.query_start_loc[mid] <= tok) lo = mid; else hi = mid - 1;
   }
+  int q0, q_len;  // a row of no sequence, or of one the partition pass skipped, is not written
+  if (!query_rows_ok(p, lo, q0, q_len) || tok < q0 || tok >= q0 + q_len) return;
   const int BS = p.block_size;
   const int max_ctx = p.max_blocks_per_seq * BS;
   int ctx = p.context_lens[lo];
   ctx = ctx < 0 ? 0 : (ctx > max_ctx ? max_ctx : ctx);
-  const int q_len = p.query_start_loc[lo + 1] - p.query_start_loc[lo];
-  const int pos = ctx - q_len + (tok - p.query_start_loc[lo]);
+  const int pos = ctx - q_len + (tok - q0);
   const int nparts = ((ctx + BS - 1) / BS + p.partition_blocks - 1) / p.partition_blocks;
   if (nparts <= 1) return;  // written directly by the partition pass
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + lane * PVV;

@@ -115,8 +115,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const int Hkv = p.num_kv_heads;
   const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = p.query_start_loc[b];
-  const int q_len = p.query_start_loc[b + 1] - q0;
+  int q0, q_len;
+  if (!query_rows_ok(p, b, q0, q_len)) {  // before any load or store
+    if (threadIdx.x == 0) set_status(p.status, PKV_STATUS_BAD_QUERY_LOC);
+    return;
+  }
   const int rows_total = q_len * G;
   if (q_len <= 0 || qt * T::ROWS >= rows_total) return;
   const int max_ctx = p.max_blocks_per_seq * BS;

@@ -586,3 +586,50 @@ def test_multiquery_one_query_per_sequence_matches_decode():
     dec = pk.paged_attention_decode(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, w.scale)
     torch.cuda.synchronize()
     assert_close(f64(mq), f64(dec), *TOL_BF16, what="multi-query vs decode")
+
+
+@pytest.mark.parametrize("q_lens", [(4, 2, 3), (100, 200, 40)], ids=["verify", "prefill"])
+@pytest.mark.parametrize("case", ["end_past_total", "negative_start", "q_len_above_max"])
+def test_multiquery_guards_bad_query_start_loc(q_lens, case):
+    """query_start_loc entries outside [0, total_q] (or a q_len above max_q_len) reach the kernels only
+    without validate: the sequence is skipped -- no store outside `out`, its rows untouched -- and the
+    status bit is set; the other sequences are computed as usual."""
+    ctxs = (300, 400, 200)
+    spec = W.DecodeSpec("mqqsl", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
+                        ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=24, device=DEV)
+    w = mw.base
+    good = mw.query_start_loc.tolist()
+    T = good[-1]
+    bad, max_q, skipped = list(good), max(q_lens), set()
+    if case == "end_past_total":
+        bad[2] = T + 8            # sequence 1 ends past total_q, sequence 2 then ends before it starts
+        skipped = {1, 2}
+    elif case == "negative_start":
+        bad[0] = -3
+        skipped = {0}
+    else:
+        max_q = min(q_lens)
+        skipped = {b for b in range(3) if q_lens[b] > max_q}
+        assert skipped
+    qsl = torch.tensor(bad, dtype=torch.int32, device=DEV)
+    sentinel = 1000.0
+    ref = oracle.paged_attention_multiquery(to_np(mw.q), to_np(mw.query_start_loc), to_np(w.key_cache),
+                                            to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
+                                            scale=w.scale, q_dtype=oracle.BF16, cache_dtype=oracle.BF16)
+    ref = ref.reshape(T, 8, 128)
+    for pt in (0, 64):
+        buf = torch.full((T + 2, 8, 128), sentinel, dtype=torch.bfloat16, device=DEV)
+        out = buf[1:T + 1]
+        pk.device_status(clear=True)
+        pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qsl,
+                                      w.scale, max_q_len=max_q, out=out, partition_tokens=pt)
+        torch.cuda.synchronize()
+        assert pk.device_status(clear=True) == pk.STATUS_BAD_QUERY_LOC, f"{case} pt={pt}"
+        assert torch.all(buf[0] == sentinel) and torch.all(buf[T + 1] == sentinel), "store outside out"
+        for b in range(3):
+            rows = slice(good[b], good[b + 1])
+            if b in skipped:
+                assert torch.all(out[rows] == sentinel), f"skipped sequence {b} was written ({case} pt={pt})"
+            else:
+                assert_close(f64(out[rows]), ref[rows], *TOL_BF16, what=f"{case} sequence {b} pt={pt}")

@@ -89,3 +89,29 @@ def test_native_cache_matches_reference_on_random_operations(seed, bs, capacity)
             assert native.evict(k) == oracle_cache.evict(k), step
         assert len(native) == len(oracle_cache)
     native.close()
+
+
+
+@pytest.mark.parametrize("impl", ["reference", "native"])
+def test_eviction_follows_last_use_not_release_order(impl):
+    """The reading of "LRU" ("vLLM KV Cache 实现机制", 3.1: a block keeps a last-accessed time for
+    LRU; 3.2: LRU eviction, reference counts protect shared blocks): a block is accessed when a
+    request matches or inserts it; dropping a reference is not an access.  So among the
+    unreferenced entries the one whose last match or insert is oldest goes first, whatever order
+    they were released in."""
+    c = ref.RefPrefixCache(2, 8) if impl == "reference" else pk.PrefixCache(2, 8)
+    A, B, C = [1, 1], [2, 2], [3, 3]
+    assert c.insert(A, [10]) == 1 and c.insert(B, [20]) == 1 and c.insert(C, [30]) == 1  # accessed A, B, C
+    assert c.match(A) == [10]                                                             # accessed B, C, A
+    # released A first (both references), then C; B keeps its reference
+    assert c.release(A, 1) == 1 and c.release(A, 1) == 1 and c.release(C, 1) == 1
+    assert c.evict(3) == [30, 10]     # C was accessed before A; least-recently-released would give [10, 30]
+    assert c.evict(3) == []           # B is referenced
+    assert c.release(B, 1) == 1 and c.evict(3) == [20]
+    # a released entry that is matched again moves behind the others
+    assert c.insert(A, [11]) == 1 and c.insert(B, [21]) == 1
+    assert c.release(A, 1) == 1 and c.release(B, 1) == 1
+    assert c.match(A) == [11] and c.release(A, 1) == 1
+    assert c.evict(1) == [21] and c.evict(1) == [11]
+    if impl == "native":
+        c.close()

@@ -7,7 +7,9 @@ no device allocator -- by keeping the split-context partials in a fixed array
 inside the library.  These tests call it through the C ABI and check it
 against pkv_paged_attention_decode (which takes a caller workspace) on two
 calls in a row with different inputs, so stale partials from the first call
-would show up in the second.  This file is collected last on purpose.
+would show up in the second.  Both entry points run the same kernels with the
+same partition length, so their outputs must be bit-identical; one case is
+also checked against the CPU oracle.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -18,7 +20,7 @@ import torch
 import paged_kv_cache_450_b200 as pk
 from paged_kv_cache_450_b200 import _lib
 from paged_kv_cache_450_b200 import workloads as W
-from step_helpers import TOL, assert_close
+from step_helpers import TOL, assert_close, oracle_step
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -74,10 +76,13 @@ def test_static_scratch_matches_workspace_entry_point_two_calls():
     assert call_static(w1, out_again, 0) == 0
     torch.cuda.synchronize()
     assert torch.cuda.mem_get_info(DEV)[0] == free_mid
-    atol, rtol = TOL["bf16"]
     for (w, pt), out, ref in zip(cases, outs, refs):
-        assert_close(f64(out), f64(ref), atol, rtol, what=f"static scratch, partition_tokens={pt}")
-    assert_close(f64(out_again), f64(refs[0]), atol, rtol, what="static scratch, third call")
+        assert torch.equal(out, ref), f"static scratch differs from the workspace call (partition_tokens={pt})"
+    assert torch.equal(out_again, refs[0]), "static scratch, third call"
+    # the second case against the oracle as well (every row)
+    _, _, oref = oracle_step(w2)
+    atol, rtol = TOL["bf16"]
+    assert_close(f64(outs[1]).reshape(oref.shape), oref, atol, rtol, what="static scratch vs oracle")
     assert pk.device_status(clear=True) == 0
 
 
@@ -95,4 +100,32 @@ def test_static_scratch_rejects_calls_that_need_more_than_the_array():
     n0 = pk.launch_count()
     assert call_static(big, out, 128) == -6        # PKV_ERR_WORKSPACE, nothing launched
     assert pk.launch_count() == n0
+    assert torch.count_nonzero(out) == 0
+
+
+def test_static_scratch_argument_errors_and_empty_batch_match_the_workspace_call():
+    w = W.make_decode_workload(W.LLAMA7B.with_(num_seqs=4, new_tokens=False), seed=24, device=DEV)
+    s = w.spec
+    lib = _lib.load()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    out = torch.zeros_like(w.q)
+    MB = w.block_tables.shape[1]
+
+    def both(num_seqs, head_dim, pt):
+        a = lib.pkv_paged_attention_decode_static(
+            out.data_ptr(), w.q.data_ptr(), w.key_cache.data_ptr(), w.value_cache.data_ptr(),
+            w.block_tables.data_ptr(), w.context_lens.data_ptr(), num_seqs, s.num_q_heads, s.num_kv_heads, head_dim,
+            s.block_size, MB, w.num_blocks, w.scale, 1.0, 1.0, 1, 1, pt, stream)
+        b = lib.pkv_paged_attention_decode(
+            out.data_ptr(), w.q.data_ptr(), w.key_cache.data_ptr(), w.value_cache.data_ptr(),
+            w.block_tables.data_ptr(), w.context_lens.data_ptr(), num_seqs, s.num_q_heads, s.num_kv_heads, head_dim,
+            s.block_size, MB, w.num_blocks, w.scale, 1.0, 1.0, 1, 1, pt, None, 0, 0, stream)
+        return a, b
+
+    n0 = pk.launch_count()
+    assert both(0, 128, 0) == (0, 0)                   # empty batch: nothing to do, nothing launched
+    assert both(s.num_seqs, 96, 0) == (-3, -3)         # PKV_ERR_HEAD_DIM before any workspace question
+    assert both(s.num_seqs, 128, 17) == (-13, -13)     # PKV_ERR_PARTITION
+    assert pk.launch_count() == n0
+    torch.cuda.synchronize()
     assert torch.count_nonzero(out) == 0
