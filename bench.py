@@ -2,15 +2,20 @@
 """Benchmark of the paged decode step on B200: KV-read GB/s and decode tokens/s per layer.
 
 One step = one pass of the whole decode path over one batch: the new-token
-KV write (one token per sequence), then paged decode attention (partition
-pass + split-context reduce), and -- for workloads with shared prefixes --
-the copy-on-write block copies first.  Inputs are synthetic and seeded
-(paged_kv_cache_450_b200.workloads) and already resident in HBM when the
-timed region starts; the KV stream per step (1.14 GB for the default
-workload) is larger than the 126 MB L2, so no flush is needed between steps.
+KV write (one token per sequence, fused into the decode launch), paged decode
+attention (partition pass + split-context reduce) and -- for workloads with
+shared prefixes -- the copy-on-write block copies first.  Inputs are
+synthetic and seeded (paged_kv_cache_450_b200.workloads) and already resident
+in HBM when the timed region starts; every workload's KV stream per step is
+larger than the 126 MB L2, so no flush is needed between steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--configs auto|all|none]
+                  [--impl reference]
 
+The headline line is the LLaMA-13B-shaped batch-256 workload (the largest
+single-GPU configuration).  At N = 1 the same line carries a ``configs``
+object with the same measurements for the other decode configurations and a
+``multiquery`` object for the multi-query workloads, all from this one run.
 N > 1 runs under torchrun, one process per GPU; every rank processes its own
 independent batch (different seed), there is no data-path collective, and the
 time is the max over ranks ("scaling": "weak").  ``--impl reference`` times
@@ -19,13 +24,14 @@ the CPU oracle (fp64 C) on the host cores instead.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
 import re
 import statistics
-import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -37,8 +43,12 @@ sys.path.insert(0, ROOT)
 from paged_kv_cache_450_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s per layer"
-DEFAULT_WORKLOAD = W.LLAMA7B.name
+DEFAULT_WORKLOAD = W.LLAMA13B.name
+# the other decode configurations measured in the same run (N = 1)
+SECONDARY = ["llama13b_decode_b256_bf16_bs32", W.PARALLEL_SAMPLING.name, W.GQA_LONG.name, W.GQA_BATCH.name,
+             W.LLAMA7B.name]
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 SPEC_HBM_GBS = 8000.0
 DTYPE_NAMES = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float8_e4m3fn: "fp8_e4m3"}
 
@@ -89,73 +99,118 @@ def barrier(device=None):
 # peaks, clocks, profiles
 # --------------------------------------------------------------------------- #
 
-def hbm_peak():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _peaks_file():
     try:
-        with open(p) as f:
-            v = float(json.load(f)["hbm_gbs"])
-        return v, "measured"
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def hbm_peak():
+    p = _peaks_file()
+    try:
+        return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def bf16_peak():
+    p = _peaks_file()
+    try:
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# NVML clock-event reason bits and the names the bench line reports
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+REJECT_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and clock-event reasons of this GPU, sampled by a background
+    thread through NVML every ~2 ms for the whole run; ``window(t0, t1)``
+    summarises the samples taken between two host timestamps (a timed region).
+    Reading clocks changes no setting of the GPU."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, device: torch.device):
-        self.proc = None
-        self.path = None
+    def __init__(self, device: torch.device, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []          # (host time, sm MHz, reason bits)
+        self.handle = None
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
         try:
-            uuid = str(torch.cuda.get_device_properties(device).uuid)
-            self.ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
-        except Exception:
-            self.ident = None
+            import pynvml
+            self.nvml = pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            try:
+                uuid = str(props.uuid)
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+            except Exception:  # the same GPU by its PCI address
+                bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # no NVML: the line says so
+            self.error = f"{type(e).__name__}: {e}"
+            self.handle = None
+
+    def _run(self):
+        nv, h = self.nvml, self.handle
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                bits = int(self._reasons(h))
+                self.samples.append((time.perf_counter(), mhz, bits))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
 
     def start(self):
-        if self.ident is None:
-            return
-        self.path = f"/tmp/pkv_clocks_{os.getpid()}.csv"
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.handle is not None and self._thread is None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+            t_end = time.perf_counter() + 1.0
+            while not self.samples and time.perf_counter() < t_end and self._thread.is_alive():
+                time.sleep(0.001)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+
+    def window(self, t0: float, t1: float):
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": f"NVML unavailable ({self.error})"}
+        rows = [s for s in list(self.samples) if t0 <= s[0] <= t1]
+        where = "inside the timed region"
+        if not rows:  # a region shorter than the sampling period: the samples just around it
+            near = sorted(list(self.samples), key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            rows = near
+            where = "the samples nearest the timed region (region shorter than the 2 ms sampling period)"
         if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "NVML, no sample"}
+        reasons = sorted({name for _, _, b in rows for bit, name in _REASONS.items() if b & bit})
+        med = statistics.median(r[1] for r in rows)
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(rows),
+                "source": f"NVML every {self.period * 1e3:.0f} ms, {where}",
+                "rejected": bool(set(reasons) & REJECT_REASONS) or (self.max_mhz is not None and not reasons
+                                                                     and med < 0.8 * self.max_mhz)}
 
 
-def profile_traffic(kernel_file: str, workload: str):
-    """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (sha256 of the files it names); else None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel_file}.md")
+def profile_traffic(profile: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (sha256 recorded in the summary); else None."""
+    path = os.path.join(ROOT, "profiles", f"{profile}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -170,6 +225,7 @@ def profile_traffic(kernel_file: str, workload: str):
 
 
 def kernel_source_hash() -> str:
+    """sha256 of the decode kernel sources (what a recorded DRAM byte count depends on)."""
     d = os.path.join(ROOT, "paged_kv_cache_450_b200", "csrc")
     hsh = hashlib.sha256()
     for name in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_mma_bf16.cuh", "decode_launch.cuh"):
@@ -179,7 +235,7 @@ def kernel_source_hash() -> str:
 
 
 # --------------------------------------------------------------------------- #
-# the GPU arm
+# byte accounting
 # --------------------------------------------------------------------------- #
 
 def kernel_name(spec) -> str:
@@ -193,6 +249,20 @@ def kernel_name(spec) -> str:
     return "paged_decode_partition_kernel"
 
 
+def unique_kv_bytes(w) -> int:
+    """KV bytes of the distinct (physical block, row) pairs one decode pass reads:
+    a block shared by several sequences counts once (prefix sharing)."""
+    s = w.spec
+    bs = s.block_size
+    tables = w.block_tables.cpu().numpy()
+    rows = {}
+    for b, c in enumerate(w.ctx_list):
+        for j in range(-(-c // bs)):
+            pid = int(tables[b, j])
+            rows[pid] = max(rows.get(pid, 0), min(bs, c - j * bs))
+    return int(sum(rows.values())) * s.num_kv_heads * s.head_dim * W.elem_size(s.cache_dtype) * 2
+
+
 def step_inputs_bytes(w) -> tuple[int, int]:
     """Bytes of one step's per-step inputs (host -> device) and result (device -> host)."""
     ts = [w.q, w.new_k, w.new_v, w.slot_mapping, w.block_tables, w.context_lens, w.copy_pairs]
@@ -200,15 +270,22 @@ def step_inputs_bytes(w) -> tuple[int, int]:
     return h2d, w.q.numel() * w.q.element_size()
 
 
-def run_gpu(args, rank, world, local_rank):
+def _events(n=2):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+# --------------------------------------------------------------------------- #
+# the GPU arm: one decode workload
+# --------------------------------------------------------------------------- #
+
+def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
+    """Step, decode-kernel, end-to-end and oracle timings of one decode workload."""
     import paged_kv_cache_450_b200 as pk
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    spec = workload_spec(args)
     w = W.make_decode_workload(spec, seed=rank_seed(args.seed, rank), device=dev)
     s = spec
     kv_bytes = w.kv_bytes()
+    kv_unique = unique_kv_bytes(w) if w.copy_pairs is not None else kv_bytes
     MB = w.block_tables.shape[1]
     pt = pk.decode_partition_tokens(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
                                     s.cache_dtype, args.partition_tokens)
@@ -216,31 +293,26 @@ def run_gpu(args, rank, world, local_rank):
                                          s.cache_dtype, pt)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     out = torch.empty_like(w.q)
-    kc, vc = w.key_cache, w.value_cache
     stream = torch.cuda.current_stream(dev)
-
     fused = w.new_k is not None and not args.unfused
 
-    def step(ev_mid=None, ev_end=None):
-        if w.copy_pairs is not None and len(w.copy_pairs):
-            pk.kv_block_copy(w.copy_pairs, kc, vc, stream=stream)
+    def decode(kc, vc, tables):
         if fused:  # the new token (one per sequence, at ctx - 1) is written inside the decode launch
-            if ev_mid is not None:
-                ev_mid.record(stream)
-            pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, w.block_tables, w.context_lens, w.scale,
+            pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, tables, w.context_lens, w.scale,
                                    k_scale=w.k_scale, v_scale=w.v_scale, out=out, workspace=workspace,
                                    partition_tokens=pt, stream=stream)
         else:
             if w.new_k is not None:
                 pk.paged_kv_write(w.new_k, w.new_v, w.slot_mapping, kc, vc, k_scale=w.k_scale, v_scale=w.v_scale,
                                   stream=stream)
-            if ev_mid is not None:
-                ev_mid.record(stream)
-            pk.paged_attention_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, k_scale=w.k_scale,
+            pk.paged_attention_decode(w.q, kc, vc, tables, w.context_lens, w.scale, k_scale=w.k_scale,
                                       v_scale=w.v_scale, out=out, workspace=workspace, partition_tokens=pt,
                                       stream=stream)
-        if ev_end is not None:
-            ev_end.record(stream)
+
+    def step():
+        if w.copy_pairs is not None and len(w.copy_pairs):
+            pk.kv_block_copy(w.copy_pairs, w.key_cache, w.value_cache, stream=stream)
+        decode(w.key_cache, w.value_cache, w.block_tables)
 
     for _ in range(args.warmup):
         step()
@@ -249,42 +321,47 @@ def run_gpu(args, rank, world, local_rank):
     # ---- timed region: device-resident inputs, K whole steps ------------------
     # No events between the kernels of a step (they would stop the launch of
     # one kernel from overlapping the tail of the previous one).
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev)
+    t0, t1 = _events()
     barrier(dev)
     torch.cuda.synchronize(dev)
-    clocks.start()
     launches0 = pk.launch_count()
+    h0 = time.perf_counter()
     t0.record(stream)
     for _ in range(args.steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
     launches = pk.launch_count() - launches0
     barrier(dev)
-    clk = clocks.stop()
-    elapsed_ms = t0.elapsed_time(t1)
+    clk = clocks.window(h0, h1)
+    step_ms = t0.elapsed_time(t1) / args.steps
 
-    # ---- the decode kernels alone (roofline): events around each decode call --
-    n_inst = max(1, min(args.steps, 1000))
-    mids = [torch.cuda.Event(enable_timing=True) for _ in range(n_inst)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_inst)]
-    for i in range(n_inst):
-        step(mids[i], ends[i])
+    # ---- the decode launches alone (roofline): one event pair around N -------
+    # back-to-back decode calls (partition pass + merge; the fused append
+    # rewrites the same token each time), on the launching stream.
+    n_dec = max(args.steps, 20)
+    d0, d1 = _events()
+    d0.record(stream)
+    for _ in range(n_dec):
+        decode(w.key_cache, w.value_cache, w.block_tables)
+    d1.record(stream)
     torch.cuda.synchronize(dev)
-    decode_ms = sum(m.elapsed_time(e) for m, e in zip(mids, ends)) / n_inst
+    decode_ms = d0.elapsed_time(d1) / n_dec
+
+    ablation = placement_ablation(w, args, dev, stream, decode, pt, n_dec) if headline and world == 1 else None
 
     # ---- end to end through the public API with pinned host buffers ----------
     host = {k: (getattr(w, k).cpu().pin_memory() if getattr(w, k) is not None else None)
             for k in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens", "copy_pairs")}
     # two steps in flight: the copies in of step i+1 overlap the kernels of step i
-    pipe = pk.HostStepPipeline(host["q"], host["new_k"], kc, host["block_tables"], host["copy_pairs"],
+    pipe = pk.HostStepPipeline(host["q"], host["new_k"], w.key_cache, host["block_tables"], host["copy_pairs"],
                                partition_tokens=pt, depth=2, compute_stream=stream)
 
     def e2e_step():
         pipe.step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
-                  host["context_lens"], kc, vc, w.scale, copy_pairs=host["copy_pairs"], k_scale=w.k_scale,
-                  v_scale=w.v_scale)
+                  host["context_lens"], w.key_cache, w.value_cache, w.scale, copy_pairs=host["copy_pairs"],
+                  k_scale=w.k_scale, v_scale=w.v_scale)
 
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(args.warmup, 10)):
@@ -294,7 +371,7 @@ def run_gpu(args, rank, world, local_rank):
     barrier(dev)
     # the timed region opens on the copy-in stream (before the first copy) and closes on the
     # copy-out stream after the last step's output has landed in host memory
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = _events()
     e0.record(pipe.copy_in)
     for _ in range(e2e_steps):
         e2e_step()
@@ -303,52 +380,291 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     barrier(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    del pipe
 
     # ---- cross-rank aggregation ------------------------------------------------
-    step_ms = max_over_ranks(elapsed_ms / args.steps, dev)
+    step_ms = max_over_ranks(step_ms, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
     decode_ms = max_over_ranks(decode_ms, dev)
     total_kv = sum_over_ranks(kv_bytes, dev)
     total_seqs = sum_over_ranks(s.num_seqs, dev)
     h2d, d2h = step_inputs_bytes(w)
-
     peak, peak_kind = hbm_peak()
     value = total_kv / (step_ms * 1e-3) / 1e9
-    achieved = kv_bytes / (decode_ms * 1e-3) / 1e9
-    res = None
-    if rank == 0:
-        cpu = cpu_baseline(w, args) if (world == 1 and not args.no_cpu_baseline) else None
-        res = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": DTYPE_NAMES[s.cache_dtype], "data": "synthetic",
-            "config": {"workload": s.name, "num_seqs_per_gpu": s.num_seqs, "num_q_heads": s.num_q_heads,
-                       "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
-                       "q_dtype": DTYPE_NAMES[s.q_dtype], "kv_dtype": DTYPE_NAMES[s.cache_dtype],
-                       "context_lens": list(s.ctx), "pool": list(s.pool),
-                       "kv_bytes_per_step_per_gpu": kv_bytes, "partition_tokens": pt,
-                       "new_tokens_per_step": 0 if w.new_k is None else int(w.new_k.shape[0]),
-                       "new_token_write": "fused into the decode launch" if fused else "separate launch",
-                       "cow_pairs_per_step": 0 if w.copy_pairs is None else int(len(w.copy_pairs)),
-                       "l2": "inputs larger than L2 (KV stream per step > 126 MB); no flush",
-                       "parallelism": f"dp{world} (independent batch per GPU, no collective)"},
-            "pct_of_hbm_peak": {"measured_copy": round(100 * value / peak, 2) if peak_kind == "measured" else None,
-                                "spec_8tbs": round(100 * value / SPEC_HBM_GBS, 2)},
-            "tokens_per_s_per_layer": round(total_seqs / (step_ms * 1e-3), 1),
-            "roofline": {"kernel": kernel_name(s) + " + paged_decode_reduce_kernel",
-                         "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "peak_kind": f"{peak_kind} (burst copy bandwidth)", "frac": round(achieved / peak, 4),
-                         "algorithmic_bytes_per_launch": kv_bytes, "decode_ms": round(decode_ms, 5),
-                         "timing": f"CUDA events around each decode call on its stream, {n_inst} steps after the timed region",
-                         "traffic": profile_traffic("paged_decode_" + s.name, s.name)},
-            "e2e": {"value": round(total_kv / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": e2e_steps,
-                    "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async (pinned host inputs and output every step; two steps in flight: copies in, kernels, copies out on three streams)"},
-            "gpu_launches": int(launches),
-            "clocks": clk,
-            "cpu_baseline": cpu,
-        }
+    shared = w.copy_pairs is not None
+    # algorithmic bytes of the decode launch: the logical KV stream, or for shared
+    # prefixes the distinct blocks (the rest is served from L2)
+    alg = kv_unique if shared else kv_bytes
+    achieved = alg / (decode_ms * 1e-3) / 1e9
+    traffic = profile_traffic("paged_decode_" + s.name, s.name)
+    res = {
+        "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(step_ms, 5),
+        "tokens_per_s_per_layer": round(total_seqs / (step_ms * 1e-3), 1),
+        "pct_of_hbm_peak": {"measured_copy": round(100 * value / peak, 2) if peak_kind == "measured" else None,
+                            "fallback_copy": round(100 * value / peak, 2) if peak_kind == "fallback" else None,
+                            "spec_8tbs": round(100 * value / SPEC_HBM_GBS, 2)},
+        "config": {"workload": s.name, "num_seqs_per_gpu": s.num_seqs, "num_q_heads": s.num_q_heads,
+                   "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
+                   "q_dtype": DTYPE_NAMES[s.q_dtype], "kv_dtype": DTYPE_NAMES[s.cache_dtype],
+                   "context_lens": list(s.ctx), "pool": list(s.pool),
+                   "kv_bytes_per_step_per_gpu": kv_bytes, "partition_tokens": pt,
+                   "new_tokens_per_step": 0 if w.new_k is None else int(w.new_k.shape[0]),
+                   "new_token_write": "fused into the decode launch" if fused else "separate launch",
+                   "cow_pairs_per_step": 0 if w.copy_pairs is None else int(len(w.copy_pairs)),
+                   "l2": "inputs larger than L2 (KV stream per step > 126 MB); no flush",
+                   "parallelism": f"dp{world} (independent batch per GPU, no collective)"},
+        "roofline": {"kernel": kernel_name(s) + " + paged_decode_reduce_kernel",
+                     "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "peak_kind": f"{peak_kind} (burst copy bandwidth)", "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes_per_launch": alg, "decode_ms": round(decode_ms, 5),
+                     "timing": f"one CUDA event pair around {n_dec} back-to-back decode launches on their stream",
+                     "traffic": traffic},
+        "e2e": {"value": round(total_kv / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": e2e_steps,
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async (pinned host "
+                       "inputs and output every step; two steps in flight: copies in, kernels, copies out on "
+                       "three streams)"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if shared:
+        res["kv_bytes_unique_per_step"] = kv_unique
+        res["value_unique"] = round(kv_unique / (step_ms * 1e-3) / 1e9, 2)
+        res["roofline"]["algorithmic_bytes_note"] = (
+            "distinct (block, row) pairs read: the shared prompt blocks count once; the logical stream "
+            f"({kv_bytes} B) re-reads them from L2")
+        if traffic:
+            res["roofline"]["dram_rate"] = round(traffic / (decode_ms * 1e-3) / 1e9, 2)
+    if ablation is not None:
+        res["placement_ablation"] = ablation
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget if headline else args.cpu_budget / 2)
+    else:
+        res["cpu_baseline"] = None
+    del w, workspace, out, host
+    gc.collect()
+    torch.cuda.empty_cache()
     return res
+
+
+def placement_ablation(w, args, dev, stream, decode, pt, n):
+    """Context for the pages' "the paged kernel is 20-26% slower than a contiguous
+    one" ("vLLM — 把操作系统的分页搬进 GPU KV cache", 踩过的坑): the same decode on
+    the same bytes with every sequence's blocks laid out contiguously (identity
+    order), the block-table reads alone (pkv_decode_table_scan, the decode grid),
+    each timed with one event pair around n back-to-back launches."""
+    import paged_kv_cache_450_b200 as pk
+    s = w.spec
+    tables = w.block_tables.cpu().numpy()
+    order, new_tab = [], np.zeros_like(tables)
+    for b, c in enumerate(w.ctx_list):
+        nb = -(-c // s.block_size)
+        new_tab[b, :nb] = np.arange(len(order), len(order) + nb)
+        order.extend(int(x) for x in tables[b, :nb])
+    idx = torch.tensor(order, dtype=torch.int64, device=dev)
+    kc, vc = w.key_cache.index_select(0, idx), w.value_cache.index_select(0, idx)
+    tab = torch.from_numpy(new_tab).to(dev)
+    res = {}
+    for name, (k_, v_, t_) in (("random_placement", (w.key_cache, w.value_cache, w.block_tables)),
+                               ("contiguous_placement", (kc, vc, tab))):
+        for _ in range(3):
+            decode(k_, v_, t_)
+        a, b = _events()
+        a.record(stream)
+        for _ in range(n):
+            decode(k_, v_, t_)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[f"{name}_decode_ms"] = round(a.elapsed_time(b) / n, 5)
+    sink = pk.decode_table_scan(w.block_tables, w.context_lens, s.num_kv_heads, s.block_size, w.num_blocks, pt,
+                                stream=stream)
+    a, b = _events()
+    a.record(stream)
+    for _ in range(n):
+        pk.decode_table_scan(w.block_tables, w.context_lens, s.num_kv_heads, s.block_size, w.num_blocks, pt,
+                             sink=sink, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    res["table_scan_ms"] = round(a.elapsed_time(b) / n, 5)
+    res["table_scan_share_of_decode"] = round(res["table_scan_ms"] / res["random_placement_decode_ms"], 4)
+    res["random_over_contiguous"] = round(res["random_placement_decode_ms"] / res["contiguous_placement_decode_ms"],
+                                          4)
+    res["note"] = ("same kernel and bytes; contiguous = each sequence's blocks at consecutive physical ids. "
+                   "table_scan = the decode grid reading only its block ids (an upper bound: in the decode "
+                   "those reads overlap the KV stream)")
+    del kc, vc, tab, sink
+    return res
+
+
+# --------------------------------------------------------------------------- #
+# the GPU arm: one multi-query workload
+# --------------------------------------------------------------------------- #
+
+def measure_multiquery(name, args, dev, rank, world, clocks):
+    """Multi-query attention (draft verification / chunked prefill) timed alone."""
+    import paged_kv_cache_450_b200 as pk
+
+    spec, n = W.MQ_SPECS[name]
+    if args.num_seqs:
+        spec = spec.with_(name=f"{spec.name}@b{args.num_seqs}", num_seqs=args.num_seqs)
+    mw = W.make_multiquery_workload(spec, [n] * spec.num_seqs, seed=rank_seed(args.seed, rank), device=dev)
+    w = mw.base
+    s = spec
+    kv_bytes = w.kv_bytes()
+    flops = mw.flops()
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(mw.q)
+    MB = w.block_tables.shape[1]
+    T = int(mw.query_start_loc[-1])
+    need = pk.multiquery_workspace_bytes(s.num_seqs, T, n, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
+                                         MB, s.cache_dtype, args.partition_tokens)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                      mw.query_start_loc, w.scale, k_scale=w.k_scale, v_scale=w.v_scale, max_q_len=n,
+                                      out=out, workspace=ws, partition_tokens=args.partition_tokens, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    steps = max(args.steps, 20)
+    t0, t1 = _events()
+    barrier(dev)
+    launches0 = pk.launch_count()
+    h0 = time.perf_counter()
+    t0.record(stream)
+    for _ in range(steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
+    launches = pk.launch_count() - launches0
+    clk = clocks.window(h0, h1)
+    step_ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    total_kv = sum_over_ranks(kv_bytes, dev)
+    total_flops = sum_over_ranks(flops, dev)
+    peak_gbs, gkind = hbm_peak()
+    peak_tf, tkind = bf16_peak()
+    gbs = kv_bytes / (step_ms * 1e-3) / 1e9
+    tflops = flops / (step_ms * 1e-3) / 1e12
+    tensor_bound = flops / max(kv_bytes, 1) > peak_tf * 1e12 / (peak_gbs * 1e9)
+    tc = n * (s.num_q_heads // s.num_kv_heads) > 16 and s.cache_dtype == torch.bfloat16
+    res = {
+        "value": round(total_kv / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(step_ms, 5),
+        "steps": steps, "dtype": DTYPE_NAMES[s.cache_dtype],
+        "tflops": round(total_flops / (step_ms * 1e-3) / 1e12, 2),
+        "config": {"workload": s.name, "op": "paged_attention_multiquery (causal, queries = last q_len positions)",
+                   "num_seqs_per_gpu": s.num_seqs, "q_len": n, "num_q_heads": s.num_q_heads,
+                   "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
+                   "context_lens": list(s.ctx), "kv_bytes_per_step_per_gpu": kv_bytes, "flops_per_step": flops},
+        "roofline": {"kernel": ("paged_multiquery_tc_kernel" if tc else "paged_multiquery_mma_kernel")
+                               + (" + paged_multiquery_reduce_kernel" if need else ""),
+                     "bound": "tensor" if tensor_bound else "hbm",
+                     "achieved": round(tflops if tensor_bound else gbs, 2),
+                     "peak": peak_tf if tensor_bound else peak_gbs,
+                     "unit": "TFLOP/s" if tensor_bound else "GB/s",
+                     "peak_kind": (f"{tkind} (burst bf16 GEMM)" if tensor_bound else f"{gkind} (burst copy bandwidth)"),
+                     "frac": round((tflops / peak_tf) if tensor_bound else (gbs / peak_gbs), 4),
+                     "timing": f"one CUDA event pair around {steps} back-to-back calls on their stream",
+                     "traffic": None},
+        "gpu_launches": int(launches), "clocks": clk,
+    }
+    del mw, w, out, ws
+    gc.collect()
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------------------- #
+# one companion operation alone (--op), for its own rate and its ncu summary
+# --------------------------------------------------------------------------- #
+
+OPS = ("kv_write", "block_copy", "swap", "amax", "table_scan")
+
+
+def measure_op(op, args, dev):
+    """Times one library call on the workload's tensors, one CUDA event pair
+    around K back-to-back calls.  Bytes are the call's algorithmic bytes: read
+    + written for the copies and the write, read for amax and the table scan."""
+    import paged_kv_cache_450_b200 as pk
+
+    spec = workload_spec(args)
+    w = W.make_decode_workload(spec, seed=rank_seed(args.seed, 0), device=dev)
+    s = spec
+    stream = torch.cuda.current_stream(dev)
+    blk = W.block_bytes(s.block_size, s.num_kv_heads, s.head_dim, s.cache_dtype)
+    extra = {}
+    if op == "kv_write":
+        T = int(w.new_k.shape[0])
+        row = s.num_kv_heads * s.head_dim
+        nbytes = 2 * T * row * (W.elem_size(s.q_dtype) + W.elem_size(s.cache_dtype)) + T * 8
+
+        def call():
+            pk.paged_kv_write(w.new_k, w.new_v, w.slot_mapping, w.key_cache, w.value_cache, k_scale=w.k_scale,
+                              v_scale=w.v_scale, stream=stream)
+        kernel = "paged_kv_write_kernel"
+    elif op == "block_copy":
+        if w.copy_pairs is None:
+            raise SystemExit("--op block_copy needs a workload with copy-on-write pairs")
+        n = int(len(w.copy_pairs))
+        nbytes = 2 * 2 * n * blk  # K and V, read + written
+
+        def call():
+            pk.kv_block_copy(w.copy_pairs, w.key_cache, w.value_cache, stream=stream)
+        kernel = "kv_block_copy_kernel"
+    elif op == "swap":
+        n = min(args.swap_blocks, w.num_blocks)
+        ids = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(args.seed))[:n]
+        pairs_out = torch.stack([ids, torch.arange(n)], 1).to(dev)
+        host_k = torch.empty((n,) + tuple(w.key_cache.shape[1:]), dtype=w.key_cache.dtype, pin_memory=True)
+        host_v = torch.empty_like(host_k, pin_memory=True)
+        nbytes = 2 * n * blk  # K and V over the host link, one direction
+
+        def call():
+            pk.swap_blocks(pairs_out, w.key_cache, w.value_cache, host_k, host_v, stream=stream)
+        kernel = "kv_block_copy_kernel (device -> pinned host)"
+        extra = {"blocks": n, "direction": "device to pinned host (swap out)"}
+    elif op == "amax":
+        if s.cache_dtype not in (torch.bfloat16, torch.float32):
+            raise SystemExit("--op amax reads a bf16 or f32 tensor")
+        x = w.key_cache.view(-1)
+        nbytes = x.numel() * x.element_size()
+        scale = torch.empty((1,), dtype=torch.float32, device=dev)
+
+        def call():
+            pk.fp8_scale_from_amax(x, out=scale, stream=stream)
+        kernel = "amax_kernel + fp8_scale_finish_kernel"
+    elif op == "table_scan":
+        MB = w.block_tables.shape[1]
+        pt = pk.decode_partition_tokens(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
+                                        s.cache_dtype, args.partition_tokens)
+        sink = pk.decode_table_scan(w.block_tables, w.context_lens, s.num_kv_heads, s.block_size, w.num_blocks, pt,
+                                    stream=stream)
+        nbytes = sum(-(-c // s.block_size) for c in w.ctx_list) * 4 * s.num_kv_heads  # id reads, all CTAs
+
+        def call():
+            pk.decode_table_scan(w.block_tables, w.context_lens, s.num_kv_heads, s.block_size, w.num_blocks, pt,
+                                 sink=sink, stream=stream)
+        kernel = "decode_table_scan_kernel"
+        extra = {"partition_tokens": pt, "bytes_note": "block-id reads of every CTA (each KV head's CTAs re-read "
+                                                      "the sequence's ids)"}
+    else:
+        raise SystemExit(f"unknown --op {op}")
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    a, b = _events()
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / args.steps
+    assert pk.device_status(clear=True) == 0
+    return {"metric": f"{op} GB/s", "op": op, "kernel": kernel, "value": round(nbytes / (ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "ms_per_call": round(ms, 5), "bytes_per_call": int(nbytes), "steps": args.steps,
+            "warmup": args.warmup, "config": {"workload": s.name, **extra}}
 
 
 # --------------------------------------------------------------------------- #
@@ -368,7 +684,7 @@ def _host_state(w):
 
     code = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float8_e4m3fn: oracle.E4M3}
     s = w.spec
-    st = {"q": to_np(w.q), "kc": to_np(w.key_cache).copy(), "vc": to_np(w.value_cache).copy(),
+    st = {"q": to_np(w.q), "kc": to_np(w.key_cache), "vc": to_np(w.value_cache),
           "tables": to_np(w.block_tables), "lens": to_np(w.context_lens), "qd": code[s.q_dtype],
           "cd": code[s.cache_dtype]}
     if w.copy_pairs is not None and len(w.copy_pairs):
@@ -394,16 +710,10 @@ def _oracle_rows(w, st, rows, threads):
                                          v_scale=w.v_scale, rows=rows, num_threads=threads)
 
 
-def cpu_baseline(w, args, budget_s: float = 15.0):
-    """The oracle as it stands, on this host's cores, over a bounded sample of
-    the same workload: whole rows (sequence, query head) in a seeded order
-    until about `budget_s` seconds of work or the whole batch."""
-    threads = os.cpu_count() or 1
-    st = _host_state(w)
-    rb = _row_bytes(w)
-    order = np.random.default_rng(0).permutation(len(rb))
+def _oracle_rate(w, st, rb, order, threads, budget_s):
+    """Whole rows in the seeded order until about budget_s seconds of oracle work."""
     done, t_used, nbytes, i = 0, 0.0, 0.0, 0
-    chunk = max(threads, 8)
+    chunk = max(threads, 2)
     while i < len(order) and t_used < budget_s:
         rows = order[i:i + chunk]
         t = time.perf_counter()
@@ -413,9 +723,28 @@ def cpu_baseline(w, args, budget_s: float = 15.0):
         done += len(rows)
         i += len(rows)
         chunk = min(chunk * 2, 4096)
-    return {"value": round(nbytes / t_used / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {len(rb)} (sequence, query head) rows of {w.spec.name} "
-                      f"({nbytes / 1e9:.3f} GB of logical KV) in {t_used:.1f} s, fp64 C oracle, OpenMP"}
+    return nbytes / max(t_used, 1e-9) / 1e9, done, nbytes, t_used
+
+
+def cpu_baseline(w, budget_s: float = 16.0):
+    """The oracle as it stands, on this host's cores, over a bounded sample of
+    the same workload: whole (sequence, query head) rows in a seeded order,
+    with OpenMP over all cores and on one thread (each about budget_s / 2)."""
+    threads = os.cpu_count() or 1
+    st = _host_state(w)
+    rb = _row_bytes(w)
+    order = np.random.default_rng(0).permutation(len(rb))
+    v_all, n_all, b_all, t_all = _oracle_rate(w, st, rb, order, threads, budget_s / 2)
+    v_one, n_one, b_one, t_one = _oracle_rate(w, st, rb, order, 1, budget_s / 2)
+    del st
+    gc.collect()
+    return {"value": round(v_all, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_all} of {len(rb)} (sequence, query head) rows of {w.spec.name} "
+                      f"({b_all / 1e9:.3f} GB of logical KV) in {t_all:.1f} s, fp64 C oracle, OpenMP on "
+                      f"{threads} threads",
+            "single_thread": {"value": round(v_one, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{n_one} rows ({b_one / 1e9:.3f} GB of logical KV) in {t_one:.1f} s, "
+                                        "the same oracle on one thread"}}
 
 
 def run_reference(args, rank, world):
@@ -478,13 +807,21 @@ def workload_spec(args):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.SPECS) + sorted(W.MQ_SPECS))
+    ap.add_argument("--configs", default="auto", choices=["auto", "all", "none"],
+                    help="also measure the other decode and multi-query workloads in this run (N = 1): "
+                         "auto = when the headline is the default workload")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--op", default="step", choices=("step",) + OPS,
+                    help="time one companion operation alone on the workload's tensors instead of the step")
+    ap.add_argument("--swap-blocks", type=int, default=4096, help="blocks moved by --op swap")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=1000)
+    ap.add_argument("--cpu-budget", type=float, default=16.0,
+                    help="seconds of oracle work for the headline's cpu_baseline (half for the other configs)")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
@@ -494,83 +831,36 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def run_multiquery(args, rank, world, local_rank):
-    """Multi-query attention (draft verification / chunked prefill) timed alone."""
-    import paged_kv_cache_450_b200 as pk
-
+def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    spec, n = W.MQ_SPECS[args.workload]
-    if args.num_seqs:
-        spec = spec.with_(name=f"{spec.name}@b{args.num_seqs}", num_seqs=args.num_seqs)
-    mw = W.make_multiquery_workload(spec, [n] * spec.num_seqs, seed=rank_seed(args.seed, rank), device=dev)
-    w = mw.base
-    s = spec
-    kv_bytes = w.kv_bytes()
-    flops = mw.flops()
-    stream = torch.cuda.current_stream(dev)
-    out = torch.empty_like(mw.q)
-    MB = w.block_tables.shape[1]
-    lib = pk._lib.load()
-    T = int(mw.query_start_loc[-1])
-    need = int(lib.pkv_multiquery_workspace_bytes(s.num_seqs, T, n, s.num_q_heads, s.num_kv_heads, s.head_dim,
-                                                  s.block_size, MB, args.partition_tokens))
-    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-
-    def call():
-        pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
-                                      mw.query_start_loc, w.scale, max_q_len=n, out=out, workspace=ws,
-                                      partition_tokens=args.partition_tokens, stream=stream)
-
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
     clocks = ClockSampler(dev)
     clocks.start()
-    launches0 = pk.launch_count()
-    t0.record(stream)
-    for _ in range(args.steps):
-        call()
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    launches = pk.launch_count() - launches0
-    clk = clocks.stop()
-    step_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
-    total_kv = sum_over_ranks(kv_bytes, dev)
-    total_flops = sum_over_ranks(flops, dev)
-    if rank != 0:
-        return None
-    peak_gbs, peak_kind = hbm_peak()
-    gbs = kv_bytes / (step_ms * 1e-3) / 1e9
-    tflops = flops / (step_ms * 1e-3) / 1e12
     try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak_tf = float(json.load(f)["bf16_tflops"])
-    except Exception:
-        peak_tf = 1590.0
-    tensor_bound = flops / max(kv_bytes, 1) > peak_tf * 1e12 / (peak_gbs * 1e9)
-    return {
-        "metric": METRIC, "value": round(total_kv / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": s.name, "op": "paged_attention_multiquery (causal, queries = last q_len positions)",
-                   "num_seqs_per_gpu": s.num_seqs, "q_len": n, "num_q_heads": s.num_q_heads,
-                   "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
-                   "context_lens": list(s.ctx), "kv_bytes_per_step_per_gpu": kv_bytes, "flops_per_step": flops},
-        "tflops": round(total_flops / (step_ms * 1e-3) / 1e12, 2),
-        "roofline": {"kernel": ("paged_multiquery_tc_kernel" if n * (s.num_q_heads // s.num_kv_heads) > 16
-                                else "paged_multiquery_bf16_kernel")
-                               + (" + paged_multiquery_reduce_kernel" if need else ""),
-                     "bound": "tensor" if tensor_bound else "hbm",
-                     "achieved": round(tflops if tensor_bound else gbs, 2),
-                     "peak": peak_tf if tensor_bound else peak_gbs,
-                     "unit": "TFLOP/s" if tensor_bound else "GB/s",
-                     "frac": round((tflops / peak_tf) if tensor_bound else (gbs / peak_gbs), 4),
-                     "traffic": None},
-        "gpu_launches": int(launches), "clocks": clk, "cpu_baseline": None,
-    }
+        common = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic"}
+        if args.workload in W.MQ_SPECS:
+            r = measure_multiquery(args.workload, args, dev, rank, world, clocks)
+            return {**common, "dtype": "bf16", **r, "cpu_baseline": None}
+        spec = workload_spec(args)
+        head = measure_decode(spec, args, dev, rank, world, clocks, headline=True)
+        res = {**common, "dtype": DTYPE_NAMES[spec.cache_dtype], **head}
+        run_configs = world == 1 and (args.configs == "all" or (args.configs == "auto" and
+                                                                 args.workload == DEFAULT_WORKLOAD
+                                                                 and not args.num_seqs))
+        if run_configs:
+            res["configs"] = {}
+            for name in SECONDARY + ([DEFAULT_WORKLOAD] if args.workload != DEFAULT_WORKLOAD else []):
+                if name == args.workload:
+                    continue
+                r = measure_decode(W.SPECS[name], args, dev, rank, world, clocks, headline=False)
+                r["dtype"] = DTYPE_NAMES[W.SPECS[name].cache_dtype]
+                res["configs"][name] = r
+            res["multiquery"] = {name: measure_multiquery(name, args, dev, rank, world, clocks)
+                                 for name in sorted(W.MQ_SPECS)}
+        return res
+    finally:
+        clocks.stop()
 
 
 def main(argv=None):
@@ -592,11 +882,14 @@ def main(argv=None):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.op != "step":
+        if world != 1:
+            raise SystemExit("--op runs on one GPU")
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_op(args.op, args, torch.device("cuda", 0))), flush=True)
+        return
     try:
-        if args.workload in W.MQ_SPECS:
-            res = run_multiquery(args, rank, world, local_rank)
-        else:
-            res = run_gpu(args, rank, world, local_rank)
+        res = run_gpu(args, rank, world, local_rank)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

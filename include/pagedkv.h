@@ -291,6 +291,9 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
  *
  * out, q            device [total_q][num_q_heads][head_dim] bf16; rows of
  *                   sequence b are query_start_loc[b] .. query_start_loc[b+1]-1.
+ * key_cache,        device, cache layout above: BF16, or FP8_E4M3 with the
+ * value_cache       dequantisation scales k_scale, v_scale (both > 0; ignored
+ *                   for BF16).
  * query_start_loc   device int32 [num_seqs + 1], non-decreasing, starting at 0,
  *                   ending at total_q; every q_len_b <= max_q_len and
  *                   <= context_lens[b] (validate checks all of this; without
@@ -303,36 +306,42 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
  *                   previous bytes) and PKV_STATUS_BAD_QUERY_LOC is set.
  * workspace         device scratch of pkv_multiquery_workspace_bytes(...) bytes
  *                   (same arguments; 0 when no split is needed), 256-byte aligned.
- * Supported: bf16 q and caches, head_dim 128, block_size 16 or 32, 1/2/4/8
- * query heads per KV head.  Runs on the tensor cores: up to 64 rows per
- * (sequence, KV head) -- rows = max_q_len x query heads per KV head -- on
- * mma.sync m16n8k16; more rows (prefill) on tcgen05 with 128-row tiles and
- * 128-token KV tiles.  Other arguments and errors: as
+ * Supported: bf16 q, bf16 or fp8 E4M3 caches, head_dim 128, block_size 16 or
+ * 32, 1/2/4/8 query heads per KV head.  Runs on the tensor cores.  bf16
+ * caches: up to 16 rows per (sequence, KV head) -- rows = max_q_len x query
+ * heads per KV head -- on mma.sync m16n8k16 (bf16 operands, P as a bf16 high
+ * part and residual); more rows (prefill) on tcgen05 with 128-row tiles and
+ * 128-token KV tiles (bf16 Q.K^T; P.V on fp16 operands, V converted from bf16
+ * in shared memory, exact for |v| in [2^-14, 65504] -- V beyond the fp16
+ * range is not supported).  fp8 caches: mma.sync for every row count, the
+ * codes widened exactly to fp16 in shared memory, q rounded once to fp16
+ * (exact for |q| in [2^-14, 65504]), fp16 P.  Other arguments and errors: as
  * pkv_paged_attention_decode.
  */
 int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cache, const void* value_cache,
                                    const int32_t* block_tables, const int32_t* context_lens,
                                    const int32_t* query_start_loc, int num_seqs, int total_q, int max_q_len,
                                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                                   int max_blocks_per_seq, int64_t num_blocks, float scale, int q_dtype,
-                                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
-                                   int validate, void* stream);
+                                   int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                                   float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                                   void* workspace, size_t workspace_bytes, int validate, void* stream);
 
 /* Split-context partition length pkv_paged_attention_multiquery uses:
  * partition_tokens if non-zero (a multiple of block_size, at most 16384), else
  * automatic -- one partition when (sequences x KV heads x query-row tiles of
- * the kernel that serves these rows) already gives two waves of its resident
- * CTAs, else the longest context split so that it does, in multiples of 256
- * tokens.  Negative PKV_ERR_* for unsupported arguments.  A sizing helper of
- * this library (no counterpart on the pages). */
+ * the kernel that serves these rows and cache_dtype) already gives two waves
+ * of its resident CTAs, else the longest context split so that it does, in
+ * multiples of 256 tokens.  Negative PKV_ERR_* for unsupported arguments.  A
+ * sizing helper of this library (no counterpart on the pages). */
 int pkv_multiquery_partition_tokens(int num_seqs, int max_q_len, int num_q_heads, int num_kv_heads, int block_size,
-                                    int max_blocks_per_seq, int partition_tokens);
+                                    int max_blocks_per_seq, int cache_dtype, int partition_tokens);
 
 /* Workspace bytes pkv_paged_attention_multiquery needs (0 when no context is
  * split): float (m, l) then, at a 256-byte boundary, float o[d] per (query
  * token, query head, partition).  A sizing helper of this library. */
 size_t pkv_multiquery_workspace_bytes(int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
-                                      int head_dim, int block_size, int max_blocks_per_seq, int partition_tokens);
+                                      int head_dim, int block_size, int max_blocks_per_seq, int cache_dtype,
+                                      int partition_tokens);
 
 /*
  * Per-tensor fp8 scale on the device: *scale = amax(|x|) / 448 (one fp32
@@ -494,6 +503,29 @@ int64_t pkv_prefix_cache_insert(void* cache, const int32_t* tokens, int64_t num_
 int64_t pkv_prefix_cache_release(void* cache, const int32_t* tokens, int64_t num_tokens, uint64_t extra_hash,
                                  int64_t num_blocks);
 int64_t pkv_prefix_cache_evict(void* cache, int64_t max_evict, int32_t* evicted_ids_out);
+
+/*
+ * The block-table reads of a decode launch, alone (a measurement aid; the
+ * pages have no counterpart).  Runs the decode grid -- one CTA per (kv head,
+ * partition of partition_tokens tokens, sequence) -- and in each CTA only the
+ * coalesced, range-checked reads of that partition's physical block ids from
+ * block_tables, the "one more int load" of "vLLM — 把操作系统的分页搬进 GPU KV
+ * cache", 核心要点.  No KV byte is read.  Its time and L2 hit rate, next to the
+ * decode's, show what the indirection costs.
+ *
+ * block_tables,   device, as pkv_paged_attention_decode.
+ * context_lens
+ * partition_tokens  the decode's partition length (pkv_decode_partition_tokens),
+ *                 a positive multiple of block_size; there is no automatic choice.
+ * sink            device unsigned [num_seqs][P][num_kv_heads], P = ceil(max_blocks_per_seq
+ *                 * block_size / partition_tokens): one word per CTA (a hash of its ids).
+ * Out-of-pool ids and context lengths set the status bits the decode sets.
+ * Errors: PKV_ERR_BAD_SHAPE, _BLOCK_SIZE, _PARTITION, _NULL_POINTER,
+ * _WORKSPACE (sink_words too small), _CUDA.  num_seqs == 0 launches nothing.
+ */
+int pkv_decode_table_scan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_kv_heads,
+                          int block_size, int max_blocks_per_seq, int64_t num_blocks, int partition_tokens,
+                          unsigned* sink, size_t sink_words, void* stream);
 
 /*
  * Reads the current device's status word (PKV_STATUS_* bits) into *status,

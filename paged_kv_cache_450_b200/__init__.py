@@ -31,10 +31,10 @@ STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 STATUS_BAD_QUERY_LOC = 0x20
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_multiquery", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
-           "decode_partition_tokens", "decode_max_partitions", "device_status", "launch_count", "PagedKVError",
+           "decode_partition_tokens", "decode_max_partitions", "decode_table_scan", "device_status", "launch_count", "PagedKVError",
            "library_path"]
 
 
@@ -203,13 +203,23 @@ def paged_decode_append(q, k_new, v_new, key_cache, value_cache, block_tables, c
     return out
 
 
+def multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                               max_blocks_per_seq, cache_dtype, partition_tokens=0) -> int:
+    """Workspace bytes paged_attention_multiquery needs (0 when no context is split)."""
+    return int(_lib.load().pkv_multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads,
+                                                          head_dim, block_size, max_blocks_per_seq,
+                                                          _cache_code(cache_dtype), partition_tokens))
+
+
 def paged_attention_multiquery(q, key_cache, value_cache, block_tables, context_lens, query_start_loc,
-                                scale: float, *, max_q_len: int | None = None, out=None, workspace=None,
+                                scale: float, *, k_scale: float = 1.0, v_scale: float = 1.0,
+                                max_q_len: int | None = None, out=None, workspace=None,
                                 partition_tokens: int = 0, validate: bool = False, stream=None):
     """Causal attention of several new query tokens per sequence over the paged
     cache (chunked prefill, speculative verification).  q: [total_q, Hq, d]
-    bf16; query_start_loc int32 [B + 1]; the queries of sequence b are its
-    last q_len_b positions (their K/V already written).  Returns [total_q, Hq, d]."""
+    bf16; caches bf16 or float8_e4m3fn (then k_scale / v_scale dequantise);
+    query_start_loc int32 [B + 1]; the queries of sequence b are its last
+    q_len_b positions (their K/V already written).  Returns [total_q, Hq, d]."""
     dev = _cuda(q, key_cache, value_cache, block_tables, context_lens, query_start_loc)
     for t in (block_tables, context_lens, query_start_loc):
         if t.dtype != torch.int32:
@@ -225,7 +235,7 @@ def paged_attention_multiquery(q, key_cache, value_cache, block_tables, context_
     if out is None:
         out = torch.empty_like(q)
     lib = _lib.load()
-    need = int(lib.pkv_multiquery_workspace_bytes(B, T, max_q_len, Hq, Hkv, d, bs, MB, partition_tokens)) if B else 0
+    need = multiquery_workspace_bytes(B, T, max_q_len, Hq, Hkv, d, bs, MB, key_cache.dtype, partition_tokens) if B else 0
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
@@ -234,8 +244,8 @@ def paged_attention_multiquery(q, key_cache, value_cache, block_tables, context_
         _check(lib.pkv_paged_attention_multiquery(
             out.data_ptr(), q.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(), block_tables.data_ptr(),
             context_lens.data_ptr(), query_start_loc.data_ptr(), B, T, max_q_len, Hq, Hkv, d, bs, MB, NB,
-            float(scale), _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr, ws_bytes, int(validate),
-            _stream(dev, stream)), "paged_attention_multiquery")
+            float(scale), float(k_scale), float(v_scale), _dtype(q), _dtype(key_cache), int(partition_tokens), ws_ptr,
+            ws_bytes, int(validate), _stream(dev, stream)), "paged_attention_multiquery")
     return out
 
 
@@ -294,6 +304,25 @@ def swap_blocks(src_dst_pairs, src_key, src_value, dst_key, dst_value, *, valida
                                            src_value.data_ptr(), src_key.shape[0], dst_key.data_ptr(),
                                            dst_value.data_ptr(), dst_key.shape[0], block_bytes, int(validate),
                                            _stream(dev, stream)), "swap_blocks")
+
+
+def decode_table_scan(block_tables, context_lens, num_kv_heads: int, block_size: int, num_blocks: int,
+                      partition_tokens: int, *, sink=None, stream=None):
+    """The decode grid's block-table reads alone (a measurement aid): one CTA per
+    (kv head, partition, sequence) reads its partition's block ids and writes one
+    word to ``sink`` (uint32-sized int32 [B * P * Hkv], allocated when not given)."""
+    dev = _cuda(block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, MB = block_tables.shape
+    P = -(-MB * block_size // partition_tokens)
+    if sink is None:
+        sink = torch.empty(max(1, B * P * num_kv_heads), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_decode_table_scan(block_tables.data_ptr(), context_lens.data_ptr(), B, num_kv_heads,
+                                                 block_size, MB, num_blocks, partition_tokens, sink.data_ptr(),
+                                                 sink.numel(), _stream(dev, stream)), "decode_table_scan")
+    return sink
 
 
 def device_status(clear: bool = True, device=None, stream=None) -> int:

@@ -33,10 +33,10 @@ SIGNATURES = {
     "pkv_decode_max_partitions": (I, [I, I, I, I, I, I, I, I]),
     "pkv_decode_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),
     "pkv_kv_block_copy": (I, [P, I64, P, P, I64, I64, I, P]),
-    "pkv_paged_attention_multiquery": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F, I, I, I, P, SZ, I,
-                                           P]),
-    "pkv_multiquery_partition_tokens": (I, [I, I, I, I, I, I, I]),
-    "pkv_multiquery_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I, I]),
+    "pkv_paged_attention_multiquery": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F, F, F, I, I, I, P, SZ,
+                                           I, P]),
+    "pkv_multiquery_partition_tokens": (I, [I, I, I, I, I, I, I, I]),
+    "pkv_multiquery_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I, I, I]),
     "pkv_fp8_scale_from_amax": (I, [P, I64, I, P, P]),
     "pkv_swap_blocks": (I, [P, I64, P, P, I64, P, P, I64, I64, I, P]),
     "pkv_prefix_block_hashes": (I64, [P, I64, I, U64, U64, P]),
@@ -47,6 +47,7 @@ SIGNATURES = {
     "pkv_prefix_cache_insert": (I64, [P, P, I64, U64, P, I64]),
     "pkv_prefix_cache_release": (I64, [P, P, I64, U64, I64]),
     "pkv_prefix_cache_evict": (I64, [P, I64, P]),
+    "pkv_decode_table_scan": (I, [P, P, I, I, I, I, I64, I, P, SZ, P]),
     "pkv_device_status": (I, [ctypes.POINTER(ctypes.c_uint), I, P]),
     "pkv_launch_count": (U64, []),
 }

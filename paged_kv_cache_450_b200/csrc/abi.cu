@@ -443,7 +443,7 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
 // of the kernel's resident CTAs, else the context split so that it does
 // (multiples of 256 tokens).
 static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int max_q_len, int block_size,
-                               int max_blocks_per_seq, int partition_tokens) {
+                               int max_blocks_per_seq, bool fp8, int partition_tokens) {
   if (partition_tokens != 0) {
     if (partition_tokens < 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
       return PKV_ERR_PARTITION;
@@ -453,8 +453,8 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
   const int64_t rows = static_cast<int64_t>(max_q_len) * group;
   // CTAs per (sequence, KV head) and resident CTAs per SM of the kernel that
   // serves these rows: 16- to 64-row mma.sync CTAs (6 to 2 per SM), or 128-row
-  // tcgen05 CTAs (1 per SM)
-  const bool tc = multiquery_uses_tc(static_cast<int>(rows > 0x7fffffff ? 0x7fffffff : rows));
+  // tcgen05 CTAs (1 per SM; bf16 caches only)
+  const bool tc = !fp8 && multiquery_uses_tc(static_cast<int>(rows > 0x7fffffff ? 0x7fffffff : rows));
   const int nwc = multiquery_compute_warps(static_cast<int>(rows > 64 ? 64 : rows));
   const int tile = tc ? 128 : 16 * nwc;
   const int per_sm = tc ? 1 : multiquery_ctas_per_sm(nwc);
@@ -470,19 +470,21 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
 }
 
 int pkv_multiquery_partition_tokens(int num_seqs, int max_q_len, int num_q_heads, int num_kv_heads, int block_size,
-                                    int max_blocks_per_seq, int partition_tokens) {
+                                    int max_blocks_per_seq, int cache_dtype, int partition_tokens) {
   if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
   if (num_seqs < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0)
     return PKV_ERR_BAD_SHAPE;
+  if (cache_dtype != PKV_DTYPE_BF16 && cache_dtype != PKV_DTYPE_FP8_E4M3) return PKV_ERR_BAD_DTYPE;
   if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
   return mq_partition_tokens(num_seqs, num_kv_heads, num_q_heads / num_kv_heads, max_q_len, block_size,
-                             max_blocks_per_seq, partition_tokens);
+                             max_blocks_per_seq, cache_dtype == PKV_DTYPE_FP8_E4M3, partition_tokens);
 }
 
 size_t pkv_multiquery_workspace_bytes(int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
-                                      int head_dim, int block_size, int max_blocks_per_seq, int partition_tokens) {
+                                      int head_dim, int block_size, int max_blocks_per_seq, int cache_dtype,
+                                      int partition_tokens) {
   const int pt = pkv_multiquery_partition_tokens(num_seqs, max_q_len, num_q_heads, num_kv_heads, block_size,
-                                                 max_blocks_per_seq, partition_tokens);
+                                                 max_blocks_per_seq, cache_dtype, partition_tokens);
   if (pt < 0 || total_q <= 0 || head_dim <= 0) return 0;
   const int64_t P = cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt);
   if (P <= 1) return 0;
@@ -494,16 +496,19 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
                                    const int32_t* block_tables, const int32_t* context_lens,
                                    const int32_t* query_start_loc, int num_seqs, int total_q, int max_q_len,
                                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                                   int max_blocks_per_seq, int64_t num_blocks, float scale, int q_dtype,
-                                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
-                                   int validate, void* stream) {
+                                   int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale,
+                                   float v_scale, int q_dtype, int cache_dtype, int partition_tokens,
+                                   void* workspace, size_t workspace_bytes, int validate, void* stream) {
   if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0)
     return PKV_ERR_BAD_SHAPE;
   if (num_seqs == 0 || total_q == 0) return PKV_OK;
   if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens || !query_start_loc)
     return PKV_ERR_NULL_POINTER;
-  if (q_dtype != PKV_DTYPE_BF16 || cache_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (q_dtype != PKV_DTYPE_BF16 || (cache_dtype != PKV_DTYPE_BF16 && cache_dtype != PKV_DTYPE_FP8_E4M3))
+    return PKV_ERR_BAD_DTYPE;
+  const bool fp8 = cache_dtype == PKV_DTYPE_FP8_E4M3;
+  if (fp8 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_BAD_SHAPE;
   if (head_dim != 128) return PKV_ERR_HEAD_DIM;
   if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
   if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
@@ -511,13 +516,14 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_HEAD_GROUPING;
   if (num_blocks > 0x7fffffffLL || num_seqs > 65535) return PKV_ERR_BAD_SHAPE;
   if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
-  const int pt = mq_partition_tokens(num_seqs, num_kv_heads, group, max_q_len, block_size, max_blocks_per_seq,
+  const int pt = mq_partition_tokens(num_seqs, num_kv_heads, group, max_q_len, block_size, max_blocks_per_seq, fp8,
                                      partition_tokens);
   if (pt < 0) return pt;
   const int P = static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
   if (P > 65535) return PKV_ERR_PARTITION;
   const size_t need = pkv_multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads,
-                                                     head_dim, block_size, max_blocks_per_seq, partition_tokens);
+                                                     head_dim, block_size, max_blocks_per_seq, cache_dtype,
+                                                     partition_tokens);
   if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -568,16 +574,44 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   p.max_partitions = P;
   p.total_q = total_q;
   p.max_q_len = max_q_len;
-  p.q_scale = scale * kLog2e;
+  p.q_scale = scale * kLog2e * (fp8 ? k_scale : 1.f);
+  p.out_scale = fp8 ? v_scale : 1.f;
   const int rows_per_seq = max_q_len * group;
   if (rows_per_seq <= 0) return PKV_OK;
+  if (fp8)
+    return launch_multiquery_mma_fp8(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
+                                                                                                    : PKV_ERR_CUDA;
   if (multiquery_uses_tc(rows_per_seq)) {
     CUtensorMap qmap;
     if (!encode_query_map(&qmap, q, total_q, num_q_heads, group)) return PKV_ERR_TENSOR_MAP;
     return launch_multiquery_tc(qmap, kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
                                                                                                      : PKV_ERR_CUDA;
   }
-  return launch_multiquery_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  return launch_multiquery_mma_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
+                                                                                                  : PKV_ERR_CUDA;
+}
+
+int pkv_decode_table_scan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_kv_heads,
+                          int block_size, int max_blocks_per_seq, int64_t num_blocks, int partition_tokens,
+                          unsigned* sink, size_t sink_words, void* stream) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return PKV_ERR_BAD_SHAPE;
+  if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (partition_tokens <= 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
+    return PKV_ERR_PARTITION;
+  if (num_seqs == 0) return PKV_OK;
+  if (!block_tables || !context_lens || !sink) return PKV_ERR_NULL_POINTER;
+  if (num_blocks > 0x7fffffffLL || num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_BAD_SHAPE;
+  if (static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffffLL) return PKV_ERR_BAD_SHAPE;
+  const int64_t P = cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, partition_tokens);
+  if (P > 65535) return PKV_ERR_PARTITION;
+  if (sink_words < static_cast<size_t>(num_seqs) * num_kv_heads * P) return PKV_ERR_WORKSPACE;
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  return launch_table_scan(block_tables, context_lens, num_seqs, num_kv_heads, max_blocks_per_seq,
+                           static_cast<int>(num_blocks), block_size, partition_tokens / block_size,
+                           static_cast<int>(P), sink, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PKV_OK
+             : PKV_ERR_CUDA;
 }
 
 int pkv_fp8_scale_from_amax(const void* x, int64_t n, int dtype, float* scale, void* stream) {

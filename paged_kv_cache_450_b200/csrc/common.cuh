@@ -134,6 +134,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Two bf16 values (one 32-bit word, first value in the low half) -> two fp16
+// values in the same order: the widening to fp32 is exact, then one
+// round-to-nearest pack (exact for magnitudes in [2^-14, 65504]).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -60,6 +60,11 @@ cudaError_t launch_block_copy(const int64_t* pairs, int64_t num_pairs, const voi
                               int64_t src_blocks, void* dst_k, void* dst_v, int64_t dst_blocks, int64_t block_bytes,
                               unsigned* status, cudaStream_t st);
 
+// The decode grid's block-table reads alone (a measurement aid, table_scan.cu).
+cudaError_t launch_table_scan(const int32_t* tables, const int32_t* lens, int num_seqs, int num_kv_heads,
+                              int max_blocks_per_seq, int num_blocks, int block_size, int partition_blocks,
+                              int num_partitions, unsigned* sink, unsigned* status, cudaStream_t st);
+
 // The tensor-core decode kernels serve head_dim 128 with 16- or 32-token
 // blocks: fp8 caches with 8 query heads per KV head, and bf16 caches with 2,
 // 4 or 8 (grouped-query attention, where CUDA-core work grows with the
@@ -74,13 +79,14 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
   return false;
 }
 
-// Multi-query (prefill / verification) attention: bf16, head_dim 128, bs 16/32.
-// Up to 16 rows per (sequence, KV head) -- rows = queries x query heads of the
-// group -- run on the mma.sync kernel (one 16-row warp per CTA); more rows on
-// the tcgen05 kernel with 128-row tiles, whose time per KV tile does not
-// depend on how many of the rows are used (measured: 40 rows, 70B-GQA
-// verification, 2.70 TB/s on mma.sync with three 16-row warps, 3.56 TB/s on
-// tcgen05).
+// Multi-query (prefill / verification) attention: bf16 q, bf16 or fp8 caches,
+// head_dim 128, bs 16/32.  bf16 caches: up to 16 rows per (sequence, KV head)
+// -- rows = queries x query heads of the group -- run on the mma.sync kernel
+// (one 16-row warp per CTA); more rows on the tcgen05 kernel with 128-row
+// tiles, whose time per KV tile does not depend on how many of the rows are
+// used (measured: 40 rows, 70B-GQA verification, 2.70 TB/s on mma.sync with
+// three 16-row warps, 3.56 TB/s on tcgen05).  fp8 caches: the mma.sync kernel
+// for every row count.
 #ifndef PKV_MQ_TC_MIN_ROWS
 #define PKV_MQ_TC_MIN_ROWS 16
 #endif
@@ -94,8 +100,11 @@ inline int multiquery_compute_warps(int rows_per_seq) {
 inline int multiquery_ctas_per_sm(int compute_warps) {
   return compute_warps == 1 ? 6 : (compute_warps == 2 ? 4 : (compute_warps == 3 ? 3 : 2));
 }
-cudaError_t launch_multiquery_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
-                                   int group, int rows_per_seq, bool reduce, cudaStream_t st);
+// The mma.sync kernel over bf16 caches and over fp8 (E4M3) caches.
+cudaError_t launch_multiquery_mma_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                                       int group, int rows_per_seq, bool reduce, cudaStream_t st);
+cudaError_t launch_multiquery_mma_fp8(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
+                                      int group, int rows_per_seq, bool reduce, cudaStream_t st);
 cudaError_t launch_multiquery_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                                  const MultiQueryParams& p, int group, int rows_per_seq, bool reduce,
                                  cudaStream_t st);

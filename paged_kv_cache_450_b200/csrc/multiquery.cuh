@@ -3,8 +3,8 @@
 // paged cache: the q_len queries of a sequence are its last q_len positions
 // and query i (position p = ctx - q_len + i) attends the logical tokens 0..p.
 //
-// FlashAttention-2 style on the tensor cores (mma.sync m16n8k16, bf16
-// operands, fp32 accumulation).  One CTA = 16, 32, 48 or 64 query rows (the
+// FlashAttention-2 style on the tensor cores (mma.sync m16n8k16, fp32
+// accumulation).  One CTA = 16, 32, 48 or 64 query rows (the
 // rows of a (sequence, KV head), rounded up to 16, at most 64) x one KV head x one
 // split-context partition of one sequence; rows are (query i, query head g)
 // with g fastest, so grouped-query heads share every K/V tile.  A producer
@@ -17,8 +17,18 @@
 //                 ldmatrix.trans; P as bf16 hi + lo, ~16 bits per weight)
 // The online softmax per row keeps a reference max as in the decode kernels.
 // Partitions write (m, l, o) partials merged by paged_multiquery_reduce_kernel.
-// The dispatch (launch.h) sends it up to 16 rows per (sequence, KV head); more
-// rows go to the tcgen05 kernel (multiquery_tc.cuh).
+//
+// Caches of fp8 (E4M3, per-tensor scales; F8 = true): the producer warp
+// TMA-loads each block's raw codes (128 bytes per token row) into a ring of
+// its own and widens them to fp16 -- exactly: every E4M3 value is an fp16
+// value -- into the stage, in the same swizzled layout a bf16 tile has, so
+// the compute warps read it with the same ldmatrix offsets.  Q is rounded
+// once to fp16, and both contractions run on fp16 operands with one fp16 P
+// (11 significant bits).  The K scale is folded into the logit scale and the
+// V scale into the output.
+// The dispatch (launch.h) sends bf16 caches here up to 16 rows per (sequence,
+// KV head) -- more rows go to the tcgen05 kernel (multiquery_tc.cuh) -- and
+// fp8 caches for every row count.
 #pragma once
 
 #include "decode.cuh"
@@ -31,7 +41,7 @@ namespace pkv {
 // NWC_ compute warps of 16 rows each: as many as the rows of a (sequence, KV
 // head) need, up to 4, so that CTAs are no larger than the work and more of
 // them fit on an SM.
-template <int BS, int NWC_ = 4, int NS_ = 0>
+template <int BS, int NWC_ = 4, int NS_ = 0, bool F8 = false>
 struct MqTraits {
   static constexpr int D = 128;
   static constexpr int NWC = NWC_;                   // compute warps (16 rows each)
@@ -45,21 +55,66 @@ struct MqTraits {
   static constexpr int MIN_BLOCKS = NWC_ == 1 ? 6 : (NWC_ == 2 ? 4 : (NWC_ == 3 ? 3 : 2));
   static constexpr int NT = BS / 16;
   static constexpr int STAGE_AREA = NS * STAGE_BYTES;
-  static constexpr int BAR_BYTES = 2 * NS * 8;
-  static constexpr size_t smem_bytes(int pb) { return 1024 + STAGE_AREA + BAR_BYTES + static_cast<size_t>(pb) * 4; }
+  // fp8 caches: a ring of raw blocks (K then V codes, 128 bytes per token row)
+  static constexpr int RAW_HALF = BS * 128;
+  static constexpr int RAW_BYTES = 2 * RAW_HALF;
+  static constexpr int NR = F8 ? 3 : 0;
+  static constexpr int RAW_AREA = NR * RAW_BYTES;
+  static constexpr int BAR_BYTES = (2 * NS + NR) * 8;  // full[NS], empty[NS], raw_full[NR]
+  static constexpr size_t smem_bytes(int pb) {
+    return 1024 + STAGE_AREA + RAW_AREA + BAR_BYTES + static_cast<size_t>(pb) * 4;
+  }
 };
 
-template <int BS, int G, int NWC>
-__global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>::MIN_BLOCKS)
-    paged_multiquery_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                                 const MultiQueryParams p) {
-  using T = MqTraits<BS, NWC>;
+// Widens one block of raw E4M3 codes (K and V: BS rows x 128 codes, 128-byte
+// swizzle) into fp16 in the bf16 stage layout (two 64-dim halves of BS rows x
+// 128 bytes, 128-byte swizzle).  Raw chunk q of row t (dims 16q .. 16q+15)
+// becomes stage chunks 2(q % 4) and 2(q % 4) + 1 of half q / 4.  One warp.
+template <int BS>
+__device__ __forceinline__ void widen_e4m3_block(const uint8_t* raw, uint8_t* stage, int lane) {
+  constexpr int RAW_HALF = BS * 128, TILE = BS * 256, HALF = BS * 128;
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+#pragma unroll
+    for (int i = lane; i < BS * 8; i += 32) {
+      const int t = i >> 3, q = i & 7;
+      const uint4 w = *reinterpret_cast<const uint4*>(raw + kv * RAW_HALF + t * 128 + ((q ^ (t & 7)) << 4));
+      uint32_t f[8];
+      e4m3x4_to_f16x2x2(w.x, f[0], f[1]);
+      e4m3x4_to_f16x2x2(w.y, f[2], f[3]);
+      e4m3x4_to_f16x2x2(w.z, f[4], f[5]);
+      e4m3x4_to_f16x2x2(w.w, f[6], f[7]);
+      uint8_t* dst = stage + kv * TILE + (q >> 2) * HALF + t * 128;
+      const int c0 = 2 * (q & 3);
+      *reinterpret_cast<uint4*>(dst + ((c0 ^ (t & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ (t & 7)) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
+    }
+  }
+}
+
+// D(16x8, f32) += A(16x16) . B(16x8): bf16 operands, or fp16 (F16 = true).
+template <bool F16>
+__device__ __forceinline__ void mma_16816_t(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    mma_16816(d, a0, a1, a2, a3, b0, b1);
+  } else {
+    mma_16816_bf16(d, a0, a1, a2, a3, b0, b1);
+  }
+}
+
+template <int BS, int G, int NWC, bool F8>
+__global__ void __launch_bounds__(MqTraits<BS, NWC, 0, F8>::THREADS, MqTraits<BS, NWC, 0, F8>::MIN_BLOCKS)
+    paged_multiquery_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                                const MultiQueryParams p) {
+  using T = MqTraits<BS, NWC, 0, F8>;
   constexpr int D = T::D;
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::STAGE_AREA);  // full[NS], empty[NS]
-  int* ids = reinterpret_cast<int*>(data + T::STAGE_AREA + T::BAR_BYTES);
+  uint8_t* raw = data + T::STAGE_AREA;  // fp8 caches: the raw ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::STAGE_AREA + T::RAW_AREA);  // full, empty, raw_full
+  int* ids = reinterpret_cast<int*>(data + T::STAGE_AREA + T::RAW_AREA + T::BAR_BYTES);
 
   const int Hkv = p.num_kv_heads;
   const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y, b = blockIdx.z;
@@ -111,18 +166,60 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
   }
   // compute warps holding at least one row of this CTA (the others leave now)
   const int n_active = min(T::NWC, (min(rows_total - qt * T::ROWS, T::ROWS) + 15) / 16);
-  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * T::NS;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * T::NS, rfull0 = empty0 + 8 * T::NS;
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, n_active);
     }
+    for (int s = 0; s < T::NR; ++s) mbar_init(rfull0 + 8 * s, 1);
     fence_barrier_init();
   }
   __syncthreads();
   if (warp < T::NWC && warp >= n_active) return;
   const uint32_t stage0 = smem_u32(data);
 
+  if (warp == T::NWC && F8) {  // ---------------- producer warp (fp8: loads and widens) ----------
+    const uint64_t policy = l2_policy_evict_first();
+    const uint32_t raw0 = smem_u32(raw);
+    int issued = 0, landed = 0;
+    auto issue_raw = [&](int j) {  // lane 0: block j's raw K and V codes into ring slot j % NR
+      const int r = j % T::NR;
+      const uint32_t bar = rfull0 + 8 * r;
+      const int id = ids[j];
+      if (id >= 0) {
+        mbar_arrive_expect_tx(bar, T::RAW_BYTES);
+        tma_load_4d(raw0 + r * T::RAW_BYTES, &kmap, bar, 0, hk, 0, id, policy);
+        tma_load_4d(raw0 + r * T::RAW_BYTES + T::RAW_HALF, &vmap, bar, 0, hk, 0, id, policy);
+      } else {
+        mbar_arrive(bar);
+      }
+    };
+    if (lane == 0)
+      for (int j = 0; j < min(nb, T::NR); ++j) issue_raw(j);
+    issued = min(nb, T::NR);
+    for (int j = 0; j < nb; ++j) {
+      const int r = j % T::NR, s = j % T::NS;
+      if (!__all_sync(kFullMask, mbar_wait_bounded(rfull0 + 8 * r, (j / T::NR) & 1, p.status))) break;
+      landed = j + 1;
+      if (j >= T::NS && !__all_sync(kFullMask, mbar_wait_bounded(empty0 + 8 * s, ((j / T::NS) - 1) & 1, p.status)))
+        break;
+      if (ids[j] >= 0) widen_e4m3_block<BS>(raw + r * T::RAW_BYTES, data + s * T::STAGE_BYTES, lane);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(full0 + 8 * s);  // (arrive releases the widened stage to the compute warps)
+        if (j + T::NR < nb) {
+          fence_proxy_async_smem();  // the raw slot's reads before the next TMA write into it
+          issue_raw(j + T::NR);
+        }
+      }
+      if (j + T::NR < nb) issued = j + T::NR + 1;
+    }
+    // Drain (bounded): every raw load started has landed before the CTA exits.
+    if (lane == 0)
+      for (int j = landed; j < issued; ++j) mbar_wait_bounded(rfull0 + 8 * (j % T::NR), (j / T::NR) & 1, p.status);
+    return;
+  }
   if (warp == T::NWC) {  // ---------------- producer warp ----------------------
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
@@ -170,6 +267,10 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
       qf[j][1] = vb_row ? qb[8 * j + c] : 0u;
       qf[j][2] = va_row ? qa[8 * j + c + 4] : 0u;
       qf[j][3] = vb_row ? qb[8 * j + c + 4] : 0u;
+      if constexpr (F8) {  // fp16 operands (exact for |q| in [2^-14, 65504])
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qf[j][e] = bf16x2_to_f16x2(qf[j][e]);
+      }
     }
   }
   const float qk = p.q_scale;
@@ -215,8 +316,8 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
         for (int jj = 0; jj < 8; ++jj) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4(kt + (jj >> 2) * T::HALF_BYTES + koff[jj & 3], b0, b1, b2, b3);
-          mma_16816_bf16(s0, qf[jj][0], qf[jj][1], qf[jj][2], qf[jj][3], b0, b1);
-          mma_16816_bf16(s1, qf[jj][0], qf[jj][1], qf[jj][2], qf[jj][3], b2, b3);
+          mma_16816_t<F8>(s0, qf[jj][0], qf[jj][1], qf[jj][2], qf[jj][3], b0, b1);
+          mma_16816_t<F8>(s1, qf[jj][0], qf[jj][1], qf[jj][2], qf[jj][3], b2, b3);
         }
         // values: row ra: s0[0..1] (tokens 2c, 2c+1), s1[0..1] (8+2c, 8+2c+1); row rb: s0[2..3], s1[2..3]
         float sa[4] = {s0[0] * qk, s0[1] * qk, s1[0] * qk, s1[1] * qk};
@@ -263,12 +364,20 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
         }
         la += (pa[0] + pa[1]) + (pa[2] + pa[3]);
         lb += (pbv[0] + pbv[1]) + (pbv[2] + pbv[3]);
-        // P (A operand of P.V): {row ra tok 2c.., row rb tok 2c.., row ra tok 8+2c.., row rb tok 8+2c..}
+        // P (A operand of P.V): {row ra tok 2c.., row rb tok 2c.., row ra tok 8+2c.., row rb tok 8+2c..};
+        // bf16: a high part and a residual (~16 bits); fp16 (fp8 caches): one fp16 value (11 bits)
         uint32_t ah[4], al[4];
-        bf16x2_split(pa[0], pa[1], ah[0], al[0]);
-        bf16x2_split(pbv[0], pbv[1], ah[1], al[1]);
-        bf16x2_split(pa[2], pa[3], ah[2], al[2]);
-        bf16x2_split(pbv[2], pbv[3], ah[3], al[3]);
+        if constexpr (F8) {
+          ah[0] = f16x2_pack(pa[0], pa[1]);
+          ah[1] = f16x2_pack(pbv[0], pbv[1]);
+          ah[2] = f16x2_pack(pa[2], pa[3]);
+          ah[3] = f16x2_pack(pbv[2], pbv[3]);
+        } else {
+          bf16x2_split(pa[0], pa[1], ah[0], al[0]);
+          bf16x2_split(pbv[0], pbv[1], ah[1], al[1]);
+          bf16x2_split(pa[2], pa[3], ah[2], al[2]);
+          bf16x2_split(pbv[2], pbv[3], ah[3], al[3]);
+        }
         // V rows past the context must not feed NaN bits into the products
         uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
         if (tok0 + 16 > ctx) {
@@ -284,10 +393,12 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
           b1 &= mhi;
           b2 &= mlo;
           b3 &= mhi;
-          mma_16816_bf16(o[2 * m], ah[0], ah[1], ah[2], ah[3], b0, b1);
-          mma_16816_bf16(o[2 * m], al[0], al[1], al[2], al[3], b0, b1);
-          mma_16816_bf16(o[2 * m + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
-          mma_16816_bf16(o[2 * m + 1], al[0], al[1], al[2], al[3], b2, b3);
+          mma_16816_t<F8>(o[2 * m], ah[0], ah[1], ah[2], ah[3], b0, b1);
+          mma_16816_t<F8>(o[2 * m + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+          if constexpr (!F8) {
+            mma_16816_bf16(o[2 * m], al[0], al[1], al[2], al[3], b0, b1);
+            mma_16816_bf16(o[2 * m + 1], al[0], al[1], al[2], al[3], b2, b3);
+          }
         }
       }
     }
@@ -302,7 +413,7 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
     la += __shfl_xor_sync(kFullMask, la, off);
     lb += __shfl_xor_sync(kFullMask, lb, off);
   }
-  const float fa = la > 0.f ? 1.f / la : 0.f, fb = lb > 0.f ? 1.f / lb : 0.f;
+  const float fa = la > 0.f ? p.out_scale / la : 0.f, fb = lb > 0.f ? p.out_scale / lb : 0.f;
   if (nparts == 1) {
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
@@ -331,58 +442,6 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC>::THREADS, MqTraits<BS, NWC>:
       }
     }
   }
-}
-
-// Merge of split-context partials, one warp per (query token, query head).
-__global__ void __launch_bounds__(128) paged_multiquery_reduce_kernel(const MultiQueryParams p) {
-  constexpr int D = 128, PVV = D / 32;
-  pdl_wait_and_release();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
-  if (row >= static_cast<int64_t>(p.total_q) * p.num_q_heads) return;
-  const int tok = static_cast<int>(row / p.num_q_heads);
-  int lo = 0, hi = p.num_seqs - 1;  // the sequence owning query token tok
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) / 2;
-    if (p.query_start_loc[mid] <= tok) lo = mid; else hi = mid - 1;
-  }
-  int q0, q_len;  // a row of no sequence, or of one the partition pass skipped, is not written
-  if (!query_rows_ok(p, lo, q0, q_len) || tok < q0 || tok >= q0 + q_len) return;
-  const int BS = p.block_size;
-  const int max_ctx = p.max_blocks_per_seq * BS;
-  int ctx = p.context_lens[lo];
-  ctx = ctx < 0 ? 0 : (ctx > max_ctx ? max_ctx : ctx);
-  const int pos = ctx - q_len + (tok - q0);
-  const int nparts = ((ctx + BS - 1) / BS + p.partition_blocks - 1) / p.partition_blocks;
-  if (nparts <= 1) return;  // written directly by the partition pass
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + lane * PVV;
-  if (pos < 0) {  // a query before the context: attends nothing
-#pragma unroll
-    for (int e = 0; e < PVV; ++e) out[e] = __float2bfloat16_rn(0.f);
-    return;
-  }
-  const int nvis = min(nparts, pos / (p.partition_blocks * BS) + 1);  // partitions the query can see
-  const float* ml = p.ws_ml + row * p.max_partitions * 2;
-  const float* o = p.ws_o + row * p.max_partitions * D;
-  float M = -INFINITY;
-  for (int i = lane; i < nvis; i += 32)
-    if (ml[2 * i + 1] > 0.f) M = fmaxf(M, ml[2 * i]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
-  float acc[PVV];
-#pragma unroll
-  for (int e = 0; e < PVV; ++e) acc[e] = 0.f;
-  float W = 0.f;
-  for (int i = 0; i < nvis; ++i) {
-    const float li = ml[2 * i + 1];
-    const float w = li > 0.f ? li * fast_exp2((ml[2 * i] - M) * kLog2e) : 0.f;
-    W += w;
-    const float* oi = o + static_cast<int64_t>(i) * D + lane * PVV;
-#pragma unroll
-    for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w, oi[e], acc[e]);
-  }
-#pragma unroll
-  for (int e = 0; e < PVV; ++e) out[e] = __float2bfloat16_rn(W > 0.f ? acc[e] / W : 0.f);
 }
 
 }  // namespace pkv

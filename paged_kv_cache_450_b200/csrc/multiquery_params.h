@@ -25,7 +25,8 @@ struct MultiQueryParams {
   int max_partitions;
   int total_q;
   int max_q_len;  // q_len of any sequence must not exceed it (the grid covers that many rows)
-  float q_scale;  // scale * log2(e)
+  float q_scale;    // scale * log2(e) (* k_scale for fp8 caches)
+  float out_scale;  // v_scale for fp8 caches, else 1
 };
 
 #ifdef __CUDACC__

@@ -18,11 +18,15 @@
 // Q, K and V sit in shared memory in the 128-byte-swizzled layout (two
 // 64-element halves of every 256-byte row) as TMA delivers them; Q and K are
 // K-major operands, V (stored token-major, dims contiguous) is the N-major B
-// operand of P . V, so no transpose is ever made.  P never touches shared
-// memory: it is the TMEM A operand of P . V (columns [384, 512)), split into
-// a bf16 high part and a bf16 residual -- two MMAs per k-step -- so each
-// probability keeps ~16 significant bits (a bf16 P alone costs up to ~3e-3
-// absolute on short contexts).  Eleven warps:
+// operand of P . V, so no transpose is ever made.  S = Q . K^T runs on bf16
+// operands.  P . V runs on fp16 operands: P never touches shared memory -- it
+// is the TMEM A operand (fp16, columns [384, 448)) -- and each V tile is
+// converted from bf16 to fp16 in place in shared memory by the softmax warps
+// before its P . V.  fp16 keeps 11 significant bits of each probability (a
+// bf16 P, 8 bits, costs up to ~3e-3 absolute on short contexts); the
+// conversion of V is exact for |v| in [2^-14, 65504] (smaller magnitudes
+// lose at most 2^-25 absolute; V beyond the fp16 range is not supported).
+// Eleven warps:
 //   warps 0-7  softmax: warp w serves rows 32 (w & 3) .. +31 (the TMEM lanes
 //              its sub-partition may touch) and half h = w >> 2 of every KV
 //              tile's tokens.  The two halves are independent online
@@ -33,11 +37,14 @@
 //              once, in the epilogue.  Per tile a thread reads its 64 scores
 //              from TMEM, applies the causal / context mask, keeps a
 //              reference max (O_h is rescaled only when a score passes it by
-//              more than 2^8), and writes its 64 probabilities into P_h.
-//   warp 8     TMA producer of Q (once) and the K tiles (three-stage ring; one
+//              more than 2^8), writes its 64 probabilities into P_h, and
+//              converts one 128-byte V row segment of its half to fp16 (rows
+//              past the loaded tokens or of a bad block are zeroed instead).
+//   warp 8     TMA producer of Q (once) and the K tiles (two-stage ring; one
 //              4-D box per block and 64-dim half); owns the TMEM allocation.
-//   warp 10    TMA producer of the V tiles (two-stage ring), so that a K load
-//              never waits behind a V stage that P . V still holds.
+//   warp 10    TMA producer of the V tiles (three-stage ring: a V tile is
+//              used one tile period after its K tile, after its conversion),
+//              so that a K load never waits behind a V stage P . V still holds.
 //   warp 9     MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
@@ -60,20 +67,20 @@ struct MqTcTraits {
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16)
   static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 bf16
-  static constexpr int NSK = 3, NSV = 2;  // K ring and V ring depth (K2 / V3 measured slower)
+  static constexpr int NSK = 2, NSV = 3;  // K ring and V ring depth
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
   static constexpr int BAR_OFF = V_OFF + NSV * TILE;
-  // mbarriers: q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_free, p_full[2], pv_done[2],
-  // mma_done (the pairs: one per token half)
+  // mbarriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free, p_full[2],
+  // pv_done[2], mma_done (the pairs: one per token half)
   static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [4][128 rows]: m_0, m_1, l_0, l_1
   static constexpr int IDS_OFF = XCH_OFF + 4 * 128 * 4;
   static constexpr int THREADS = 352;
   static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
-  static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O_0 128 | O_1 128 | P hi 0,1 (32 + 32), lo 0,1 (32 + 32)
+  static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O_0 128 | O_1 128 | P_0, P_1 (32 + 32 packed fp16 pairs)
   static constexpr size_t smem_bytes(int pb) { return 1024 + IDS_OFF + static_cast<size_t>(pb) * 4; }
 };
 
@@ -236,8 +243,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(data + T::SLOT_OFF);
   const uint32_t tmem_s = tmem;
   auto tmem_o = [&](int h) { return tmem + 128 + 128 * h; };
-  auto tmem_phi = [&](int h) { return tmem + 384 + 32 * h; };  // tokens 64h .. 64h+63, packed in pairs
-  auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };
+  auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };  // tokens 64h .. 64h+63, fp16 packed in pairs
 
   if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
     if (lane == 0) {
@@ -272,7 +278,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
       bool ok = mbar_wait_bounded(q_full, 0, p.status);
@@ -296,16 +302,15 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         }
         if (j > 0) {
           const int jj = j - 1, sv = jj % T::NSV;
-          if (!(ok = mbar_wait_bounded(v_full(sv), (jj / T::NSV) & 1, p.status))) break;
           const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
           for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
+            // P_h is in TMEM and the half's V rows are fp16 (the softmax warps waited for the tile)
             if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
               const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
-              tc_mma_bf16_tmem_a(tmem_o(h), tmem_phi(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-              tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+              tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(pv_done(h));
           }
@@ -395,29 +400,47 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
       }
       const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
       // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add, and at once the
-      // row's half of P as packed pairs (tokens 2k, 2k+1 in word k): a high part (the top 16 bits of
-      // the fp32 value: truncation) and the residual (exact in fp32, then truncated to its top 16
-      // bits), ~16 significant bits per probability.  One loop, so the special-function unit (ex2)
-      // and the integer / FMA pipes (packing) work side by side; the stores to TMEM wait below.
+      // row's half of P as fp16 pairs (tokens 2k, 2k+1 in word k, round to nearest; p <= 2^8).  One
+      // loop, so the special-function unit (ex2) and the conversion pipe work side by side; the
+      // stores to TMEM wait below.
       const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
       float2 sum4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
-      uint32_t phi[32], plo[32];
+      uint32_t ph[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
         const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
         sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
-        const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
-        // residual = value - its truncation (the negated truncation is one logic op)
-        const float2 rr = __fadd2_rn(make_float2(a, bb), make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
-                                                                      __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
-        phi[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
-        plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+        const __half2 hp = __floats2half2_rn(a, bb);  // token 2k in the low half
+        ph[k] = *reinterpret_cast<const uint32_t*>(&hp);
       }
       const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
       l += s2.x + s2.y;
+      // This thread's 128-byte V row segment of the half tile to fp16, in place: row 64h + 16 quarter +
+      // lane / 2, dims half lane & 1.  Rows that must not contribute (past tok_end: never loaded; bad
+      // blocks: stale) are zeroed instead, since 0 * NaN would poison O.
+      {
+        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
+        const int vr = 64 * h + 16 * quarter + (lane >> 1);
+        const int t = tok_begin + j * T::TOK + vr;
+        uint4* vrow = reinterpret_cast<uint4*>(data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF +
+                                               vr * 128);
+        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          uint4 w[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) w[c] = vrow[c];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            vrow[c] = make_uint4(bf16x2_to_f16x2(w[c].x), bf16x2_to_f16x2(w[c].y), bf16x2_to_f16x2(w[c].z),
+                                 bf16x2_to_f16x2(w[c].w));
+        }
+        fence_proxy_async_smem();  // the generic-proxy writes before the MMA (async proxy) reads them
+      }
       // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
       if (j > 0) {
         wait(pv_done(h), (j - 1) & 1);
@@ -435,31 +458,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
           }
         }
       }
-      // V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed: 0 * NaN would
-      // poison O.  The 64 rows of this half: thread (quarter, lane) takes row 16 quarter + lane / 2,
-      // dims half lane & 1.
-      if (ragged || bad) {
-        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
-        const int vr = 64 * h + 16 * quarter + (lane >> 1);
-        const int t = tok_begin + j * T::TOK + vr;
-        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
-          uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
-      }
       // this half of row r of P into TMEM lane r
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t hi[16], lo[16];
+        uint32_t pw[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          hi[k] = phi[16 * c + k];
-          lo[k] = plo[16 * c + k];
-        }
-        tmem_st16(tmem_phi(h) + lane_off + 16 * c, hi);
-        tmem_st16(tmem_plo(h) + lane_off + 16 * c, lo);
+        for (int k = 0; k < 16; ++k) pw[k] = ph[16 * c + k];
+        tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
       }
       tmem_st_wait();
       tc_fence_before();

@@ -335,11 +335,13 @@ def make_multiquery_workload(spec: DecodeSpec, q_lens, seed: int = 0,
 
 # Multi-query workload families: draft verification (4 draft tokens + the
 # accepted one per sequence) and chunked prefill (512-token chunks after a
-# prefix), on the LLaMA-7B and 70B-GQA (bf16) shapes.
+# prefix), on the LLaMA-7B and 70B-GQA (bf16 and fp8 cache) shapes.
 MQ_SPECS = {
     "llama7b_verify_b64_q5": (LLAMA7B.with_(name="llama7b_verify_b64_q5"), 5),
     "llama7b_prefill_b8_chunk512": (LLAMA7B.with_(name="llama7b_prefill_b8_chunk512", num_seqs=8,
                                                   ctx=("uniform", 512, 2048)), 512),
     "gqa70b_bf16_verify_b64_q5": (GQA_BATCH_BF16.with_(name="gqa70b_bf16_verify_b64_q5", num_seqs=64,
                                                         ctx=("uniform", 1024, 8192)), 5),
+    "gqa70b_fp8_verify_b64_q5": (GQA_BATCH.with_(name="gqa70b_fp8_verify_b64_q5", num_seqs=64,
+                                                 ctx=("uniform", 1024, 8192)), 5),
 }

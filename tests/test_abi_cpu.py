@@ -107,8 +107,15 @@ def test_partition_choice_and_workspace_size():
 
 def test_multiquery_partition_and_workspace():
     lib = _lib.load()
-    PT, WS = lib.pkv_multiquery_partition_tokens, lib.pkv_multiquery_workspace_bytes
-    # (num_seqs, max_q_len, Hq, Hkv, bs, max_blocks, partition_tokens)
+    BF, F8 = pk.DTYPE_BF16, pk.DTYPE_FP8_E4M3
+    PT0, WS0 = lib.pkv_multiquery_partition_tokens, lib.pkv_multiquery_workspace_bytes
+
+    def PT(B, ql, hq, hkv, bs, mb, pt, cd=BF):  # (num_seqs, max_q_len, Hq, Hkv, bs, max_blocks, cache dtype, pt)
+        return PT0(B, ql, hq, hkv, bs, mb, cd, pt)
+
+    def WS(B, T, ql, hq, hkv, d, bs, mb, pt, cd=BF):
+        return WS0(B, T, ql, hq, hkv, d, bs, mb, cd, pt)
+
     # prefill-sized rows, 1024 tcgen05 CTAs >= two waves: one partition over the longest context
     assert PT(8, 512, 32, 32, 16, 128, 0) == 2048
     assert WS(8, 8 * 512, 512, 32, 32, 128, 16, 128, 0) == 0
@@ -121,6 +128,10 @@ def test_multiquery_partition_and_workspace():
     P = -(-512 * 16 // pt)
     rows = 8 * 5 * 64 * P
     assert WS(8, 8 * 5, 5, 64, 8, 128, 16, 512, 0) == ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
+    # fp8 caches run on the mma.sync kernel (48-row CTAs, 3 per SM): 512 CTAs are not two waves there
+    pt8 = PT(64, 5, 64, 8, 16, 512, 0, F8)
+    assert pt8 % 256 == 0 and 256 <= pt8 < 8192
+    assert WS(64, 64 * 5, 5, 64, 8, 128, 16, 512, 0, F8) > 0
     # MHA verification (5 rows): 16-row CTAs, 6 per SM
     assert PT(64, 5, 32, 32, 16, 128, 0) > 0
     # explicit partition lengths: a multiple of the block size up to 16384 tokens
@@ -132,15 +143,21 @@ def test_multiquery_partition_and_workspace():
     assert PT(1, 4, 8, 8, 8, 100, 0) == ERR_BLOCK_SIZE
     assert PT(1, 4, 8, 3, 16, 100, 0) == ERR_HEAD_GROUPING
     assert PT(-1, 4, 8, 8, 16, 100, 0) == ERR_BAD_SHAPE
+    assert PT(1, 4, 8, 8, 16, 100, 0, pk.DTYPE_F32) == ERR_BAD_DTYPE
     # a call with no work launches nothing and needs nothing
     assert lib.pkv_paged_attention_multiquery(None, None, None, None, None, None, None, 0, 0, 0, 8, 8, 128, 16, 10,
-                                              100, 0.1, pk.DTYPE_BF16, pk.DTYPE_BF16, 0, None, 0, 0, None) == 0
+                                              100, 0.1, 1.0, 1.0, BF, BF, 0, None, 0, 0, None) == 0
     # unsupported shapes are refused before anything else happens
     args = [ctypes.c_void_p(16)] * 7 + [1, 4, 4, 8, 8]
-    assert lib.pkv_paged_attention_multiquery(*args, 64, 16, 10, 100, 0.1, pk.DTYPE_BF16, pk.DTYPE_BF16, 0, None, 0,
+    assert lib.pkv_paged_attention_multiquery(*args, 64, 16, 10, 100, 0.1, 1.0, 1.0, BF, BF, 0, None, 0,
                                               0, None) == ERR_HEAD_DIM
-    assert lib.pkv_paged_attention_multiquery(*args, 128, 16, 10, 100, 0.1, pk.DTYPE_F32, pk.DTYPE_BF16, 0, None,
+    assert lib.pkv_paged_attention_multiquery(*args, 128, 16, 10, 100, 0.1, 1.0, 1.0, pk.DTYPE_F32, BF, 0, None,
                                               0, 0, None) == ERR_BAD_DTYPE
+    assert lib.pkv_paged_attention_multiquery(*args, 128, 16, 10, 100, 0.1, 1.0, 1.0, BF, pk.DTYPE_F32, 0, None,
+                                              0, 0, None) == ERR_BAD_DTYPE
+    # fp8 caches need positive dequantisation scales
+    assert lib.pkv_paged_attention_multiquery(*args, 128, 16, 10, 100, 0.1, 0.0, 1.0, BF, F8, 0, None,
+                                              0, 0, None) == ERR_BAD_SHAPE
 
 
 def test_ops_refuse_cpu_tensors():

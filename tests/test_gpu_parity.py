@@ -387,24 +387,28 @@ def test_fp8_scale_on_device_matches_oracle(dtype, n):
 
 
 def _mq_check(mw, partition_tokens=0, rows=None, what="", validate=True):
+    """Multi-query attention through the C ABI against the oracle on the same stored bytes
+    (bf16 caches: 2e-3 + 1e-2 |ref|; fp8 caches: 2e-3 + 3e-2 |ref|)."""
     w = mw.base
     s = w.spec
     out = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
-                                        mw.query_start_loc, w.scale, partition_tokens=partition_tokens,
-                                        validate=validate)
+                                        mw.query_start_loc, w.scale, k_scale=w.k_scale, v_scale=w.v_scale,
+                                        partition_tokens=partition_tokens, validate=validate)
     torch.cuda.synchronize()
     ref = oracle.paged_attention_multiquery(to_np(mw.q), to_np(mw.query_start_loc), to_np(w.key_cache),
                                             to_np(w.value_cache), to_np(w.block_tables), to_np(w.context_lens),
-                                            scale=w.scale, q_dtype=oracle.BF16, cache_dtype=oracle.BF16, rows=rows)
+                                            scale=w.scale, q_dtype=oracle.BF16, cache_dtype=ocode(s.cache_dtype),
+                                            k_scale=w.k_scale, v_scale=w.v_scale, rows=rows)
     got = f64(out)
     if rows is not None:
         got = got.reshape(-1, s.head_dim)[rows]
-    assert_close(got, ref, *TOL_BF16, what=what)
+    assert_close(got, ref, *(TOL_FP8 if s.cache_dtype == FP8 else TOL_BF16), what=what)
     assert pk.device_status(clear=True) == 0
     return out
 
 
 TOL_BF16 = (2e-3, 1e-2)
+TOL_FP8 = (2e-3, 3e-2)
 
 
 @pytest.mark.parametrize("bs", [16, 32])
@@ -633,3 +637,80 @@ def test_multiquery_guards_bad_query_start_loc(q_lens, case):
                 assert torch.all(out[rows] == sentinel), f"skipped sequence {b} was written ({case} pt={pt})"
             else:
                 assert_close(f64(out[rows]), ref[rows], *TOL_BF16, what=f"{case} sequence {b} pt={pt}")
+
+
+
+# ---- multi-query attention over fp8 (E4M3) caches: the mma.sync kernel, codes widened to fp16 ----
+
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 4), (16, 2)])
+def test_multiquery_fp8_small(bs, hq, hkv):
+    # ragged query counts: one, verification-sized, a full prefill from scratch (129 of 129), none
+    ctxs = (1, 20, 700, 129, 33, 64)
+    q_lens = (1, 5, 8, 129, 0, 17)
+    spec = W.DecodeSpec("mqf8", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, FP8, ("list", ctxs), ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs + hq + hkv, device=DEV)
+    for pt in (0, 2 * bs, 256):
+        _mq_check(mw, partition_tokens=pt, what=f"fp8 bs={bs} hq={hq} hkv={hkv} pt={pt}")
+
+
+def test_multiquery_fp8_queries_before_the_context_get_zero_rows():
+    ctxs = (40, 300, 20, 900)
+    spec = W.DecodeSpec("mqf8neg", len(ctxs), 16, 2, 128, 16, torch.bfloat16, FP8, ("list", ctxs), ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, (20, 5, 20, 100), seed=31, device=DEV)
+    w = mw.base
+    w.context_lens.copy_(torch.tensor([7, 300, 0, 60], dtype=torch.int32, device=DEV))
+    for pt in (0, 16, 128):
+        out = _mq_check(mw, partition_tokens=pt, what=f"fp8 negative positions pt={pt}", validate=False)
+        qsl = mw.query_start_loc.tolist()
+        assert torch.all(out[qsl[0]:qsl[0] + 13] == 0) and torch.all(out[qsl[2]:qsl[3]] == 0)
+        assert torch.all(out[qsl[3]:qsl[3] + 40] == 0)
+
+
+@pytest.mark.parametrize("q_lens", [(5, 5, 5, 5), (200, 129, 64, 300)], ids=["verify", "prefill"])
+def test_multiquery_fp8_rows_past_the_context_are_never_used(q_lens):
+    ctxs = (300, 129, 100, 700)
+    spec = W.DecodeSpec("mqf8nan", len(ctxs), 16, 2, 128, 16, torch.bfloat16, FP8, ("list", ctxs), ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=32, device=DEV)
+    _poison_unused_rows(mw.base)
+    for pt in (0, 128, 32):
+        out = _mq_check(mw, partition_tokens=pt, what=f"fp8 poisoned pool pt={pt}")
+        assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_multiquery_fp8_random_shapes(seed):
+    """Seeded random mixes over fp8 caches: grouping, block size, context and query lengths, partition."""
+    rng = np.random.default_rng(500 + seed)
+    hkv = int(rng.choice([1, 2, 4]))
+    g = int(rng.choice([1, 2, 4, 8]))
+    bs = int(rng.choice([16, 32]))
+    B = int(rng.integers(1, 7))
+    ctxs = tuple(int(c) for c in rng.integers(1, 1500, B))
+    q_lens = tuple(int(min(c, rng.choice([0, 1, 3, 5, 9, 40, 200, c]))) for c in ctxs)
+    spec = W.DecodeSpec("mqf8rand", B, hkv * g, hkv, 128, bs, torch.bfloat16, FP8, ("list", ctxs), ("slack", 1.3))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=600 + seed, device=DEV)
+    pt = int(rng.choice([0, bs, 4 * bs, 512]))
+    _mq_check(mw, partition_tokens=pt,
+              what=f"fp8 seed={seed} g={g} hkv={hkv} bs={bs} ctxs={ctxs} q_lens={q_lens} pt={pt}")
+
+
+def test_multiquery_fp8_one_query_per_sequence_matches_decode():
+    spec = W.GQA_BATCH.with_(num_seqs=5, ctx=("list", (1, 40, 300, 17, 1000)))
+    mw = W.make_multiquery_workload(spec, (1,) * 5, seed=33, device=DEV)
+    w = mw.base
+    mq = pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                       mw.query_start_loc, w.scale, k_scale=w.k_scale, v_scale=w.v_scale)
+    dec = pk.paged_attention_decode(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, w.scale,
+                                    k_scale=w.k_scale, v_scale=w.v_scale)
+    torch.cuda.synchronize()
+    assert_close(f64(mq), f64(dec), *TOL_FP8, what="fp8 multi-query vs fp8 decode")
+
+
+def test_multiquery_fp8_rejects_missing_scales():
+    spec = W.GQA_BATCH.with_(num_seqs=2, ctx=("list", (40, 30)))
+    mw = W.make_multiquery_workload(spec, (3, 3), seed=34, device=DEV)
+    w = mw.base
+    with pytest.raises(pk.PagedKVError):
+        pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                                      mw.query_start_loc, w.scale, k_scale=0.0, v_scale=w.v_scale)
