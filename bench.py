@@ -363,7 +363,7 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
                   host["context_lens"], w.key_cache, w.value_cache, w.scale, copy_pairs=host["copy_pairs"],
                   k_scale=w.k_scale, v_scale=w.v_scale)
 
-    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e2e_steps = max(1, args.e2e_steps)  # its own count: the two-deep pipeline's fill and drain amortised
     for _ in range(min(args.warmup, 10)):
         e2e_step()
     pipe.synchronize()
@@ -549,7 +549,7 @@ def measure_multiquery(name, args, dev, rank, world, clocks):
     gbs = kv_bytes / (step_ms * 1e-3) / 1e9
     tflops = flops / (step_ms * 1e-3) / 1e12
     tensor_bound = flops / max(kv_bytes, 1) > peak_tf * 1e12 / (peak_gbs * 1e9)
-    tc = n * (s.num_q_heads // s.num_kv_heads) > 16 and s.cache_dtype == torch.bfloat16
+    tc = n * (s.num_q_heads // s.num_kv_heads) > 16  # the library's kernel split (both cache types)
     res = {
         "value": round(total_kv / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(step_ms, 5),
         "steps": steps, "dtype": DTYPE_NAMES[s.cache_dtype],
@@ -584,9 +584,11 @@ OPS = ("kv_write", "block_copy", "swap", "amax", "table_scan")
 
 
 def measure_op(op, args, dev):
-    """Times one library call on the workload's tensors, one CUDA event pair
-    around K back-to-back calls.  Bytes are the call's algorithmic bytes: read
-    + written for the copies and the write, read for amax and the table scan."""
+    """Times one library call on the workload's tensors: K back-to-back calls
+    captured in a CUDA graph and replayed between one CUDA event pair (device
+    time; the eager loop of K calls is reported beside it, host launch cost
+    included).  Bytes are the call's algorithmic bytes: read + written for the
+    copies and the write, read for amax and the table scan."""
     import paged_kv_cache_450_b200 as pk
 
     spec = workload_spec(args)
@@ -602,7 +604,7 @@ def measure_op(op, args, dev):
 
         def call():
             pk.paged_kv_write(w.new_k, w.new_v, w.slot_mapping, w.key_cache, w.value_cache, k_scale=w.k_scale,
-                              v_scale=w.v_scale, stream=stream)
+                              v_scale=w.v_scale, stream=torch.cuda.current_stream(dev))
         kernel = "paged_kv_write_kernel"
     elif op == "block_copy":
         if w.copy_pairs is None:
@@ -611,7 +613,7 @@ def measure_op(op, args, dev):
         nbytes = 2 * 2 * n * blk  # K and V, read + written
 
         def call():
-            pk.kv_block_copy(w.copy_pairs, w.key_cache, w.value_cache, stream=stream)
+            pk.kv_block_copy(w.copy_pairs, w.key_cache, w.value_cache, stream=torch.cuda.current_stream(dev))
         kernel = "kv_block_copy_kernel"
     elif op == "swap":
         n = min(args.swap_blocks, w.num_blocks)
@@ -622,7 +624,7 @@ def measure_op(op, args, dev):
         nbytes = 2 * n * blk  # K and V over the host link, one direction
 
         def call():
-            pk.swap_blocks(pairs_out, w.key_cache, w.value_cache, host_k, host_v, stream=stream)
+            pk.swap_blocks(pairs_out, w.key_cache, w.value_cache, host_k, host_v, stream=torch.cuda.current_stream(dev))
         kernel = "kv_block_copy_kernel (device -> pinned host)"
         extra = {"blocks": n, "direction": "device to pinned host (swap out)"}
     elif op == "amax":
@@ -633,7 +635,7 @@ def measure_op(op, args, dev):
         scale = torch.empty((1,), dtype=torch.float32, device=dev)
 
         def call():
-            pk.fp8_scale_from_amax(x, out=scale, stream=stream)
+            pk.fp8_scale_from_amax(x, out=scale, stream=torch.cuda.current_stream(dev))
         kernel = "amax_kernel + fp8_scale_finish_kernel"
     elif op == "table_scan":
         MB = w.block_tables.shape[1]
@@ -645,7 +647,7 @@ def measure_op(op, args, dev):
 
         def call():
             pk.decode_table_scan(w.block_tables, w.context_lens, s.num_kv_heads, s.block_size, w.num_blocks, pt,
-                                 sink=sink, stream=stream)
+                                 sink=sink, stream=torch.cuda.current_stream(dev))
         kernel = "decode_table_scan_kernel"
         extra = {"partition_tokens": pt, "bytes_note": "block-id reads of every CTA (each KV head's CTAs re-read "
                                                       "the sequence's ids)"}
@@ -660,11 +662,28 @@ def measure_op(op, args, dev):
         call()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / args.steps
+    eager_ms = a.elapsed_time(b) / args.steps
+    timing = "CUDA graph of the calls, replayed between one event pair"
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(args.steps):
+                call()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / args.steps
+        del g
+    except Exception as e:  # capture not possible here: the eager loop stands
+        ms, timing = eager_ms, f"eager loop (graph capture failed: {type(e).__name__})"
     assert pk.device_status(clear=True) == 0
     return {"metric": f"{op} GB/s", "op": op, "kernel": kernel, "value": round(nbytes / (ms * 1e-3) / 1e9, 2),
-            "unit": "GB/s", "ms_per_call": round(ms, 5), "bytes_per_call": int(nbytes), "steps": args.steps,
-            "warmup": args.warmup, "config": {"workload": s.name, **extra}}
+            "unit": "GB/s", "ms_per_call": round(ms, 5), "eager_ms_per_call": round(eager_ms, 5),
+            "timing": timing, "bytes_per_call": int(nbytes), "steps": args.steps, "warmup": args.warmup,
+            "config": {"workload": s.name, **extra}}
 
 
 # --------------------------------------------------------------------------- #
@@ -819,7 +838,7 @@ def parse_args(argv=None):
     ap.add_argument("--swap-blocks", type=int, default=4096, help="blocks moved by --op swap")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition-tokens", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=200, help="steps of the end-to-end (host buffers) timing")
     ap.add_argument("--cpu-budget", type=float, default=16.0,
                     help="seconds of oracle work for the headline's cpu_baseline (half for the other configs)")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")

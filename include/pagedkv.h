@@ -307,16 +307,14 @@ int pkv_kv_block_copy(const int64_t* src_dst_pairs, int64_t num_pairs, void* key
  * workspace         device scratch of pkv_multiquery_workspace_bytes(...) bytes
  *                   (same arguments; 0 when no split is needed), 256-byte aligned.
  * Supported: bf16 q, bf16 or fp8 E4M3 caches, head_dim 128, block_size 16 or
- * 32, 1/2/4/8 query heads per KV head.  Runs on the tensor cores.  bf16
- * caches: up to 16 rows per (sequence, KV head) -- rows = max_q_len x query
- * heads per KV head -- on mma.sync m16n8k16 (bf16 operands, P as a bf16 high
- * part and residual); more rows (prefill) on tcgen05 with 128-row tiles and
- * 128-token KV tiles (bf16 Q.K^T; P.V on fp16 operands, V converted from bf16
- * in shared memory, exact for |v| in [2^-14, 65504] -- V beyond the fp16
- * range is not supported).  fp8 caches: mma.sync for every row count, the
- * codes widened exactly to fp16 in shared memory, q rounded once to fp16
- * (exact for |q| in [2^-14, 65504]), fp16 P.  Other arguments and errors: as
- * pkv_paged_attention_decode.
+ * 32, 1/2/4/8 query heads per KV head.  Runs on the tensor cores: up to 16
+ * rows per (sequence, KV head) -- rows = max_q_len x query heads per KV head
+ * -- on mma.sync m16n8k16; more rows (prefill, grouped verification) on
+ * tcgen05 with 128-row tiles and 128-token KV tiles.  bf16 caches: bf16
+ * operands, P as a bf16 high part and residual (~16 significant bits).  fp8
+ * caches: the codes widened exactly to fp16 in shared memory, q rounded once
+ * to fp16 (exact for |q| in [2^-14, 65504]), fp16 operands and one fp16 P, in
+ * both kernels.  Other arguments and errors: as pkv_paged_attention_decode.
  */
 int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cache, const void* value_cache,
                                    const int32_t* block_tables, const int32_t* context_lens,
@@ -526,6 +524,19 @@ int64_t pkv_prefix_cache_evict(void* cache, int64_t max_evict, int32_t* evicted_
 int pkv_decode_table_scan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_kv_heads,
                           int block_size, int max_blocks_per_seq, int64_t num_blocks, int partition_tokens,
                           unsigned* sink, size_t sink_words, void* stream);
+
+/*
+ * Self-test of the failure reporting (the pages have no counterpart).  Every
+ * wait inside the library's kernels gives up after a time limit, sets
+ * PKV_STATUS_WAIT_TIMEOUT in the device status word and lets the kernel
+ * return.  This call runs that path on purpose: one warp waits, through the
+ * same bounded-wait helper, on an mbarrier that nothing completes, for
+ * limit_ns nanoseconds (at most 0.1 s); no copy or MMA is started, so nothing
+ * is in flight when it gives up.  Afterwards PKV_STATUS_WAIT_TIMEOUT is set
+ * and *gave_up (device unsigned) is 1; the context stays usable.
+ * Errors: PKV_ERR_BAD_SHAPE (limit outside (0, 1e8]), _NULL_POINTER, _CUDA.
+ */
+int pkv_selftest_wait_timeout(int64_t limit_ns, unsigned* gave_up, void* stream);
 
 /*
  * Reads the current device's status word (PKV_STATUS_* bits) into *status,

@@ -47,6 +47,7 @@ SIGNATURES = {
     "pkv_prefix_cache_insert": (I64, [P, P, I64, U64, P, I64]),
     "pkv_prefix_cache_release": (I64, [P, P, I64, U64, I64]),
     "pkv_prefix_cache_evict": (I64, [P, I64, P]),
+    "pkv_selftest_wait_timeout": (I, [I64, P, P]),
     "pkv_decode_table_scan": (I, [P, P, I, I, I, I, I64, I, P, SZ, P]),
     "pkv_device_status": (I, [ctypes.POINTER(ctypes.c_uint), I, P]),
     "pkv_launch_count": (U64, []),

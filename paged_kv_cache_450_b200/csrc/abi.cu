@@ -453,8 +453,9 @@ static int mq_partition_tokens(int num_seqs, int num_kv_heads, int group, int ma
   const int64_t rows = static_cast<int64_t>(max_q_len) * group;
   // CTAs per (sequence, KV head) and resident CTAs per SM of the kernel that
   // serves these rows: 16- to 64-row mma.sync CTAs (6 to 2 per SM), or 128-row
-  // tcgen05 CTAs (1 per SM; bf16 caches only)
-  const bool tc = !fp8 && multiquery_uses_tc(static_cast<int>(rows > 0x7fffffff ? 0x7fffffff : rows));
+  // tcgen05 CTAs (1 per SM)
+  (void)fp8;  // the same kernel split for both cache types
+  const bool tc = multiquery_uses_tc(static_cast<int>(rows > 0x7fffffff ? 0x7fffffff : rows));
   const int nwc = multiquery_compute_warps(static_cast<int>(rows > 64 ? 64 : rows));
   const int tile = tc ? 128 : 16 * nwc;
   const int per_sm = tc ? 1 : multiquery_ctas_per_sm(nwc);
@@ -578,17 +579,27 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   p.out_scale = fp8 ? v_scale : 1.f;
   const int rows_per_seq = max_q_len * group;
   if (rows_per_seq <= 0) return PKV_OK;
-  if (fp8)
-    return launch_multiquery_mma_fp8(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
-                                                                                                    : PKV_ERR_CUDA;
   if (multiquery_uses_tc(rows_per_seq)) {
     CUtensorMap qmap;
     if (!encode_query_map(&qmap, q, total_q, num_q_heads, group)) return PKV_ERR_TENSOR_MAP;
-    return launch_multiquery_tc(qmap, kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
-                                                                                                     : PKV_ERR_CUDA;
+    return launch_multiquery_tc(qmap, kmap, vmap, p, group, rows_per_seq, fp8, P > 1, st) == cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_CUDA;
   }
-  return launch_multiquery_mma_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st) == cudaSuccess ? PKV_OK
-                                                                                                  : PKV_ERR_CUDA;
+  const cudaError_t e = fp8 ? launch_multiquery_mma_fp8(kmap, vmap, p, group, rows_per_seq, P > 1, st)
+                            : launch_multiquery_mma_bf16(kmap, vmap, p, group, rows_per_seq, P > 1, st);
+  return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_selftest_wait_timeout(int64_t limit_ns, unsigned* gave_up, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 100000000LL) return PKV_ERR_BAD_SHAPE;
+  if (!gave_up) return PKV_ERR_NULL_POINTER;
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  return launch_wait_timeout_selftest(status, static_cast<uint64_t>(limit_ns), gave_up,
+                                      static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PKV_OK
+             : PKV_ERR_CUDA;
 }
 
 int pkv_decode_table_scan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_kv_heads,

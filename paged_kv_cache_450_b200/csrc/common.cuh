@@ -87,13 +87,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for phase `parity` of the barrier to complete.  Gives up after
-// kWaitLimitNs, sets PKV_STATUS_WAIT_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned* status) {
+// limit_ns (kWaitLimitNs in every kernel of the library; the self-test uses a
+// shorter one), sets PKV_STATUS_WAIT_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, PKV_STATUS_WAIT_TIMEOUT);
       return false;
     }
@@ -140,6 +142,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Four E4M3 codes (bytes 0..3 of w) -> two fp16x2 words: lo = bytes {0,1}, hi = bytes {2,3}
+// (the lower byte of each pair lands in the lower half).  Exact: every E4M3
+// value is an fp16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -57,15 +57,6 @@ struct MmaTraits {
   }
 };
 
-// Four E4M3 codes (bytes 0..3 of w) -> two fp16x2 words: lo = bytes {0,1}, hi = bytes {2,3}
-// (the lower byte of each pair lands in the lower half).
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
 __device__ __forceinline__ uint32_t f16x2_pack(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);

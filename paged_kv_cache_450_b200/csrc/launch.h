@@ -65,6 +65,9 @@ cudaError_t launch_table_scan(const int32_t* tables, const int32_t* lens, int nu
                               int max_blocks_per_seq, int num_blocks, int block_size, int partition_blocks,
                               int num_partitions, unsigned* sink, unsigned* status, cudaStream_t st);
 
+// A warp waits on an mbarrier nothing completes, with a short limit (selftest.cu).
+cudaError_t launch_wait_timeout_selftest(unsigned* status, uint64_t limit_ns, unsigned* gave_up, cudaStream_t st);
+
 // The tensor-core decode kernels serve head_dim 128 with 16- or 32-token
 // blocks: fp8 caches with 8 query heads per KV head, and bf16 caches with 2,
 // 4 or 8 (grouped-query attention, where CUDA-core work grows with the
@@ -80,13 +83,12 @@ inline bool decode_uses_mma(int cache_dtype, int head_dim, int group, int block_
 }
 
 // Multi-query (prefill / verification) attention: bf16 q, bf16 or fp8 caches,
-// head_dim 128, bs 16/32.  bf16 caches: up to 16 rows per (sequence, KV head)
+// head_dim 128, bs 16/32.  Up to 16 rows per (sequence, KV head)
 // -- rows = queries x query heads of the group -- run on the mma.sync kernel
 // (one 16-row warp per CTA); more rows on the tcgen05 kernel with 128-row
 // tiles, whose time per KV tile does not depend on how many of the rows are
 // used (measured: 40 rows, 70B-GQA verification, 2.70 TB/s on mma.sync with
-// three 16-row warps, 3.56 TB/s on tcgen05).  fp8 caches: the mma.sync kernel
-// for every row count.
+// three 16-row warps, 3.56 TB/s on tcgen05).  The same split for fp8 caches.
 #ifndef PKV_MQ_TC_MIN_ROWS
 #define PKV_MQ_TC_MIN_ROWS 16
 #endif
@@ -106,7 +108,7 @@ cudaError_t launch_multiquery_mma_bf16(const CUtensorMap& kmap, const CUtensorMa
 cudaError_t launch_multiquery_mma_fp8(const CUtensorMap& kmap, const CUtensorMap& vmap, const MultiQueryParams& p,
                                       int group, int rows_per_seq, bool reduce, cudaStream_t st);
 cudaError_t launch_multiquery_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                                 const MultiQueryParams& p, int group, int rows_per_seq, bool reduce,
+                                 const MultiQueryParams& p, int group, int rows_per_seq, bool fp8, bool reduce,
                                  cudaStream_t st);
 // The split-context merge of either multi-query kernel.
 cudaError_t launch_multiquery_reduce(const MultiQueryParams& p, cudaStream_t st);

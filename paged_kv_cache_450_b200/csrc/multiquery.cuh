@@ -26,9 +26,8 @@
 // once to fp16, and both contractions run on fp16 operands with one fp16 P
 // (11 significant bits).  The K scale is folded into the logit scale and the
 // V scale into the output.
-// The dispatch (launch.h) sends bf16 caches here up to 16 rows per (sequence,
-// KV head) -- more rows go to the tcgen05 kernel (multiquery_tc.cuh) -- and
-// fp8 caches for every row count.
+// The dispatch (launch.h) sends it up to 16 rows per (sequence, KV head), for
+// either cache type; more rows go to the tcgen05 kernel (multiquery_tc.cuh).
 #pragma once
 
 #include "decode.cuh"

@@ -18,15 +18,14 @@
 // Q, K and V sit in shared memory in the 128-byte-swizzled layout (two
 // 64-element halves of every 256-byte row) as TMA delivers them; Q and K are
 // K-major operands, V (stored token-major, dims contiguous) is the N-major B
-// operand of P . V, so no transpose is ever made.  S = Q . K^T runs on bf16
-// operands.  P . V runs on fp16 operands: P never touches shared memory -- it
-// is the TMEM A operand (fp16, columns [384, 448)) -- and each V tile is
-// converted from bf16 to fp16 in place in shared memory by the softmax warps
-// before its P . V.  fp16 keeps 11 significant bits of each probability (a
-// bf16 P, 8 bits, costs up to ~3e-3 absolute on short contexts); the
-// conversion of V is exact for |v| in [2^-14, 65504] (smaller magnitudes
-// lose at most 2^-25 absolute; V beyond the fp16 range is not supported).
-// Eleven warps:
+// operand of P . V, so no transpose is ever made.  P never touches shared
+// memory: it is the TMEM A operand of P . V (columns [384, 512)).  With bf16
+// caches it is split into a bf16 high part and a bf16 residual -- two MMAs per
+// k-step -- so each probability keeps ~16 significant bits (a bf16 P alone
+// costs up to ~3e-3 absolute on short contexts), packed with integer byte
+// permutes.  (One fp16 P over V converted to fp16 in shared memory halves the
+// P . V MMAs but measured 1.7x slower: the conversions compete with the
+// exponentials.)  Eleven warps:
 //   warps 0-7  softmax: warp w serves rows 32 (w & 3) .. +31 (the TMEM lanes
 //              its sub-partition may touch) and half h = w >> 2 of every KV
 //              tile's tokens.  The two halves are independent online
@@ -37,17 +36,22 @@
 //              once, in the epilogue.  Per tile a thread reads its 64 scores
 //              from TMEM, applies the causal / context mask, keeps a
 //              reference max (O_h is rescaled only when a score passes it by
-//              more than 2^8), writes its 64 probabilities into P_h, and
-//              converts one 128-byte V row segment of its half to fp16 (rows
-//              past the loaded tokens or of a bad block are zeroed instead).
-//   warp 8     TMA producer of Q (once) and the K tiles (two-stage ring; one
+//              more than 2^8), and writes its 64 probabilities into P_h.
+//   warp 8     TMA producer of Q (once) and the K tiles (three-stage ring; one
 //              4-D box per block and 64-dim half); owns the TMEM allocation.
-//   warp 10    TMA producer of the V tiles (three-stage ring: a V tile is
-//              used one tile period after its K tile, after its conversion),
-//              so that a K load never waits behind a V stage P . V still holds.
+//   warp 10    TMA producer of the V tiles (two-stage ring), so that a K load
+//              never waits behind a V stage that P . V still holds.
 //   warp 9     MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
+// Caches of fp8 (E4M3, F8 = true): the K and V producer warps TMA each tile's
+// raw codes (128 bytes per token row) into two-slot rings of their own and
+// then, all 32 lanes, widen them exactly to fp16 into the operand buffers (K:
+// one buffer, V: two; V rows that must not contribute are zeroed there); the
+// softmax warps round their Q rows to fp16 once; both MMAs run on fp16
+// operands, and P is one fp16 value (11 significant bits; columns [384,
+// 448)).  The K scale is folded into the logit scale, the V scale into the
+// output.
 // Every wait is bounded (2 s); on a timeout the status bit is set, the
 // producer and issuer loops stop, the softmax warps skip their remaining
 // waits, in-flight work is drained with bounded waits and TMEM is freed.
@@ -59,28 +63,35 @@
 
 namespace pkv {
 
-template <int BS>
+template <int BS, bool F8 = false>
 struct MqTcTraits {
   static constexpr int D = 128;
   static constexpr int ROWS = 128;           // query rows per CTA (MMA M)
   static constexpr int TOK = 128;            // tokens per KV tile
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
-  static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16)
-  static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 bf16
-  static constexpr int NSK = 2, NSV = 3;  // K ring and V ring depth
+  static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
+  static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 16-bit values
+  // K and V operand buffers: TMA rings for bf16 caches; for fp8 caches the
+  // buffers the producers widen into (K one, V two), fed by raw rings of RAW
+  static constexpr int NSK = F8 ? 1 : 3, NSV = 2;
+  static constexpr int RAW = 128 * 128;      // 16 KB: 128 rows x 128 fp8 codes
+  static constexpr int NR = F8 ? 2 : 0;      // raw ring depth of K and of V
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
-  static constexpr int BAR_OFF = V_OFF + NSV * TILE;
+  static constexpr int RAWK_OFF = V_OFF + NSV * TILE;
+  static constexpr int RAWV_OFF = RAWK_OFF + NR * RAW;
+  static constexpr int BAR_OFF = RAWV_OFF + NR * RAW;
   // mbarriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free, p_full[2],
-  // pv_done[2], mma_done (the pairs: one per token half)
-  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7;
+  // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, rk_full[NR], rv_full[NR]
+  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + 2 * NR : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [4][128 rows]: m_0, m_1, l_0, l_1
   static constexpr int IDS_OFF = XCH_OFF + 4 * 128 * 4;
   static constexpr int THREADS = 352;
   static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
-  static constexpr uint32_t TMEM_COLS = 512;  // S 128 | O_0 128 | O_1 128 | P_0, P_1 (32 + 32 packed fp16 pairs)
+  // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or fp16 0,1 (32 + 32)
+  static constexpr uint32_t TMEM_COLS = 512;
   static constexpr size_t smem_bytes(int pb) { return 1024 + IDS_OFF + static_cast<size_t>(pb) * 4; }
 };
 
@@ -107,11 +118,65 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
   return __all_sync(kFullMask, mbar_wait_bounded(bar, parity, status));
 }
 
-template <int BS, int G>
-__global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
+// Longest work first.  CTAs start roughly in grid order and one runs per SM,
+// so the tail of a launch is set by the long units that start last.  Grid z
+// index z therefore takes the sequence whose context is the z-th longest
+// (ties by index: a permutation of the sequences); every thread of the CTA
+// takes part (two CTA barriers).  More than 1024 sequences keep grid order.
+__device__ __forceinline__ int longest_first_sequence(const MultiQueryParams& p, int z, int* slot) {
+  const int B = p.num_seqs;
+  if (B > 1024) return z;
+  if (threadIdx.x == 0) *slot = z;
+  __syncthreads();
+  for (int t = threadIdx.x; t < B; t += blockDim.x) {
+    const int lt = p.context_lens[t];
+    int rank = 0;
+    for (int j = 0; j < B; ++j) {
+      const int lj = p.context_lens[j];
+      rank += (lj > lt) || (lj == lt && j < t);
+    }
+    if (rank == z) *slot = t;
+  }
+  __syncthreads();
+  return *slot;
+}
+
+// Widens one KV tile of raw E4M3 codes (128 token rows x 128 codes, 128-byte
+// swizzle) to fp16 in the operand layout (two 64-dim halves of 128 rows x 128
+// bytes, 128-byte swizzle): raw chunk q of row t (dims 16q .. 16q+15) becomes
+// chunks 2(q % 4) and 2(q % 4) + 1 of half q / 4.  Rows for which zero_row(t)
+// holds are written as zeros.  One warp; each lane then orders its writes
+// before the tensor core's (async proxy) reads.
+template <typename ZeroRow>
+__device__ __forceinline__ void widen_e4m3_tile(const uint8_t* raw, uint8_t* dst, int lane, ZeroRow zero_row) {
+  constexpr int HALF = 128 * 128;
+#pragma unroll 4
+  for (int i = lane; i < 128 * 8; i += 32) {
+    const int t = i >> 3, q = i & 7;
+    uint32_t f[8];
+    if (zero_row(t)) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0u;
+    } else {
+      const uint4 w = *reinterpret_cast<const uint4*>(raw + t * 128 + ((q ^ (t & 7)) << 4));
+      e4m3x4_to_f16x2x2(w.x, f[0], f[1]);
+      e4m3x4_to_f16x2x2(w.y, f[2], f[3]);
+      e4m3x4_to_f16x2x2(w.z, f[4], f[5]);
+      e4m3x4_to_f16x2x2(w.w, f[6], f[7]);
+    }
+    uint8_t* row = dst + (q >> 2) * HALF + t * 128;
+    const int c0 = 2 * (q & 3);
+    *reinterpret_cast<uint4*>(row + ((c0 ^ (t & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (t & 7)) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
+  }
+  fence_proxy_async_smem();
+}
+
+template <int BS, int G, bool F8>
+__global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     paged_multiquery_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap, const MultiQueryParams p) {
-  using T = MqTcTraits<BS>;
+  using T = MqTcTraits<BS, F8>;
   constexpr int D = T::D;
   constexpr int QPT = T::ROWS / G;  // queries per CTA tile
   pdl_wait_and_release();
@@ -120,7 +185,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   int* ids = reinterpret_cast<int*>(data + T::IDS_OFF);
 
   const int Hkv = p.num_kv_heads;
-  const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y, b = blockIdx.z;
+  __shared__ int seq_slot;
+  const int b = longest_first_sequence(p, blockIdx.z, &seq_slot);
+  // the last query tile of a sequence sees the most tokens: it goes first
+  const int hk = blockIdx.x % Hkv, qt = gridDim.x / Hkv - 1 - blockIdx.x / Hkv, part = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int q0, q_len;
   if (!query_rows_ok(p, b, q0, q_len)) {  // before any load or store
@@ -174,6 +242,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1), mma_done = bar0 + 8 * (B2 + 6);
   auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
   auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
+  // fp8 caches: Q rounded to fp16, raw K / V tiles landed
+  constexpr int B3 = B2 + 7;
+  const uint32_t q_ready = bar0 + 8 * B3;
+  auto rk_full = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
+  auto rv_full = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NR + s); };
   const uint64_t policy = l2_policy_evict_first();
   const int* table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb;
   if (warp == T::W_K) {
@@ -197,6 +270,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         mbar_init(pv_done(h), 1);
       }
       mbar_init(mma_done, 1);
+      if constexpr (F8) {
+        mbar_init(q_ready, 8);
+        for (int s = 0; s < T::NR; ++s) {
+          mbar_init(rk_full(s), 1);
+          mbar_init(rv_full(s), 1);
+        }
+      }
       fence_barrier_init();
       mbar_arrive_expect_tx(q_full, T::TILE);
       tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
@@ -209,15 +289,21 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
       if (id < 0 || id >= p.num_blocks) id = -1;  // (reported by the scan below)
     }
     const unsigned valid = __ballot_sync(kFullMask, id >= 0);
+    // bf16: the tile straight into K buffer 0; fp8: the raw codes into raw slot 0
+    const uint32_t kbar = F8 ? rk_full(0) : k_full(0);
     if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(__popc(valid)) * 2u * BS * 128u;
-      if (bytes) mbar_arrive_expect_tx(k_full(0), bytes); else mbar_arrive(k_full(0));
+      const uint32_t bytes = static_cast<uint32_t>(__popc(valid)) * (F8 ? 1u : 2u) * BS * 128u;
+      if (bytes) mbar_arrive_expect_tx(kbar, bytes); else mbar_arrive(kbar);
     }
     __syncwarp();
     if (id >= 0) {
-      const uint32_t dst = base + T::K_OFF + lane * BS * 128;
-      tma_load_4d(dst, &kmap, k_full(0), 0, hk, 0, id, policy);
-      tma_load_4d(dst + T::HALF, &kmap, k_full(0), 64, hk, 0, id, policy);
+      if constexpr (F8) {
+        tma_load_4d(base + T::RAWK_OFF + lane * BS * 128, &kmap, kbar, 0, hk, 0, id, policy);
+      } else {
+        const uint32_t dst = base + T::K_OFF + lane * BS * 128;
+        tma_load_4d(dst, &kmap, k_full(0), 0, hk, 0, id, policy);
+        tma_load_4d(dst + T::HALF, &kmap, k_full(0), 64, hk, 0, id, policy);
+      }
     }
   }
 
@@ -243,9 +329,63 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(data + T::SLOT_OFF);
   const uint32_t tmem_s = tmem;
   auto tmem_o = [&](int h) { return tmem + 128 + 128 * h; };
-  auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };  // tokens 64h .. 64h+63, fp16 packed in pairs
+  auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };    // tokens 64h .. 64h+63 packed in pairs: hi / fp16
+  auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };  // bf16 caches: the residual
 
-  if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
+  if (F8 && (warp == T::W_K || warp == T::W_V)) {  // ---------- fp8: load raw tiles, widen to fp16 ----------
+    const bool is_k = warp == T::W_K;
+    const CUtensorMap* map = is_k ? &kmap : &vmap;
+    const uint32_t raw_area = base + (is_k ? T::RAWK_OFF : T::RAWV_OFF);
+    const int nd = is_k ? T::NSK : T::NSV;
+    auto raw_full = [&](int s) { return is_k ? rk_full(s) : rv_full(s); };
+    auto issue_raw = [&](int j) {  // lane 0: tile j's raw codes into slot j % NR
+      const int r = j % T::NR;
+      const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
+      int nvalid = 0;
+      for (int i = i0; i < i1; ++i) nvalid += ids[i] >= 0;
+      const uint32_t bytes = static_cast<uint32_t>(nvalid) * BS * 128u;
+      if (bytes) mbar_arrive_expect_tx(raw_full(r), bytes); else mbar_arrive(raw_full(r));
+      for (int i = i0; i < i1; ++i)
+        if (ids[i] >= 0) tma_load_4d(raw_area + r * T::RAW + (i - i0) * BS * 128, map, raw_full(r), 0, hk, 0, ids[i], policy);
+    };
+    int issued = is_k ? 1 : 0;  // K tile 0 was issued in the prologue
+    if (lane == 0)
+      for (int j = issued; j < min(nt, T::NR); ++j) issue_raw(j);
+    issued = min(nt, T::NR);
+    int landed = 0;
+    for (int j = 0; j < nt; ++j) {
+      const int r = j % T::NR, d = j % nd;
+      if (!__all_sync(kFullMask, mbar_wait_bounded(raw_full(r), (j / T::NR) & 1, p.status))) break;
+      landed = j + 1;
+      if (j >= nd && !__all_sync(kFullMask, mbar_wait_bounded(is_k ? k_empty(d) : v_empty(d), ((j / nd) - 1) & 1,
+                                                              p.status)))
+        break;
+      const uint8_t* src = data + (is_k ? T::RAWK_OFF : T::RAWV_OFF) + r * T::RAW;
+      uint8_t* dst = data + (is_k ? T::K_OFF : T::V_OFF) + d * T::TILE;
+      const int tile0 = tok_begin + j * T::TOK;
+      if (is_k) {  // scores of rows that are not loaded are masked, whatever these rows hold
+        widen_e4m3_tile(src, dst, lane, [](int) { return false; });
+      } else {     // V rows that must not contribute (past tok_end, bad blocks) are zeroed
+        widen_e4m3_tile(src, dst, lane, [&](int t) {
+          return tile0 + t >= tok_end || (any_bad && ids[(tile0 + t - tok_begin) / BS] < 0);
+        });
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(is_k ? k_full(d) : v_full(d));
+        if (j + T::NR < nt) {
+          fence_proxy_async_smem();  // the raw slot's reads before the next TMA write into it
+          issue_raw(j + T::NR);
+        }
+      }
+      if (j + T::NR < nt) issued = j + T::NR + 1;
+    }
+    // drain (bounded): the raw loads started have landed before exit
+    if (lane == 0) {
+      if (is_k) mbar_wait_bounded(q_full, 0, p.status);
+      for (int j = landed; j < issued; ++j) mbar_wait_bounded(raw_full(j % T::NR), (j / T::NR) & 1, p.status);
+    }
+  } else if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
     if (lane == 0) {
       const bool is_k = warp == T::W_K;
       const int ns = is_k ? T::NSK : T::NSV;
@@ -277,11 +417,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
     }
   } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, 1);
+      constexpr uint32_t idesc_s = F8 ? idesc_f16_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
-      bool ok = mbar_wait_bounded(q_full, 0, p.status);
+      bool ok = mbar_wait_bounded(F8 ? q_ready : q_full, 0, p.status);
       // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1)
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
@@ -303,14 +443,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
         if (j > 0) {
           const int jj = j - 1, sv = jj % T::NSV;
           const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
+          // the V tile (bf16: landed; fp8: widened)
+          if (!(ok = mbar_wait_bounded(v_full(sv), (jj / T::NSV) & 1, p.status))) break;
           for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
-            // P_h is in TMEM and the half's V rows are fp16 (the softmax warps waited for the tile)
             if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
               const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
               tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+              if constexpr (!F8) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
             }
             tc_commit(pv_done(h));
           }
@@ -339,6 +481,18 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
       if (ok) ok = warp_wait_bounded(bar, parity, p.status);
       return ok;
     };
+    if constexpr (F8) {  // this thread's Q row half to fp16, in place (exact for |q| in [2^-14, 65504])
+      wait(q_full, 0);
+      uint4* qrow = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + r * 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w = qrow[c];
+        qrow[c] = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
     for (int j = 0; j < nt; ++j) {
       const int t0 = tok_begin + j * T::TOK + 64 * h;  // first token of this half of the tile
       wait(s_full, j & 1);
@@ -400,47 +554,37 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
       }
       const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
       // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add, and at once the
-      // row's half of P as fp16 pairs (tokens 2k, 2k+1 in word k, round to nearest; p <= 2^8).  One
-      // loop, so the special-function unit (ex2) and the conversion pipe work side by side; the
-      // stores to TMEM wait below.
+      // row's half of P as packed pairs (tokens 2k, 2k+1 in word k).  bf16 caches: a high part (the
+      // top 16 bits of the fp32 value: truncation) and the residual (exact in fp32, then truncated to
+      // its top 16 bits), ~16 significant bits per probability, with integer ops only.  fp8 caches:
+      // one fp16 value (round to nearest; p <= 2^8).  One loop, so the special-function unit (ex2)
+      // and the integer / FMA pipes (packing) work side by side; the stores to TMEM wait below.
       const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
       float2 sum4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
-      uint32_t ph[32];
+      uint32_t ph[32], plo[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
         const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
         sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
-        const __half2 hp = __floats2half2_rn(a, bb);  // token 2k in the low half
-        ph[k] = *reinterpret_cast<const uint32_t*>(&hp);
+        if constexpr (F8) {
+          const __half2 hp = __floats2half2_rn(a, bb);  // token 2k in the low half
+          ph[k] = *reinterpret_cast<const uint32_t*>(&hp);
+          plo[k] = 0u;
+        } else {
+          const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
+          // residual = value - its truncation (the negated truncation is one logic op)
+          const float2 rr = __fadd2_rn(make_float2(a, bb),
+                                       make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
+                                                   __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
+          ph[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
+          plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+        }
       }
       const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
       l += s2.x + s2.y;
-      // This thread's 128-byte V row segment of the half tile to fp16, in place: row 64h + 16 quarter +
-      // lane / 2, dims half lane & 1.  Rows that must not contribute (past tok_end: never loaded; bad
-      // blocks: stale) are zeroed instead, since 0 * NaN would poison O.
-      {
-        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
-        const int vr = 64 * h + 16 * quarter + (lane >> 1);
-        const int t = tok_begin + j * T::TOK + vr;
-        uint4* vrow = reinterpret_cast<uint4*>(data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF +
-                                               vr * 128);
-        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
-        } else {
-          uint4 w[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) w[c] = vrow[c];
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            vrow[c] = make_uint4(bf16x2_to_f16x2(w[c].x), bf16x2_to_f16x2(w[c].y), bf16x2_to_f16x2(w[c].z),
-                                 bf16x2_to_f16x2(w[c].w));
-        }
-        fence_proxy_async_smem();  // the generic-proxy writes before the MMA (async proxy) reads them
-      }
       // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
       if (j > 0) {
         wait(pv_done(h), (j - 1) & 1);
@@ -458,13 +602,31 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
           }
         }
       }
+      // bf16 caches: V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed:
+      // 0 * NaN would poison O.  The 64 rows of this half: thread (quarter, lane) takes row
+      // 16 quarter + lane / 2, dims half lane & 1.  (fp8 caches: the V producer zeroed them.)
+      if (!F8 && (ragged || bad)) {
+        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
+        const int vr = 64 * h + 16 * quarter + (lane >> 1);
+        const int t = tok_begin + j * T::TOK + vr;
+        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
+          uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
+      }
       // this half of row r of P into TMEM lane r
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t pw[16];
+        uint32_t pw[16], lw[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) pw[k] = ph[16 * c + k];
+        for (int k = 0; k < 16; ++k) {
+          pw[k] = ph[16 * c + k];
+          lw[k] = plo[16 * c + k];
+        }
         tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
+        if constexpr (!F8) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -482,7 +644,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS>::THREADS, 1)
     const float M = fmaxf(l > 0.f ? m : -INFINITY, l_o > 0.f ? m_o : -INFINITY);
     const float w_self = l > 0.f ? fast_exp2(m - M) : 0.f, w_oth = l_o > 0.f ? fast_exp2(m_o - M) : 0.f;
     const float lsum = l * w_self + l_o * w_oth;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const float inv = lsum > 0.f ? p.out_scale / lsum : 0.f;
     const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
     const int64_t orow = static_cast<int64_t>(q0 + row / G) * Hq + hk * G + row % G;
 #pragma unroll 1

@@ -128,10 +128,10 @@ def test_multiquery_partition_and_workspace():
     P = -(-512 * 16 // pt)
     rows = 8 * 5 * 64 * P
     assert WS(8, 8 * 5, 5, 64, 8, 128, 16, 512, 0) == ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
-    # fp8 caches run on the mma.sync kernel (48-row CTAs, 3 per SM): 512 CTAs are not two waves there
-    pt8 = PT(64, 5, 64, 8, 16, 512, 0, F8)
-    assert pt8 % 256 == 0 and 256 <= pt8 < 8192
-    assert WS(64, 64 * 5, 5, 64, 8, 128, 16, 512, 0, F8) > 0
+    # fp8 caches follow the same kernel split (40 rows: tcgen05), hence the same partitions
+    assert PT(64, 5, 64, 8, 16, 512, 0, F8) == 8192
+    assert WS(64, 64 * 5, 5, 64, 8, 128, 16, 512, 0, F8) == 0
+    assert PT(8, 5, 64, 8, 16, 512, 0, F8) == pt
     # MHA verification (5 rows): 16-row CTAs, 6 per SM
     assert PT(64, 5, 32, 32, 16, 128, 0) > 0
     # explicit partition lengths: a multiple of the block size up to 16384 tokens

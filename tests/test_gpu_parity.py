@@ -714,3 +714,15 @@ def test_multiquery_fp8_rejects_missing_scales():
     with pytest.raises(pk.PagedKVError):
         pk.paged_attention_multiquery(mw.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
                                       mw.query_start_loc, w.scale, k_scale=0.0, v_scale=w.v_scale)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("hq,hkv,q_lens", [(4, 4, (1, 5, 16, 0, 3, 7)), (8, 4, (8, 1, 0, 5, 2, 8)),
+                                           (16, 4, (4, 1, 0, 2, 3, 4)), (16, 2, (2, 1, 0, 2, 1, 2))])
+def test_multiquery_fp8_verify_sized(bs, hq, hkv, q_lens):
+    # at most 16 rows per (sequence, KV head): the mma.sync kernel with its widening producer warp
+    ctxs = (9, 20, 700, 129, 2100, 64)
+    spec = W.DecodeSpec("mqf8v", len(ctxs), hq, hkv, 128, bs, torch.bfloat16, FP8, ("list", ctxs), ("slack", 1.2))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=bs * hq + hkv, device=DEV)
+    for pt in (0, bs, 512):
+        _mq_check(mw, partition_tokens=pt, what=f"fp8 verify bs={bs} hq={hq} hkv={hkv} pt={pt}")

@@ -670,3 +670,36 @@ def test_multiquery_chunked_prefill_is_consistent():
     second = oracle.paged_attention_multiquery(q[30:], np.array([0, 20], np.int32), kp, vp, tk,
                                                np.array([n], np.int32), scale=0.125)
     np.testing.assert_allclose(np.concatenate([first, second]), whole, rtol=1e-13, atol=1e-14)
+
+
+def test_multiquery_fp8_cache_bf16_q_equals_sdpa_on_scaled_codes():
+    """Multi-query over E4M3 caches with per-tensor scales and bf16 queries (grouped heads): torch's
+    fp64 SDPA, with a bottom-right causal mask, on the codes decoded by torch's own float8_e4m3fn and
+    multiplied by their scales, and on the bf16 queries decoded by torch."""
+    rng = np.random.default_rng(25)
+    ctxs, qlens = [5, 40, 70], [5, 3, 17]
+    Hq, Hkv, d, bs = 8, 2, 128, 16
+    codes = lambda c: rng.integers(0, 256, (c, Hkv, d)).astype(np.uint8)  # noqa: E731
+    ks, vs = [codes(c) for c in ctxs], [codes(c) for c in ctxs]
+    for arr in ks + vs:                       # no NaN codes (S.1111.111)
+        arr[(arr & 0x7F) == 0x7F] = 0x3F
+    order = rng.permutation(12)
+    tk, kp = page_logical(ks, bs, rng, num_blocks=12, order=order)
+    _, vp = page_logical(vs, bs, rng, num_blocks=12, order=order)
+    kp[(kp & 0x7F) == 0x7F] = 0
+    vp[(vp & 0x7F) == 0x7F] = 0
+    qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = bf16_bits(rng.standard_normal((int(qsl[-1]), Hq, d)))
+    k_scale, v_scale = float(np.float32(0.0173)), float(np.float32(0.0391))
+    scale = float(np.float32(1 / math.sqrt(d)))
+    out = oracle.paged_attention_multiquery(q, qsl, kp, vp, tk, np.array(ctxs, np.int32), scale=scale,
+                                            q_dtype=oracle.BF16, cache_dtype=oracle.E4M3, k_scale=k_scale,
+                                            v_scale=v_scale)
+    g = Hq // Hkv
+    for b, (c, n) in enumerate(zip(ctxs, qlens)):
+        qb = torch.from_numpy(bf16_value(q[qsl[b]:qsl[b + 1]])).permute(1, 0, 2)                       # [Hq, n, d]
+        kb = torch.from_numpy(fp8_value(ks[b], k_scale)).repeat_interleave(g, 1).permute(1, 0, 2)   # [Hq, c, d]
+        vb = torch.from_numpy(fp8_value(vs[b], v_scale)).repeat_interleave(g, 1).permute(1, 0, 2)
+        mask = torch.arange(c)[None, :] <= (c - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(out[qsl[b]:qsl[b + 1]], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
