@@ -233,10 +233,13 @@ int pkv_paged_attention_decode_static(void* out, const void* q, const void* key_
  * partition_tokens if it is non-zero, else the automatic choice.  The
  * automatic choice depends on the shape, on which kernel serves it
  * (cache_dtype, head_dim and the query-head group select it) and on the
- * current device's SM count: the largest power of two <= 4096 that still
- * splits the longest possible context (max_blocks_per_seq * block_size) into
- * at least 4 partitions and gives at least one CTA per resident slot of the
- * kernel; a single partition when that context is 512 tokens or less.
+ * current device's SM count.  A single partition when the longest possible
+ * context (max_blocks_per_seq * block_size) is 512 tokens or less.  With
+ * fewer (sequence, KV head) pairs than four waves of the kernel's resident
+ * CTAs: the largest power of two <= 4096 that splits that context into at
+ * least 4 partitions and gives at least three quarters of a wave of CTAs.
+ * With more pairs: the largest power of two <= 2048 that gives three quarters
+ * of a wave (so one partition for contexts up to 2048 tokens).
  * Returns a negative PKV_ERR_* code for unsupported arguments.  (This and the
  * other sizing helpers below are this library's; the pages have no
  * counterpart: the split-context partition is its design for long contexts.)

@@ -45,13 +45,14 @@
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
 // Caches of fp8 (E4M3, F8 = true): the K and V producer warps TMA each tile's
-// raw codes (128 bytes per token row) into two-slot rings of their own and
-// then, all 32 lanes, widen them exactly to fp16 into the operand buffers (K:
-// one buffer, V: two; V rows that must not contribute are zeroed there); the
-// softmax warps round their Q rows to fp16 once; both MMAs run on fp16
-// operands, and P is one fp16 value (11 significant bits; columns [384,
-// 448)).  The K scale is folded into the logit scale, the V scale into the
-// output.
+// raw codes (128 bytes per token row) into the upper half of the tile's own
+// ring stage and then, all 32 lanes, widen them exactly to fp16 in place (one
+// thread per token row reads the raw row whole, then writes its two fp16
+// halves; V rows that must not contribute are zeroed there) -- the rings have
+// the bf16 layout and depths, so widening overlaps the MMAs; the softmax warps
+// round their Q rows to fp16 once; both MMAs run on fp16 operands, and P is
+// one fp16 value (11 significant bits; columns [384, 448)).  The K scale is
+// folded into the logit scale, the V scale into the output.
 // Every wait is bounded (2 s); on a timeout the status bit is set, the
 // producer and issuer loops stop, the softmax warps skip their remaining
 // waits, in-flight work is drained with bounded waits and TMEM is freed.
@@ -71,20 +72,16 @@ struct MqTcTraits {
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
   static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 16-bit values
-  // K and V operand buffers: TMA rings for bf16 caches; for fp8 caches the
-  // buffers the producers widen into (K one, V two), fed by raw rings of RAW
-  static constexpr int NSK = F8 ? 1 : 3, NSV = 2;
-  static constexpr int RAW = 128 * 128;      // 16 KB: 128 rows x 128 fp8 codes
-  static constexpr int NR = F8 ? 2 : 0;      // raw ring depth of K and of V
+  // K and V rings (fp8 caches: the raw codes land in a stage's upper half and
+  // are widened to fp16 in place)
+  static constexpr int NSK = 3, NSV = 2;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
-  static constexpr int RAWK_OFF = V_OFF + NSV * TILE;
-  static constexpr int RAWV_OFF = RAWK_OFF + NR * RAW;
-  static constexpr int BAR_OFF = RAWV_OFF + NR * RAW;
+  static constexpr int BAR_OFF = V_OFF + NSV * TILE;
   // mbarriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free, p_full[2],
-  // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, rk_full[NR], rv_full[NR]
-  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + 2 * NR : 0);
+  // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, k_ready[NSK], v_ready[NSV]
+  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + NSK + NSV : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [4][128 rows]: m_0, m_1, l_0, l_1
   static constexpr int IDS_OFF = XCH_OFF + 4 * 128 * 4;
@@ -141,33 +138,48 @@ __device__ __forceinline__ int longest_first_sequence(const MultiQueryParams& p,
   return *slot;
 }
 
-// Widens one KV tile of raw E4M3 codes (128 token rows x 128 codes, 128-byte
-// swizzle) to fp16 in the operand layout (two 64-dim halves of 128 rows x 128
-// bytes, 128-byte swizzle): raw chunk q of row t (dims 16q .. 16q+15) becomes
-// chunks 2(q % 4) and 2(q % 4) + 1 of half q / 4.  Rows for which zero_row(t)
-// holds are written as zeros.  One warp; each lane then orders its writes
-// before the tensor core's (async proxy) reads.
+// Widens one KV tile of raw E4M3 codes in place.  The raw codes of token row
+// t (128 codes, 128 bytes) sit in the stage's upper half at line t, 16-byte
+// chunk q (dims 16q .. 16q+15) at position q ^ (t & 7) (128-byte swizzle);
+// the fp16 result is the operand layout -- dims 0..63 in the lower half,
+// 64..127 in the upper half, line t, chunk c at position c ^ (t & 7), raw
+// chunk q giving chunks 2(q % 4) and 2(q % 4) + 1 of half q / 4.  Each thread
+// takes whole rows (t = lane, lane + 32, ...): it reads the raw line fully
+// before it writes the same line, so no row is read after another thread
+// wrote it.  Rows for which zero_row(t) holds are written as zeros.  One warp;
+// each lane then orders its writes before the tensor core's (async proxy)
+// reads.
 template <typename ZeroRow>
-__device__ __forceinline__ void widen_e4m3_tile(const uint8_t* raw, uint8_t* dst, int lane, ZeroRow zero_row) {
+__device__ __forceinline__ void widen_e4m3_tile_in_place(uint8_t* stage, int lane, ZeroRow zero_row) {
   constexpr int HALF = 128 * 128;
-#pragma unroll 4
-  for (int i = lane; i < 128 * 8; i += 32) {
-    const int t = i >> 3, q = i & 7;
-    uint32_t f[8];
+#pragma unroll 1
+  for (int t = lane; t < 128; t += 32) {
+    uint8_t* line0 = stage + t * 128;
+    uint8_t* line1 = stage + HALF + t * 128;
+    const int sw = t & 7;
     if (zero_row(t)) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0u;
-    } else {
-      const uint4 w = *reinterpret_cast<const uint4*>(raw + t * 128 + ((q ^ (t & 7)) << 4));
-      e4m3x4_to_f16x2x2(w.x, f[0], f[1]);
-      e4m3x4_to_f16x2x2(w.y, f[2], f[3]);
-      e4m3x4_to_f16x2x2(w.z, f[4], f[5]);
-      e4m3x4_to_f16x2x2(w.w, f[6], f[7]);
+      for (int c = 0; c < 8; ++c) {
+        *reinterpret_cast<uint4*>(line0 + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(line1 + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      continue;
     }
-    uint8_t* row = dst + (q >> 2) * HALF + t * 128;
-    const int c0 = 2 * (q & 3);
-    *reinterpret_cast<uint4*>(row + ((c0 ^ (t & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
-    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (t & 7)) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
+    uint4 w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) w[q] = *reinterpret_cast<const uint4*>(line1 + ((q ^ sw) << 4));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t f[8];
+      e4m3x4_to_f16x2x2(w[q].x, f[0], f[1]);
+      e4m3x4_to_f16x2x2(w[q].y, f[2], f[3]);
+      e4m3x4_to_f16x2x2(w[q].z, f[4], f[5]);
+      e4m3x4_to_f16x2x2(w[q].w, f[6], f[7]);
+      uint8_t* line = q < 4 ? line0 : line1;
+      const int c0 = 2 * (q & 3);
+      *reinterpret_cast<uint4*>(line + ((c0 ^ sw) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<uint4*>(line + (((c0 + 1) ^ sw) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
+    }
   }
   fence_proxy_async_smem();
 }
@@ -242,11 +254,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
   const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1), mma_done = bar0 + 8 * (B2 + 6);
   auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
   auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
-  // fp8 caches: Q rounded to fp16, raw K / V tiles landed
+  // fp8 caches: Q rounded to fp16, K / V stages widened (k_full / v_full: their raw codes landed)
   constexpr int B3 = B2 + 7;
   const uint32_t q_ready = bar0 + 8 * B3;
-  auto rk_full = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
-  auto rv_full = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NR + s); };
+  auto k_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
+  auto v_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NSK + s); };
   const uint64_t policy = l2_policy_evict_first();
   const int* table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb;
   if (warp == T::W_K) {
@@ -272,10 +284,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       mbar_init(mma_done, 1);
       if constexpr (F8) {
         mbar_init(q_ready, 8);
-        for (int s = 0; s < T::NR; ++s) {
-          mbar_init(rk_full(s), 1);
-          mbar_init(rv_full(s), 1);
-        }
+        for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
+        for (int s = 0; s < T::NSV; ++s) mbar_init(v_ready(s), 1);
       }
       fence_barrier_init();
       mbar_arrive_expect_tx(q_full, T::TILE);
@@ -289,16 +299,15 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       if (id < 0 || id >= p.num_blocks) id = -1;  // (reported by the scan below)
     }
     const unsigned valid = __ballot_sync(kFullMask, id >= 0);
-    // bf16: the tile straight into K buffer 0; fp8: the raw codes into raw slot 0
-    const uint32_t kbar = F8 ? rk_full(0) : k_full(0);
+    // bf16: the tile into K stage 0; fp8: the raw codes into the stage's upper half
     if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(__popc(valid)) * (F8 ? 1u : 2u) * BS * 128u;
-      if (bytes) mbar_arrive_expect_tx(kbar, bytes); else mbar_arrive(kbar);
+      if (bytes) mbar_arrive_expect_tx(k_full(0), bytes); else mbar_arrive(k_full(0));
     }
     __syncwarp();
     if (id >= 0) {
       if constexpr (F8) {
-        tma_load_4d(base + T::RAWK_OFF + lane * BS * 128, &kmap, kbar, 0, hk, 0, id, policy);
+        tma_load_4d(base + T::K_OFF + T::HALF + lane * BS * 128, &kmap, k_full(0), 0, hk, 0, id, policy);
       } else {
         const uint32_t dst = base + T::K_OFF + lane * BS * 128;
         tma_load_4d(dst, &kmap, k_full(0), 0, hk, 0, id, policy);
@@ -332,58 +341,62 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
   auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };    // tokens 64h .. 64h+63 packed in pairs: hi / fp16
   auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };  // bf16 caches: the residual
 
-  if (F8 && (warp == T::W_K || warp == T::W_V)) {  // ---------- fp8: load raw tiles, widen to fp16 ----------
+  if (F8 && (warp == T::W_K || warp == T::W_V)) {  // ---------- fp8: TMA raw codes, widen in place ----------
     const bool is_k = warp == T::W_K;
     const CUtensorMap* map = is_k ? &kmap : &vmap;
-    const uint32_t raw_area = base + (is_k ? T::RAWK_OFF : T::RAWV_OFF);
-    const int nd = is_k ? T::NSK : T::NSV;
-    auto raw_full = [&](int s) { return is_k ? rk_full(s) : rv_full(s); };
-    auto issue_raw = [&](int j) {  // lane 0: tile j's raw codes into slot j % NR
-      const int r = j % T::NR;
+    const int ns = is_k ? T::NSK : T::NSV;
+    const int area = is_k ? T::K_OFF : T::V_OFF;
+    auto full = [&](int st) { return is_k ? k_full(st) : v_full(st); };
+    auto issue = [&](int j) {  // lane 0: tile j's raw codes into the upper half of stage j % ns
+      const int st = j % ns;
       const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
       int nvalid = 0;
       for (int i = i0; i < i1; ++i) nvalid += ids[i] >= 0;
       const uint32_t bytes = static_cast<uint32_t>(nvalid) * BS * 128u;
-      if (bytes) mbar_arrive_expect_tx(raw_full(r), bytes); else mbar_arrive(raw_full(r));
+      if (bytes) mbar_arrive_expect_tx(full(st), bytes); else mbar_arrive(full(st));
       for (int i = i0; i < i1; ++i)
-        if (ids[i] >= 0) tma_load_4d(raw_area + r * T::RAW + (i - i0) * BS * 128, map, raw_full(r), 0, hk, 0, ids[i], policy);
+        if (ids[i] >= 0)
+          tma_load_4d(base + area + st * T::TILE + T::HALF + (i - i0) * BS * 128, map, full(st), 0, hk, 0, ids[i],
+                      policy);
     };
-    int issued = is_k ? 1 : 0;  // K tile 0 was issued in the prologue
+    int issued = min(nt, ns);
     if (lane == 0)
-      for (int j = issued; j < min(nt, T::NR); ++j) issue_raw(j);
-    issued = min(nt, T::NR);
+      for (int j = is_k ? 1 : 0; j < issued; ++j) issue(j);  // (K tile 0 went out in the prologue)
     int landed = 0;
     for (int j = 0; j < nt; ++j) {
-      const int r = j % T::NR, d = j % nd;
-      if (!__all_sync(kFullMask, mbar_wait_bounded(raw_full(r), (j / T::NR) & 1, p.status))) break;
+      const int st = j % ns;
+      if (!__all_sync(kFullMask, mbar_wait_bounded(full(st), (j / ns) & 1, p.status))) break;
       landed = j + 1;
-      if (j >= nd && !__all_sync(kFullMask, mbar_wait_bounded(is_k ? k_empty(d) : v_empty(d), ((j / nd) - 1) & 1,
-                                                              p.status)))
-        break;
-      const uint8_t* src = data + (is_k ? T::RAWK_OFF : T::RAWV_OFF) + r * T::RAW;
-      uint8_t* dst = data + (is_k ? T::K_OFF : T::V_OFF) + d * T::TILE;
+      uint8_t* stage = data + area + st * T::TILE;
       const int tile0 = tok_begin + j * T::TOK;
       if (is_k) {  // scores of rows that are not loaded are masked, whatever these rows hold
-        widen_e4m3_tile(src, dst, lane, [](int) { return false; });
+        widen_e4m3_tile_in_place(stage, lane, [](int) { return false; });
       } else {     // V rows that must not contribute (past tok_end, bad blocks) are zeroed
-        widen_e4m3_tile(src, dst, lane, [&](int t) {
+        widen_e4m3_tile_in_place(stage, lane, [&](int t) {
           return tile0 + t >= tok_end || (any_bad && ids[(tile0 + t - tok_begin) / BS] < 0);
         });
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(is_k ? k_full(d) : v_full(d));
-        if (j + T::NR < nt) {
-          fence_proxy_async_smem();  // the raw slot's reads before the next TMA write into it
-          issue_raw(j + T::NR);
+      if (lane == 0) mbar_arrive(is_k ? k_ready(st) : v_ready(st));
+      // refill the stage of tile j - 1 with tile j - 1 + ns once its MMA has read it (by now it
+      // usually has: S(j-1) / P.V(j-1) were issued before tile j landed)
+      const int jr = j - 1 + ns;
+      if (j >= 1 && jr < nt) {
+        const int sp = (j - 1) % ns;
+        if (!__all_sync(kFullMask, mbar_wait_bounded(is_k ? k_empty(sp) : v_empty(sp), ((j - 1) / ns) & 1,
+                                                     p.status)))
+          break;
+        if (lane == 0) {
+          fence_proxy_async_smem();  // this warp's reads and writes of the stage before the TMA write
+          issue(jr);
         }
+        issued = jr + 1;
       }
-      if (j + T::NR < nt) issued = j + T::NR + 1;
     }
     // drain (bounded): the raw loads started have landed before exit
     if (lane == 0) {
       if (is_k) mbar_wait_bounded(q_full, 0, p.status);
-      for (int j = landed; j < issued; ++j) mbar_wait_bounded(raw_full(j % T::NR), (j / T::NR) & 1, p.status);
+      for (int j = landed; j < issued; ++j) mbar_wait_bounded(full(j % ns), (j / ns) & 1, p.status);
     }
   } else if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
     if (lane == 0) {
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
           const int sk = j % T::NSK;
-          if (!(ok = mbar_wait_bounded(k_full(sk), (j / T::NSK) & 1, p.status))) break;
+          if (!(ok = mbar_wait_bounded(F8 ? k_ready(sk) : k_full(sk), (j / T::NSK) & 1, p.status))) break;
           if (j > 0 && !(ok = mbar_wait_bounded(s_free, (j - 1) & 1, p.status))) break;
           tc_fence_after();
           // descriptors differ only in the start-address field (address >> 4 in the low bits, all
@@ -444,7 +457,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
           const int jj = j - 1, sv = jj % T::NSV;
           const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
           // the V tile (bf16: landed; fp8: widened)
-          if (!(ok = mbar_wait_bounded(v_full(sv), (jj / T::NSV) & 1, p.status))) break;
+          if (!(ok = mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (jj / T::NSV) & 1, p.status))) break;
           for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
             if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
             tc_fence_after();
@@ -493,6 +506,49 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
+    // bf16 caches: V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed:
+    // 0 * NaN would poison O.  The 64 rows of this half: thread (quarter, lane) takes row
+    // 16 quarter + lane / 2, dims half lane & 1.  (fp8 caches: the V producer zeroed them.)
+    auto zero_v_rows = [&](int j, bool bad) {
+      wait(v_full(j % T::NSV), (j / T::NSV) & 1);
+      const int vr = 64 * h + 16 * quarter + (lane >> 1);
+      const int t = tok_begin + j * T::TOK + vr;
+      if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
+        uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
+    };
+    auto half_tile_bad = [&](int t0) {  // a block of this half tile with a bad id
+      bool bad = false;
+      if (any_bad) {
+        const int i0 = (t0 - tok_begin) / BS, i1 = min(nb, (t0 + 64 - tok_begin) / BS);
+        for (int i = i0; i < i1; ++i) bad |= ids[i] < 0;
+      }
+      return bad;
+    };
+    // A warp whose 32 rows all lie past the CTA's query rows (grouped verification uses 40 of 128)
+    // computes nothing: it keeps every barrier step -- including the wait for the previous tile's
+    // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
+    // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
+    // output rows nobody writes.
+    if (qt * T::ROWS + 32 * quarter >= rows_total) {
+      for (int j = 0; j < nt; ++j) {
+        const int t0 = tok_begin + j * T::TOK + 64 * h;
+        wait(s_full, j & 1);
+        tc_fence_after();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        const bool bad = half_tile_bad(t0);
+        if (j > 0) wait(pv_done(h), (j - 1) & 1);
+        if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(h));
+      }
+    } else
     for (int j = 0; j < nt; ++j) {
       const int t0 = tok_begin + j * T::TOK + 64 * h;  // first token of this half of the tile
       wait(s_full, j & 1);
@@ -515,11 +571,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       if (lane == 0) mbar_arrive(s_free);
 
       // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
-      bool bad = false;
-      if (any_bad) {
-        const int i0 = (t0 - tok_begin) / BS, i1 = min(nb, (t0 + 64 - tok_begin) / BS);
-        for (int i = i0; i < i1; ++i) bad |= ids[i] < 0;
-      }
+      const bool bad = half_tile_bad(t0);
       const bool ragged = t0 + 64 > tok_end;  // tokens at or past tok_end in this half tile
       // row max of the raw scores (q_scale > 0 commutes with the max); masked scores -> -inf.
       // Eight independent partial maxima / sums: instruction-level parallelism hides latency.
@@ -602,20 +654,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
           }
         }
       }
-      // bf16 caches: V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed:
-      // 0 * NaN would poison O.  The 64 rows of this half: thread (quarter, lane) takes row
-      // 16 quarter + lane / 2, dims half lane & 1.  (fp8 caches: the V producer zeroed them.)
-      if (!F8 && (ragged || bad)) {
-        wait(v_full(j % T::NSV), (j / T::NSV) & 1);
-        const int vr = 64 * h + 16 * quarter + (lane >> 1);
-        const int t = tok_begin + j * T::TOK + vr;
-        if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
-          uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
-      }
+      if (!F8 && (ragged || bad)) zero_v_rows(j, bad);
       // this half of row r of P into TMEM lane r
 #pragma unroll
       for (int c = 0; c < 2; ++c) {

@@ -94,10 +94,13 @@ def test_partition_choice_and_workspace_size():
     rows = 64 * 32 * P
     assert pk.decode_workspace_bytes(64, 32, 32, 128, 16, 128, bf16) == \
         ((rows * 8 + 255) // 256) * 256 + rows * 128 * 4
-    # 256 x 40 heads up to 4096 tokens: 1024
-    assert pk.decode_partition_tokens(256, 40, 40, 128, 16, 256, bf16) == 1024
-    # fp8 GQA 64/8: 16 x 32k -> enough CTAs for one per resident slot (148 SMs assumed without a GPU)
-    assert pk.decode_partition_tokens(16, 64, 8, 128, 16, 2048, fp8) == 1024
+    # 256 x 40 heads up to 4096 tokens: more pairs than four waves of CTAs -> up to 2048 tokens
+    assert pk.decode_partition_tokens(256, 40, 40, 128, 16, 256, bf16) == 2048
+    # parallel sampling, 128 x 40 heads up to 1088 tokens: a single partition, no workspace
+    assert pk.decode_partition_tokens(128, 40, 40, 128, 16, 68, bf16) == 2048
+    assert pk.decode_workspace_bytes(128, 40, 40, 128, 16, 68, bf16) == 0
+    # fp8 GQA 64/8: 16 x 32k -> 2048 CTAs, at least three quarters of a wave (148 SMs assumed without a GPU)
+    assert pk.decode_partition_tokens(16, 64, 8, 128, 16, 2048, fp8) == 2048
     assert pk.decode_partition_tokens(128, 64, 8, 128, 16, 512, fp8) == 2048
     # explicit partition lengths
     assert pk.decode_partition_tokens(1, 1, 1, 128, 16, 100, bf16, 48) == 48
