@@ -291,13 +291,25 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
                                     s.cache_dtype, args.partition_tokens)
     ws_bytes = pk.decode_workspace_bytes(s.num_seqs, s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, MB,
                                          s.cache_dtype, pt)
+    fused = w.new_k is not None and not args.unfused
+    # groups sharing their prompt's blocks (parallel sampling): each shared block read once per group
+    grouped = w.group_start is not None and fused and not args.no_shared_prefix
+    if grouped:
+        n_groups = int(w.group_start.shape[0]) - 1
+        max_group = int((w.group_start[1:] - w.group_start[:-1]).max().item())
+        ws_bytes = pk.decode_shared_prefix_workspace_bytes(s.num_seqs, n_groups, s.num_q_heads, s.num_kv_heads,
+                                                           s.head_dim, s.block_size, MB, args.partition_tokens)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     out = torch.empty_like(w.q)
     stream = torch.cuda.current_stream(dev)
-    fused = w.new_k is not None and not args.unfused
 
     def decode(kc, vc, tables):
-        if fused:  # the new token (one per sequence, at ctx - 1) is written inside the decode launch
+        if grouped:
+            pk.paged_attention_decode_shared_prefix(w.q, kc, vc, tables, w.context_lens, w.group_start,
+                                                    w.shared_blocks, w.scale, k_new=w.new_k, v_new=w.new_v,
+                                                    max_group_size=max_group, out=out, workspace=workspace,
+                                                    partition_tokens=args.partition_tokens, stream=stream)
+        elif fused:  # the new token (one per sequence, at ctx - 1) is written inside the decode launch
             pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, tables, w.context_lens, w.scale,
                                    k_scale=w.k_scale, v_scale=w.v_scale, out=out, workspace=workspace,
                                    partition_tokens=pt, stream=stream)
@@ -410,10 +422,13 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
                    "kv_bytes_per_step_per_gpu": kv_bytes, "partition_tokens": pt,
                    "new_tokens_per_step": 0 if w.new_k is None else int(w.new_k.shape[0]),
                    "new_token_write": "fused into the decode launch" if fused else "separate launch",
+                   "decode": ("shared prefix: each group's shared blocks read once for all its members, own "
+                              "blocks per sequence, partials merged" if grouped else "per sequence"),
                    "cow_pairs_per_step": 0 if w.copy_pairs is None else int(len(w.copy_pairs)),
                    "l2": "inputs larger than L2 (KV stream per step > 126 MB); no flush",
                    "parallelism": f"dp{world} (independent batch per GPU, no collective)"},
-        "roofline": {"kernel": kernel_name(s) + " + paged_decode_reduce_kernel",
+        "roofline": {"kernel": ("paged_decode_mma_bf16_kernel (shared-prefix units)" if grouped else kernel_name(s))
+                               + " + paged_decode_reduce_kernel",
                      "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "peak_kind": f"{peak_kind} (burst copy bandwidth)", "frac": round(achieved / peak, 4),
                      "algorithmic_bytes_per_launch": alg, "decode_ms": round(decode_ms, 5),
@@ -423,7 +438,8 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async (pinned host "
                        "inputs and output every step; two steps in flight: copies in, kernels, copies out on "
-                       "three streams)"},
+                       "three streams)" + ("; the host step decodes per sequence (it takes no groups)"
+                                           if grouped else "")},
         "gpu_launches": int(launches),
         "clocks": clk,
     }
@@ -843,6 +859,8 @@ def parse_args(argv=None):
                     help="seconds of oracle work for the headline's cpu_baseline (half for the other configs)")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shared-prefix", action="store_true",
+                    help="decode parallel-sampling workloads per sequence instead of reading shared prefixes once")
     ap.add_argument("--unfused", action="store_true",
                     help="write the new tokens with a separate paged_kv_write launch instead of inside the decode")
     ap.add_argument("--num-seqs", type=int, default=0,

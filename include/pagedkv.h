@@ -73,6 +73,8 @@ extern "C" {
 #define PKV_STATUS_WAIT_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up */
 #define PKV_STATUS_BAD_QUERY_LOC 0x20u  /* multi-query met query_start_loc entries outside [0, total_q] or a
                                            q_len above max_q_len: that sequence's rows are left unwritten */
+#define PKV_STATUS_BAD_GROUP 0x40u      /* shared-prefix decode met a group outside [0, num_seqs), empty, or
+                                           wider than 8 columns: its shared unit was skipped */
 
 /*
  * Human-readable name of a PKV_* status code (static storage).
@@ -183,6 +185,57 @@ int pkv_paged_decode_append(void* out, const void* q, const void* k_new, const v
                             int max_blocks_per_seq, int64_t num_blocks, float scale, float k_scale, float v_scale,
                             int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
                             size_t workspace_bytes, int validate, void* stream);
+
+/*
+ * Paged decode attention with shared prefixes read once.
+ *
+ * Source: "vLLM — 把操作系统的分页搬进 GPU KV cache", 核心要点 and 实践案例 2 --
+ * the n candidates of parallel sampling share their prompt's physical blocks
+ * (ref_count n), one copy of the prompt's KV for all of them; the attention is
+ * pkv_paged_attention_decode's.  This call computes exactly that attention
+ * (every output row equals pkv_paged_attention_decode's for the same
+ * arguments, up to rounding order), but reads each shared block once for all
+ * the sequences that share it: the queries of a group's members are the
+ * columns of one tensor-core tile over the group's shared blocks, each member
+ * then attends its own blocks, and the two partial softmaxes are merged by the
+ * softmax identity.  With k_new / v_new (both or neither) each sequence's new
+ * token is written first, as by pkv_paged_decode_append.
+ *
+ * group_start     device int32 [num_groups + 1]: the sequences of group g are
+ *                 group_start[g] .. group_start[g+1] - 1 (consecutive; every
+ *                 sequence in exactly one group; a group of one is allowed).
+ * shared_blocks   device int32 [num_groups]: the first shared_blocks[g] logical
+ *                 blocks of every member of group g are the same physical
+ *                 blocks (the group's first member's table is read for them),
+ *                 and lie within every member's context -- before its new
+ *                 token when k_new is given.  validate checks all of this; a
+ *                 wrong grouping without validate gives wrong results.
+ * max_group_size  the largest group; max_group_size x (num_q_heads /
+ *                 num_kv_heads) <= 8 (the tile's columns), else PKV_ERR_BAD_SHAPE.
+ * workspace       device scratch of pkv_decode_shared_prefix_workspace_bytes()
+ *                 bytes, 256-byte aligned (the shared and own partials of every
+ *                 (sequence, head)).
+ * Supported: bf16 q and caches, head_dim 128, block_size 16 or 32, 1/2/4/8
+ * query heads per KV head.  Other arguments and errors: as
+ * pkv_paged_decode_append.  num_seqs == 0 launches nothing.
+ */
+int pkv_paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                                             void* key_cache, void* value_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, const int32_t* group_start,
+                                             const int32_t* shared_blocks, int num_seqs, int num_groups,
+                                             int max_group_size, int num_q_heads, int num_kv_heads, int head_dim,
+                                             int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                                             int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                                             size_t workspace_bytes, int validate, void* stream);
+
+/* Workspace bytes of pkv_paged_attention_decode_shared_prefix (0 for
+ * unsupported arguments).  Its partition length is partition_tokens, or the
+ * automatic choice of pkv_decode_partition_tokens made for the groups' shared
+ * units (num_groups x num_kv_heads) on the bf16 tensor-core kernel.  A sizing
+ * helper of this library. */
+size_t pkv_decode_shared_prefix_workspace_bytes(int num_seqs, int num_groups, int num_q_heads, int num_kv_heads,
+                                                int head_dim, int block_size, int max_blocks_per_seq,
+                                                int partition_tokens);
 
 /*
  * Paged decode attention that allocates nothing and takes no workspace.

@@ -30,8 +30,10 @@ STATUS_BAD_SLOT = 0x4
 STATUS_BAD_COPY_PAIR = 0x8
 STATUS_WAIT_TIMEOUT = 0x10
 STATUS_BAD_QUERY_LOC = 0x20
+STATUS_BAD_GROUP = 0x40
 
-__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
+__all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_decode_shared_prefix",
+           "decode_shared_prefix_workspace_bytes", "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "decode_table_scan", "device_status", "launch_count", "PagedKVError",
@@ -209,6 +211,59 @@ def multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv
     return int(_lib.load().pkv_multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads,
                                                           head_dim, block_size, max_blocks_per_seq,
                                                           _cache_code(cache_dtype), partition_tokens))
+
+
+def decode_shared_prefix_workspace_bytes(num_seqs, num_groups, num_q_heads, num_kv_heads, head_dim, block_size,
+                                         max_blocks_per_seq, partition_tokens=0) -> int:
+    """Workspace bytes of paged_attention_decode_shared_prefix."""
+    return int(_lib.load().pkv_decode_shared_prefix_workspace_bytes(num_seqs, num_groups, num_q_heads, num_kv_heads,
+                                                                    head_dim, block_size, max_blocks_per_seq,
+                                                                    partition_tokens))
+
+
+def paged_attention_decode_shared_prefix(q, key_cache, value_cache, block_tables, context_lens, group_start,
+                                         shared_blocks, scale: float, *, k_new=None, v_new=None,
+                                         max_group_size: int | None = None, out=None, workspace=None,
+                                         partition_tokens: int = 0, validate: bool = False, stream=None):
+    """Decode attention where groups of consecutive sequences share their first
+    shared_blocks[g] physical blocks (parallel sampling): each shared block is
+    read once for the whole group.  group_start int32 [G + 1], shared_blocks
+    int32 [G].  Same result as paged_attention_decode (or paged_decode_append
+    when k_new / v_new are given).  Returns out [B, Hq, d]."""
+    dev = _cuda(q, key_cache, value_cache, block_tables, context_lens, group_start, shared_blocks)
+    for t in (block_tables, context_lens, group_start, shared_blocks):
+        if t.dtype != torch.int32:
+            raise TypeError("block_tables, context_lens, group_start and shared_blocks must be int32")
+    B, Hq, d = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    Gn = shared_blocks.shape[0]
+    if group_start.shape != (Gn + 1,) or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("shape mismatch")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    if k_new is not None:
+        _cuda(k_new, v_new)
+        if k_new.shape != (B, Hkv, d) or v_new.shape != k_new.shape or k_new.dtype != q.dtype:
+            raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] in q's dtype")
+    MB = block_tables.shape[1]
+    if max_group_size is None:
+        max_group_size = int((group_start[1:] - group_start[:-1]).max().item()) if Gn else 1
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_shared_prefix_workspace_bytes(B, max(Gn, 1), Hq, Hkv, d, bs, MB, partition_tokens) if B else 0
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    with torch.cuda.device(dev):
+        _check(_lib.load().pkv_paged_attention_decode_shared_prefix(
+            out.data_ptr(), q.data_ptr(), ptr(k_new), ptr(v_new), key_cache.data_ptr(), value_cache.data_ptr(),
+            block_tables.data_ptr(), context_lens.data_ptr(), group_start.data_ptr(), shared_blocks.data_ptr(), B, Gn,
+            int(max_group_size), Hq, Hkv, d, bs, MB, NB, float(scale), _dtype(q), _dtype(key_cache),
+            int(partition_tokens), ws_ptr, ws_bytes, int(validate), _stream(dev, stream)),
+            "paged_attention_decode_shared_prefix")
+    return out
 
 
 def paged_attention_multiquery(q, key_cache, value_cache, block_tables, context_lens, query_start_loc,

@@ -599,6 +599,141 @@ int pkv_paged_attention_multiquery(void* out, const void* q, const void* key_cac
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Partition length and slot counts of the shared-prefix decode: the automatic
+// choice is made for the groups' shared units (one per group and KV head, the
+// bulk of the bytes) on the bf16 tensor-core kernel.
+static int shared_prefix_partition_tokens(int num_groups, int num_kv_heads, int block_size, int max_blocks_per_seq,
+                                          int partition_tokens) {
+  if (partition_tokens != 0) {
+    if (partition_tokens < 0 || partition_tokens % block_size != 0 || partition_tokens > kMaxPartitionTokens)
+      return PKV_ERR_PARTITION;
+    return partition_tokens;
+  }
+  return auto_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq,
+                               decode_ctas_per_sm(PKV_DTYPE_BF16, 128, 2, block_size));
+}
+
+size_t pkv_decode_shared_prefix_workspace_bytes(int num_seqs, int num_groups, int num_q_heads, int num_kv_heads,
+                                                int head_dim, int block_size, int max_blocks_per_seq,
+                                                int partition_tokens) {
+  if (num_seqs <= 0 || num_groups <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_blocks_per_seq <= 0 || (block_size != 16 && block_size != 32))
+    return 0;
+  const int pt = shared_prefix_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq,
+                                                partition_tokens);
+  if (pt < 0) return 0;
+  const int64_t P = 2 * cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt);
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * P;
+  return align256(rows * 2 * sizeof(float)) + rows * head_dim * sizeof(float);
+}
+
+int pkv_paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                                             void* key_cache, void* value_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, const int32_t* group_start,
+                                             const int32_t* shared_blocks, int num_seqs, int num_groups,
+                                             int max_group_size, int num_q_heads, int num_kv_heads, int head_dim,
+                                             int block_size, int max_blocks_per_seq, int64_t num_blocks, float scale,
+                                             int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                                             size_t workspace_bytes, int validate, void* stream) {
+  if (num_seqs < 0 || num_groups < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_seqs == 0) return PKV_OK;
+  if (num_groups < 1 || num_groups > num_seqs || max_group_size < 1) return PKV_ERR_BAD_SHAPE;
+  if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens || !group_start || !shared_blocks)
+    return PKV_ERR_NULL_POINTER;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PKV_ERR_NULL_POINTER;
+  if (q_dtype != PKV_DTYPE_BF16 || cache_dtype != PKV_DTYPE_BF16) return PKV_ERR_BAD_DTYPE;
+  if (head_dim != 128) return PKV_ERR_HEAD_DIM;
+  if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_HEAD_GROUPING;
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_HEAD_GROUPING;
+  if (static_cast<int64_t>(max_group_size) * group > 8) return PKV_ERR_BAD_SHAPE;  // members x heads: 8 columns
+  if (num_blocks > 0x7fffffffLL || num_seqs + num_groups > 65535) return PKV_ERR_BAD_SHAPE;
+  if (static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffffLL) return PKV_ERR_BAD_SHAPE;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_MISALIGNED;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PKV_ERR_MISALIGNED;
+  const int pt = shared_prefix_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq,
+                                                partition_tokens);
+  if (pt < 0) return pt;
+  const int Ph = static_cast<int>(cdiv64(static_cast<int64_t>(max_blocks_per_seq) * block_size, pt));
+  if (Ph > 32767) return PKV_ERR_PARTITION;
+  const size_t need = pkv_decode_shared_prefix_workspace_bytes(num_seqs, num_groups, num_q_heads, num_kv_heads,
+                                                               head_dim, block_size, max_blocks_per_seq,
+                                                               partition_tokens);
+  if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (validate) {
+    std::vector<int32_t> lens, tables, gs, sh;
+    if (!copy_to_host(lens, context_lens, static_cast<size_t>(num_seqs), st) ||
+        !copy_to_host(tables, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st) ||
+        !copy_to_host(gs, group_start, static_cast<size_t>(num_groups) + 1, st) ||
+        !copy_to_host(sh, shared_blocks, static_cast<size_t>(num_groups), st))
+      return PKV_ERR_CUDA;
+    if (gs[0] != 0 || gs[num_groups] != num_seqs) return PKV_ERR_OUT_OF_RANGE;
+    for (int g = 0; g < num_groups; ++g) {
+      const int n = gs[g + 1] - gs[g];
+      if (n < 1 || n > max_group_size || sh[g] < 0) return PKV_ERR_OUT_OF_RANGE;
+      for (int b = gs[g]; b < gs[g + 1]; ++b) {
+        // the shared blocks are whole blocks of every member's context (and the appended token is its own)
+        if (static_cast<int64_t>(sh[g]) * block_size > static_cast<int64_t>(lens[b]) - (k_new ? 1 : 0))
+          return PKV_ERR_OUT_OF_RANGE;
+        for (int j = 0; j < sh[g]; ++j)
+          if (tables[static_cast<size_t>(b) * max_blocks_per_seq + j] !=
+              tables[static_cast<size_t>(gs[g]) * max_blocks_per_seq + j])
+            return PKV_ERR_OUT_OF_RANGE;
+      }
+    }
+    for (int b = 0; b < num_seqs; ++b) {
+      const int64_t ctx = lens[b];
+      if (ctx < 0 || ctx > static_cast<int64_t>(max_blocks_per_seq) * block_size) return PKV_ERR_OUT_OF_RANGE;
+      for (int64_t j = 0; j < cdiv64(ctx, block_size); ++j) {
+        const int64_t id = tables[static_cast<size_t>(b) * max_blocks_per_seq + j];
+        if (id < 0 || id >= num_blocks) return PKV_ERR_OUT_OF_RANGE;
+      }
+    }
+  }
+  unsigned* status = status_word();
+  if (!status) return PKV_ERR_CUDA;
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, true) ||
+      !encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype, true))
+    return PKV_ERR_TENSOR_MAP;
+  DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * (2 * Ph);
+  p.ws_ml = static_cast<float*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * 2 * sizeof(float)));
+  p.status = status;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = static_cast<int>(num_blocks);
+  p.block_size = block_size;
+  p.partition_blocks = pt / block_size;
+  p.max_partitions = 2 * Ph;
+  p.q_scale = scale * kLog2e;
+  p.out_scale = 1.f;
+  p.new_k = k_new;
+  p.new_v = v_new;
+  p.key_cache = key_cache;
+  p.value_cache = value_cache;
+  p.k_inv = 1.f;
+  p.v_inv = 1.f;
+  p.group_start = group_start;
+  p.shared_blocks = shared_blocks;
+  p.num_groups = num_groups;
+  p.shared_partitions = Ph;
+  return launch_decode_shared_prefix_bf16(kmap, vmap, p, group, num_kv_heads, Ph, st) == cudaSuccess ? PKV_OK
+                                                                                                     : PKV_ERR_CUDA;
+}
+
 int pkv_selftest_wait_timeout(int64_t limit_ns, unsigned* gave_up, void* stream) {
   if (limit_ns <= 0 || limit_ns > 100000000LL) return PKV_ERR_BAD_SHAPE;
   if (!gave_up) return PKV_ERR_NULL_POINTER;

@@ -63,7 +63,33 @@ struct DecodeParams {
   void* value_cache;
   float k_inv;  // fp8 caches: 1/k_scale and 1/v_scale rounded to fp32
   float v_inv;
+  // Shared-prefix decode (pkv_paged_attention_decode_shared_prefix): groups of
+  // consecutive sequences whose first shared_blocks[g] logical blocks are the
+  // same physical blocks.  Partial slots [0, shared_partitions) of a
+  // (sequence, head) hold its group's shared-prefix partials, the slots from
+  // shared_partitions on its own blocks'.  group_start is NULL otherwise.
+  const int32_t* group_start = nullptr;    // [num_groups + 1]
+  const int32_t* shared_blocks = nullptr;  // [num_groups]
+  int num_groups = 0;
+  int shared_partitions = 0;
 };
+
+// The group holding sequence b (group_start is non-decreasing; the last g with
+// group_start[g] <= b).
+__device__ __forceinline__ int group_of_sequence(const DecodeParams& p, int b) {
+  int lo = 0, hi = p.num_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (p.group_start[mid] <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Shared blocks of group g, clamped to what the table and the context allow.
+__device__ __forceinline__ int shared_blocks_of(const DecodeParams& p, int g, int nblk) {
+  const int s = p.shared_blocks[g];
+  return s < 0 ? 0 : (s > nblk ? nblk : s);
+}
 
 // Fused append: the CTA that reads the last block of sequence b writes that
 // sequence's new token for its kv head (row (ctx-1) % BS of physical block
@@ -414,19 +440,33 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   const int max_ctx = p.max_blocks_per_seq * BS;
   int ctx = p.context_lens[b];
   ctx = ctx < 0 ? 0 : (ctx > max_ctx ? max_ctx : ctx);
-  const int nparts = ((ctx + BS - 1) / BS + p.partition_blocks - 1) / p.partition_blocks;
-  if (nparts <= 1) return;  // written by the partition pass
+  const int nblk = (ctx + BS - 1) / BS;
+  // slots [0, n0) and [s1, s1 + n1): one range for plain decode, the group's
+  // shared-prefix partials and the sequence's own for shared-prefix decode
+  int n0, s1 = 0, n1 = 0;
+  if (p.group_start) {  // every partial is merged here, even a single one
+    const int sh = shared_blocks_of(p, group_of_sequence(p, b), nblk);
+    n0 = (sh + p.partition_blocks - 1) / p.partition_blocks;
+    s1 = p.shared_partitions;
+    n1 = (nblk - sh + p.partition_blocks - 1) / p.partition_blocks;
+  } else {
+    n0 = (nblk + p.partition_blocks - 1) / p.partition_blocks;
+    if (n0 <= 1) return;  // written by the partition pass
+  }
+  const int nparts = n0 + n1;
+  auto slot = [&](int i) { return i < n0 ? i : s1 + (i - n0); };
   const float* ml = p.ws_ml + row * p.max_partitions * 2;
   const float* o = p.ws_o + row * p.max_partitions * D;
   float M = -INFINITY;
-  for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[2 * i]);
+  for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[2 * slot(i)]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
   float acc[PVV];
 #pragma unroll
   for (int e = 0; e < PVV; ++e) acc[e] = 0.f;
   float W = 0.f;
-  for (int i = 0; i < nparts; ++i) {
+  for (int k = 0; k < nparts; ++k) {
+    const int i = slot(k);
     const float li = ml[2 * i + 1];
     const float w = li > 0.f ? li * fast_exp2((ml[2 * i] - M) * kLog2e) : 0.f;
     W += w;

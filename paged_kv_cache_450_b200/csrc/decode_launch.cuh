@@ -51,6 +51,21 @@ static cudaError_t launch_mma_bf16(const CUtensorMap& kmap, const CUtensorMap& v
   return launch_pdl(kern, grid, dim3(32), smem, st, kmap, vmap, p);
 }
 
+// Shared-prefix decode: grid z = the groups' shared units, then one unit per
+// sequence for its own blocks; the merge always runs.
+template <int BS, int G>
+static cudaError_t launch_mma_bf16_grouped(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                                           int num_kv_heads, int grid_partitions, cudaStream_t st) {
+  using T = MmaBf16Traits<BS>;
+  auto kern = paged_decode_mma_bf16_kernel<BS, G, true>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  dim3 grid(num_kv_heads, grid_partitions, p.num_groups + p.num_seqs);
+  return launch_pdl(kern, grid, dim3(32), smem, st, kmap, vmap, p);
+}
+
 template <typename TQ, int D>
 static cudaError_t launch_reduce(const DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_q_heads;
@@ -106,6 +121,18 @@ static cudaError_t dispatch_decode(const CUtensorMap& kmap, const CUtensorMap& v
   }
   if (e != cudaSuccess || !reduce) return e;
   return head_dim == 64 ? launch_reduce<TQ, 64>(p, st) : launch_reduce<TQ, 128>(p, st);
+}
+
+template <int BS>
+static cudaError_t dispatch_grouped_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                                          int group, int num_kv_heads, int grid_partitions, cudaStream_t st) {
+  switch (group) {
+    case 1: return launch_mma_bf16_grouped<BS, 1>(kmap, vmap, p, num_kv_heads, grid_partitions, st);
+    case 2: return launch_mma_bf16_grouped<BS, 2>(kmap, vmap, p, num_kv_heads, grid_partitions, st);
+    case 4: return launch_mma_bf16_grouped<BS, 4>(kmap, vmap, p, num_kv_heads, grid_partitions, st);
+    case 8: return launch_mma_bf16_grouped<BS, 8>(kmap, vmap, p, num_kv_heads, grid_partitions, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace pkv

@@ -20,6 +20,17 @@
 // needed multiply-adds, which costs nothing here (the kernel is bound by
 // HBM and the pipe is otherwise idle) and removes the shuffles and the
 // per-element widening of the CUDA-core kernel.
+//
+// Shared-prefix mode (GROUPED, pkv_paged_attention_decode_shared_prefix):
+// sequences come in groups of consecutive members whose first
+// shared_blocks[g] logical blocks are the same physical blocks (the n
+// candidates of parallel sampling share their prompt's blocks, ref_count n:
+// "vLLM — 把操作系统的分页搬进 GPU KV cache", 实践案例 2).  Grid z < num_groups
+// is a shared unit: the queries of all members (members x G <= 8 columns) over
+// the group's shared blocks, read once; grid z >= num_groups is sequence
+// z - num_groups over its own blocks past the shared prefix (the fused append
+// included).  Every unit writes partials; the merge combines a sequence's
+// shared and own partials by the softmax identity.
 #pragma once
 
 #include "decode.cuh"
@@ -77,7 +88,7 @@ __device__ __forceinline__ void bf16x2_split(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-template <int BS, int G, int NS = 0, int MINB = MmaBf16Traits<BS, NS>::MIN_BLOCKS>
+template <int BS, int G, bool GROUPED = false, int NS = 0, int MINB = MmaBf16Traits<BS, NS>::MIN_BLOCKS>
 __global__ void __launch_bounds__(32, MINB)
     paged_decode_mma_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                                  const DecodeParams p) {
@@ -90,28 +101,80 @@ __global__ void __launch_bounds__(32, MINB)
   uint64_t* bars = reinterpret_cast<uint64_t*>(data + T::STAGE_AREA);
   int* ids = reinterpret_cast<int*>(data + T::STAGE_AREA + T::BAR_BYTES);
 
-  const int hk = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
+  const int hk = blockIdx.x, part = blockIdx.y;
   const int lane = threadIdx.x;
   const int r = lane >> 2, c = lane & 3;
   const int max_ctx = p.max_blocks_per_seq * BS;
-  int ctx = p.context_lens[b];
-  if (ctx < 0 || ctx > max_ctx) {
-    if (lane == 0 && hk == 0 && part == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
-    ctx = ctx < 0 ? 0 : max_ctx;
-  }
-  const int nblk = (ctx + BS - 1) / BS;
   const int pb = p.partition_blocks;
-  const int nparts = (nblk + pb - 1) / pb;
-  const int64_t out_row0 = static_cast<int64_t>(b) * p.num_q_heads + hk * G;
+  const int Hq = p.num_q_heads;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-  if (nparts == 0) {
-    if (part == 0)
-      for (int i = lane; i < G * D; i += 32) out[out_row0 * D + i] = __float2bfloat16_rn(0.f);
-    return;
+  // This CTA's unit: table row b, blocks [blk0, blk0 + nb) of it, `cols` real
+  // MMA columns (query rows), column j being q / out row row_of(j), partial
+  // slot slot0 + part; ctx_eff = the tokens of the table row that count.
+  int b, ctx, ctx_eff, nparts, blk0, nb, cols, slot0 = 0;
+  int64_t row_first, member_stride = 0;  // row_of(j) = row_first + (j / G) * member_stride + j % G
+  bool append;
+  if constexpr (GROUPED) {
+    const int z = blockIdx.z;
+    if (z < p.num_groups) {  // the group's shared prefix, all members at once
+      const int b0 = p.group_start[z], n = p.group_start[z + 1] - b0;
+      if (b0 < 0 || n < 1 || n * G > 8 || b0 + n > p.num_seqs) {  // before any load or store
+        if (lane == 0 && hk == 0 && part == 0) set_status(p.status, PKV_STATUS_BAD_GROUP);
+        return;
+      }
+      b = b0;
+      const int sh = shared_blocks_of(p, z, p.max_blocks_per_seq);
+      cols = n * G;
+      ctx = ctx_eff = sh * BS;
+      nparts = (sh + pb - 1) / pb;
+      if (part >= nparts) return;
+      blk0 = part * pb;
+      nb = min(pb, sh - blk0);
+      row_first = static_cast<int64_t>(b0) * Hq + hk * G;
+      member_stride = Hq;
+      append = false;
+    } else {  // the sequence's own blocks past its group's shared prefix
+      b = z - p.num_groups;
+      ctx = p.context_lens[b];
+      if (ctx < 0 || ctx > max_ctx) {
+        if (lane == 0 && hk == 0 && part == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
+        ctx = ctx < 0 ? 0 : max_ctx;
+      }
+      ctx_eff = ctx;
+      const int nblk = (ctx + BS - 1) / BS;
+      const int sh = shared_blocks_of(p, group_of_sequence(p, b), nblk);
+      nparts = (nblk - sh + pb - 1) / pb;
+      if (part >= nparts) return;
+      blk0 = sh + part * pb;
+      nb = min(pb, nblk - blk0);
+      cols = G;
+      row_first = static_cast<int64_t>(b) * Hq + hk * G;
+      slot0 = p.shared_partitions;
+      append = p.new_k != nullptr && part == nparts - 1;
+    }
+  } else {
+    b = blockIdx.z;
+    ctx = p.context_lens[b];
+    if (ctx < 0 || ctx > max_ctx) {
+      if (lane == 0 && hk == 0 && part == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
+      ctx = ctx < 0 ? 0 : max_ctx;
+    }
+    ctx_eff = ctx;
+    const int nblk = (ctx + BS - 1) / BS;
+    nparts = (nblk + pb - 1) / pb;
+    row_first = static_cast<int64_t>(b) * Hq + hk * G;
+    cols = G;
+    if (nparts == 0) {
+      if (part == 0)
+        for (int i = lane; i < G * D; i += 32) out[row_first * D + i] = __float2bfloat16_rn(0.f);
+      return;
+    }
+    if (part >= nparts) return;
+    blk0 = part * pb;
+    nb = min(pb, nblk - blk0);
+    append = p.new_k != nullptr && part == nparts - 1;
   }
-  if (part >= nparts) return;
-  const int blk0 = part * pb;
-  const int nb = min(pb, nblk - blk0);
+  auto row_of = [&](int j) -> int64_t { return row_first + (j / G) * member_stride + j % G; };
 
   for (int i = lane; i < nb; i += 32) {
     int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + blk0 + i];
@@ -121,7 +184,6 @@ __global__ void __launch_bounds__(32, MINB)
     }
     ids[i] = id;
   }
-  const bool append = p.new_k != nullptr && part == nparts - 1;
   if (append) append_new_token<__nv_bfloat16, __nv_bfloat16, D, BS>(p, b, hk, ctx, lane, 32);
   const uint32_t bar0 = smem_u32(bars);
   if (lane == 0) {
@@ -156,15 +218,15 @@ __global__ void __launch_bounds__(32, MINB)
   }
 
   // q (B operand of S) as stored: chunk j, lane (r, c): dims 16j + 2c (+1) and +8 (+9).
-  // Columns r >= G are padding (zero).
+  // Columns r >= cols are padding (zero).
   uint32_t qf[8][2];
   {
-    const uint32_t* qrow =
-        reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(p.q) + (out_row0 + r) * D);
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                             (r < cols ? row_of(r) : 0) * D);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      qf[j][0] = r < G ? qrow[8 * j + c] : 0u;
-      qf[j][1] = r < G ? qrow[8 * j + c + 4] : 0u;
+      qf[j][0] = r < cols ? qrow[8 * j + c] : 0u;
+      qf[j][1] = r < cols ? qrow[8 * j + c + 4] : 0u;
     }
   }
   const float qk = p.q_scale;
@@ -196,7 +258,7 @@ __global__ void __launch_bounds__(32, MINB)
   auto tile_valid = [&](int u) -> int {
     const int j = u / T::NT;
     if (ids[j] < 0) return 0;
-    const int v = ctx - (blk0 + j) * BS - 16 * (u % T::NT);
+    const int v = ctx_eff - (blk0 + j) * BS - 16 * (u % T::NT);
     return v < 0 ? 0 : (v > 16 ? 16 : v);
   };
   auto compute_s = [&](int u, float (&sacc)[4]) {
@@ -322,41 +384,41 @@ __global__ void __launch_bounds__(32, MINB)
   }
   const float f0 = l0 > 0.f ? p.out_scale / l0 : 0.f;
   const float f1 = l1 > 0.f ? p.out_scale / l1 : 0.f;
-  const int ha = 2 * c, hb = 2 * c + 1;  // query heads of this lane's columns (real if < G)
-  if (nparts == 1) {
+  const int ha = 2 * c, hb = 2 * c + 1;  // this lane's columns (real if < cols)
+  if (!GROUPED && nparts == 1) {
 #pragma unroll
     for (int mi = 0; mi < 8; ++mi) {
       const int d0 = 16 * mi + r, d1 = d0 + 8;
-      if (ha < G) {
-        out[(out_row0 + ha) * D + d0] = __float2bfloat16_rn(o[mi][0] * f0);
-        out[(out_row0 + ha) * D + d1] = __float2bfloat16_rn(o[mi][2] * f0);
+      if (ha < cols) {
+        out[row_of(ha) * D + d0] = __float2bfloat16_rn(o[mi][0] * f0);
+        out[row_of(ha) * D + d1] = __float2bfloat16_rn(o[mi][2] * f0);
       }
-      if (hb < G) {
-        out[(out_row0 + hb) * D + d0] = __float2bfloat16_rn(o[mi][1] * f1);
-        out[(out_row0 + hb) * D + d1] = __float2bfloat16_rn(o[mi][3] * f1);
+      if (hb < cols) {
+        out[row_of(hb) * D + d0] = __float2bfloat16_rn(o[mi][1] * f1);
+        out[row_of(hb) * D + d1] = __float2bfloat16_rn(o[mi][3] * f1);
       }
     }
   } else {
-    const int64_t slot_a = (out_row0 + ha) * p.max_partitions + part;
-    const int64_t slot_b = (out_row0 + hb) * p.max_partitions + part;
+    const int64_t slot_a = (ha < cols ? row_of(ha) : 0) * p.max_partitions + slot0 + part;
+    const int64_t slot_b = (hb < cols ? row_of(hb) : 0) * p.max_partitions + slot0 + part;
 #pragma unroll
     for (int mi = 0; mi < 8; ++mi) {
       const int d0 = 16 * mi + r, d1 = d0 + 8;
-      if (ha < G) {
+      if (ha < cols) {
         p.ws_o[slot_a * D + d0] = o[mi][0] * f0;
         p.ws_o[slot_a * D + d1] = o[mi][2] * f0;
       }
-      if (hb < G) {
+      if (hb < cols) {
         p.ws_o[slot_b * D + d0] = o[mi][1] * f1;
         p.ws_o[slot_b * D + d1] = o[mi][3] * f1;
       }
     }
     if (r == 0) {
-      if (ha < G) {
+      if (ha < cols) {
         p.ws_ml[slot_a * 2] = m0 * kLn2;
         p.ws_ml[slot_a * 2 + 1] = l0;
       }
-      if (hb < G) {
+      if (hb < cols) {
         p.ws_ml[slot_b * 2] = m1 * kLn2;
         p.ws_ml[slot_b * 2 + 1] = l1;
       }

@@ -124,5 +124,8 @@ PKV_DECLARE_DECODE(launch_decode_bf16_bf16)
 PKV_DECLARE_DECODE(launch_decode_f32_fp8)
 PKV_DECLARE_DECODE(launch_decode_bf16_fp8)
 #undef PKV_DECLARE_DECODE
+// Shared-prefix decode, bf16 q and cache, head_dim 128, bs 16/32 (the merge included).
+cudaError_t launch_decode_shared_prefix_bf16(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                                             int group, int num_kv_heads, int grid_partitions, cudaStream_t st);
 
 }  // namespace pkv

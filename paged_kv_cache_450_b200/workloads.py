@@ -105,6 +105,10 @@ class DecodeWorkload:
     slot_mapping: torch.Tensor | None  # int64 [T]
     copy_pairs: torch.Tensor | None    # int64 [n, 2] (src, dst)
     info: dict = field(default_factory=dict)
+    # parallel sampling: the n candidates of a prompt form a group of consecutive
+    # sequences whose first shared_blocks[g] blocks are the same physical blocks
+    group_start: torch.Tensor | None = None    # int32 [G + 1]
+    shared_blocks: torch.Tensor | None = None  # int32 [G]
 
     @property
     def ctx_list(self) -> list[int]:
@@ -223,7 +227,11 @@ def _layout_sampling(spec, rng):
                 tables[b, j] = next(perm)
     info = {"demand_blocks": demand, "shared_prompt_blocks": P * n_prompt_blk,
             "ref_count_prompt": n, "cow_pairs": len(pairs),
-            "ref_count_last_prompt_block_after_cow": ref_count[int(tables[0, n_prompt_blk - 1])]}
+            "ref_count_last_prompt_block_after_cow": ref_count[int(tables[0, n_prompt_blk - 1])],
+            # blocks every candidate of a prompt still shares: all but the copied-on-write last one (a
+            # single candidate: the prompt's full blocks, before the one its new tokens go to)
+            "groups": (np.arange(0, P * n + 1, n, dtype=np.int32),
+                       np.full(P, n_prompt_blk - 1 if n > 1 else plen // bs, np.int32))}
     return ctx, tables, NB, np.asarray(pairs, np.int64).reshape(-1, 2), info
 
 
@@ -281,6 +289,7 @@ def make_decode_workload(spec: DecodeSpec, seed: int = 0, device: str | torch.de
             if c > 0:
                 s[b] = int(tables[b, (c - 1) // bs]) * bs + (c - 1) % bs
         slot = torch.from_numpy(s).to(device)
+    groups = info.pop("groups", None)
     info.update({"num_blocks": NB, "max_blocks_per_seq": int(tables.shape[1]),
                  "total_tokens": int(ctx.sum())})
     return DecodeWorkload(
@@ -292,7 +301,9 @@ def make_decode_workload(spec: DecodeSpec, seed: int = 0, device: str | torch.de
         scale=float(np.float32(1.0 / math.sqrt(d))),
         new_k=new_k, new_v=new_v, slot_mapping=slot,
         copy_pairs=None if pairs is None else torch.from_numpy(pairs).to(device),
-        info=info)
+        info=info,
+        group_start=None if groups is None else torch.from_numpy(groups[0]).to(device),
+        shared_blocks=None if groups is None else torch.from_numpy(groups[1]).to(device))
 
 
 @dataclass
