@@ -297,8 +297,10 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
     if grouped:
         n_groups = int(w.group_start.shape[0]) - 1
         max_group = int((w.group_start[1:] - w.group_start[:-1]).max().item())
+        pt = pk.decode_shared_prefix_partition_tokens(n_groups, s.num_kv_heads, s.block_size, MB,
+                                                      args.partition_tokens)
         ws_bytes = pk.decode_shared_prefix_workspace_bytes(s.num_seqs, n_groups, s.num_q_heads, s.num_kv_heads,
-                                                           s.head_dim, s.block_size, MB, args.partition_tokens)
+                                                           s.head_dim, s.block_size, MB, pt)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     out = torch.empty_like(w.q)
     stream = torch.cuda.current_stream(dev)
@@ -308,7 +310,7 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
             pk.paged_attention_decode_shared_prefix(w.q, kc, vc, tables, w.context_lens, w.group_start,
                                                     w.shared_blocks, w.scale, k_new=w.new_k, v_new=w.new_v,
                                                     max_group_size=max_group, out=out, workspace=workspace,
-                                                    partition_tokens=args.partition_tokens, stream=stream)
+                                                    partition_tokens=pt, stream=stream)
         elif fused:  # the new token (one per sequence, at ctx - 1) is written inside the decode launch
             pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, tables, w.context_lens, w.scale,
                                    k_scale=w.k_scale, v_scale=w.v_scale, out=out, workspace=workspace,

@@ -228,11 +228,19 @@ int pkv_paged_attention_decode_shared_prefix(void* out, const void* q, const voi
                                              int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
                                              size_t workspace_bytes, int validate, void* stream);
 
+/* Partition length pkv_paged_attention_decode_shared_prefix uses: partition_tokens
+ * when non-zero (a positive multiple of block_size, at most 16384, else
+ * PKV_ERR_PARTITION), otherwise the automatic choice of pkv_decode_partition_tokens
+ * made for the groups' shared units (num_groups x num_kv_heads) on the bf16
+ * tensor-core kernel, with at least three partitions per long context instead of
+ * four (the members' own units fill the last wave).  Negative PKV_ERR_* on bad
+ * arguments.  A sizing helper of this library. */
+int pkv_decode_shared_prefix_partition_tokens(int num_groups, int num_kv_heads, int block_size,
+                                              int max_blocks_per_seq, int partition_tokens);
+
 /* Workspace bytes of pkv_paged_attention_decode_shared_prefix (0 for
- * unsupported arguments).  Its partition length is partition_tokens, or the
- * automatic choice of pkv_decode_partition_tokens made for the groups' shared
- * units (num_groups x num_kv_heads) on the bf16 tensor-core kernel.  A sizing
- * helper of this library. */
+ * unsupported arguments): 2 x ceil(max_blocks_per_seq x block_size / P)
+ * partial slots per (sequence, query head), P the partition length above. */
 size_t pkv_decode_shared_prefix_workspace_bytes(int num_seqs, int num_groups, int num_q_heads, int num_kv_heads,
                                                 int head_dim, int block_size, int max_blocks_per_seq,
                                                 int partition_tokens);

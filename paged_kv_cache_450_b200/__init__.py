@@ -33,7 +33,8 @@ STATUS_BAD_QUERY_LOC = 0x20
 STATUS_BAD_GROUP = 0x40
 
 __all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "paged_attention_decode_shared_prefix",
-           "decode_shared_prefix_workspace_bytes", "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
+           "decode_shared_prefix_workspace_bytes", "decode_shared_prefix_partition_tokens",
+           "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "decode_table_scan", "device_status", "launch_count", "PagedKVError",
@@ -211,6 +212,15 @@ def multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv
     return int(_lib.load().pkv_multiquery_workspace_bytes(num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads,
                                                           head_dim, block_size, max_blocks_per_seq,
                                                           _cache_code(cache_dtype), partition_tokens))
+
+
+def decode_shared_prefix_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq,
+                                          partition_tokens=0) -> int:
+    """Partition length paged_attention_decode_shared_prefix uses for these arguments."""
+    r = _lib.load().pkv_decode_shared_prefix_partition_tokens(num_groups, num_kv_heads, block_size,
+                                                              max_blocks_per_seq, partition_tokens)
+    _check(min(r, 0), "decode_shared_prefix_partition_tokens")
+    return int(r)
 
 
 def decode_shared_prefix_workspace_bytes(num_seqs, num_groups, num_q_heads, num_kv_heads, head_dim, block_size,

@@ -25,6 +25,7 @@ SIGNATURES = {
     "pkv_paged_decode_append": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I64, F, F, F, I, I, I, P, SZ, I, P]),
     "pkv_paged_attention_decode_shared_prefix": (I, [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F, I,
                                                      I, I, P, SZ, I, P]),
+    "pkv_decode_shared_prefix_partition_tokens": (I, [I, I, I, I, I]),
     "pkv_decode_shared_prefix_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),
     "pkv_paged_attention_decode_static": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I64, F, F, F, I, I, I, P]),
     "pkv_decode_step_host": (I, [P, P, P, P, P, I64, P, P, P, I64, P, P, I, I, I, I, I, I, I64, F, F, F, I, I, I,

@@ -145,13 +145,13 @@ static int decode_ctas_per_sm(int cache_dtype, int head_dim, int group, int bloc
 // for shorter contexts (measured 22% faster than four on the 128-sequence
 // parallel-sampling batch).
 static int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_blocks_per_seq,
-                                 int ctas_per_sm) {
+                                 int ctas_per_sm, int64_t few_pairs_min_parts = 4) {
   const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
   if (max_ctx <= 512) return static_cast<int>(cdiv64(max_ctx, block_size) * block_size);
   const int64_t slots = static_cast<int64_t>(ctas_per_sm) * sm_count();
   const bool many = pairs >= 4 * slots;
-  const int64_t min_parts = many ? 1 : 4;
+  const int64_t min_parts = many ? 1 : few_pairs_min_parts;
   int pt = many ? 2048 : 4096;
   while (pt > 128 && (cdiv64(max_ctx, pt) < min_parts || 4 * pairs * cdiv64(max_ctx, pt) < 3 * slots)) pt /= 2;
   return pt < block_size ? block_size : pt;
@@ -609,8 +609,19 @@ static int shared_prefix_partition_tokens(int num_groups, int num_kv_heads, int 
       return PKV_ERR_PARTITION;
     return partition_tokens;
   }
+  // The members' own units (one per sequence and KV head) run beside the shared ones and fill
+  // the gaps of the last wave, so the shared part takes three splits at least rather than four
+  // (measured on 32 prompts of 1024 tokens x 4 candidates x 40 heads: 512-token partitions
+  // 2.4% faster than 256, 128 19% slower).
   return auto_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq,
-                               decode_ctas_per_sm(PKV_DTYPE_BF16, 128, 2, block_size));
+                               decode_ctas_per_sm(PKV_DTYPE_BF16, 128, 2, block_size), 3);
+}
+
+int pkv_decode_shared_prefix_partition_tokens(int num_groups, int num_kv_heads, int block_size,
+                                              int max_blocks_per_seq, int partition_tokens) {
+  if (num_groups <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_BAD_SHAPE;
+  if (block_size != 16 && block_size != 32) return PKV_ERR_BLOCK_SIZE;
+  return shared_prefix_partition_tokens(num_groups, num_kv_heads, block_size, max_blocks_per_seq, partition_tokens);
 }
 
 size_t pkv_decode_shared_prefix_workspace_bytes(int num_seqs, int num_groups, int num_q_heads, int num_kv_heads,

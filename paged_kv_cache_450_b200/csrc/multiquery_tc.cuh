@@ -73,8 +73,10 @@ struct MqTcTraits {
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
   static constexpr int TILE = 2 * HALF;      // 32 KB: 128 rows x 128 16-bit values
   // K and V rings (fp8 caches: the raw codes land in a stage's upper half and
-  // are widened to fp16 in place)
-  static constexpr int NSK = 3, NSV = 2;
+  // are widened to fp16 in place).  Three V stages: a V tile is issued once the
+  // P . V two tiles back has read its stage, so it has about two tiles' time
+  // to land.
+  static constexpr int NSK = 3, NSV = 3;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
@@ -83,13 +85,16 @@ struct MqTcTraits {
   // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, k_ready[NSK], v_ready[NSV]
   static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + NSK + NSV : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
-  static constexpr int XCH_OFF = SLOT_OFF + 16;          // float [4][128 rows]: m_0, m_1, l_0, l_1
-  static constexpr int IDS_OFF = XCH_OFF + 4 * 128 * 4;
+  // float [4][128 rows]: m_0, m_1, l_0, l_1 of the epilogue, over the Q tile: every S has
+  // completed before the epilogue starts (the last P . V, which it waits for, was issued after them)
+  static constexpr int XCH_OFF = Q_OFF;
   static constexpr int THREADS = 352;
   static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or fp16 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr size_t smem_bytes(int pb) { return 1024 + IDS_OFF + static_cast<size_t>(pb) * 4; }
+  // (block ids are read from the table as the tiles are issued: nothing depends on the partition length)
+  static constexpr size_t smem_bytes(int /*partition_blocks*/) { return 1024 + SLOT_OFF + 16; }
+  static_assert(1024 + SLOT_OFF + 16 + 64 <= 232448, "shared memory of one CTA");
 };
 
 // 3-D tiled TMA load (coordinates innermost first; c0 is 0 or 64 elements).
@@ -194,7 +199,6 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int* ids = reinterpret_cast<int*>(data + T::IDS_OFF);
 
   const int Hkv = p.num_kv_heads;
   __shared__ int seq_slot;
@@ -261,6 +265,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
   auto v_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NSK + s); };
   const uint64_t policy = l2_policy_evict_first();
   const int* table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb;
+  // physical id of the partition's block i (i < nb), -1 when outside the pool
+  auto block_id = [&](int i) {
+    const int id = table[i];
+    return id < 0 || id >= p.num_blocks ? -1 : id;
+  };
+  // producers: lane i < BPT takes block i of tile j (-1 past the partition's blocks or outside the pool)
+  auto tile_block = [&](int j) {
+    const int i = j * T::BPT + lane;
+    return lane < T::BPT && i < nb ? block_id(i) : -1;
+  };
   if (warp == T::W_K) {
     // The K producer starts the first loads before the CTA-wide set-up: it
     // initialises the barriers (no other thread touches them before the
@@ -318,15 +332,12 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
 
   int local_bad = 0;
   for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-    int id = table[i];
-    if (id < 0 || id >= p.num_blocks) {
+    if (block_id(i) < 0) {
       set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
-      id = -1;
       local_bad = 1;
     }
-    ids[i] = id;
   }
-  const bool any_bad = __syncthreads_or(local_bad) != 0;  // (also orders the ids before their use)
+  const bool any_bad = __syncthreads_or(local_bad) != 0;
   if (warp == T::W_K) {
     __syncwarp();
     tmem_alloc(base + T::SLOT_OFF, T::TMEM_COLS);
@@ -347,21 +358,26 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     const int ns = is_k ? T::NSK : T::NSV;
     const int area = is_k ? T::K_OFF : T::V_OFF;
     auto full = [&](int st) { return is_k ? k_full(st) : v_full(st); };
-    auto issue = [&](int j) {  // lane 0: tile j's raw codes into the upper half of stage j % ns
+    // whole warp: tile j's raw codes into the upper half of stage j % ns, lane i loading block i;
+    // `id` is tile_block(j), read one issue ahead so that the table's latency is off the path
+    auto issue = [&](int j, int id) {
       const int st = j % ns;
-      const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
-      int nvalid = 0;
-      for (int i = i0; i < i1; ++i) nvalid += ids[i] >= 0;
-      const uint32_t bytes = static_cast<uint32_t>(nvalid) * BS * 128u;
-      if (bytes) mbar_arrive_expect_tx(full(st), bytes); else mbar_arrive(full(st));
-      for (int i = i0; i < i1; ++i)
-        if (ids[i] >= 0)
-          tma_load_4d(base + area + st * T::TILE + T::HALF + (i - i0) * BS * 128, map, full(st), 0, hk, 0, ids[i],
-                      policy);
+      const unsigned vm = __ballot_sync(kFullMask, id >= 0);
+      if (lane == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(__popc(vm)) * BS * 128u;
+        if (bytes) mbar_arrive_expect_tx(full(st), bytes); else mbar_arrive(full(st));
+      }
+      __syncwarp();
+      if (id >= 0)
+        tma_load_4d(base + area + st * T::TILE + T::HALF + lane * BS * 128, map, full(st), 0, hk, 0, id, policy);
     };
     int issued = min(nt, ns);
-    if (lane == 0)
-      for (int j = is_k ? 1 : 0; j < issued; ++j) issue(j);  // (K tile 0 went out in the prologue)
+    int next = is_k ? 1 : 0;  // (K tile 0 went out in the prologue)
+    int next_id = next < nt ? tile_block(next) : -1;
+    for (; next < issued; ++next) {
+      issue(next, next_id);
+      next_id = next + 1 < nt ? tile_block(next + 1) : -1;
+    }
     int landed = 0;
     for (int j = 0; j < nt; ++j) {
       const int st = j % ns;
@@ -373,7 +389,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         widen_e4m3_tile_in_place(stage, lane, [](int) { return false; });
       } else {     // V rows that must not contribute (past tok_end, bad blocks) are zeroed
         widen_e4m3_tile_in_place(stage, lane, [&](int t) {
-          return tile0 + t >= tok_end || (any_bad && ids[(tile0 + t - tok_begin) / BS] < 0);
+          return tile0 + t >= tok_end || (any_bad && block_id((tile0 + t - tok_begin) / BS) < 0);
         });
       }
       __syncwarp();
@@ -386,10 +402,9 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         if (!__all_sync(kFullMask, mbar_wait_bounded(is_k ? k_empty(sp) : v_empty(sp), ((j - 1) / ns) & 1,
                                                      p.status)))
           break;
-        if (lane == 0) {
-          fence_proxy_async_smem();  // this warp's reads and writes of the stage before the TMA write
-          issue(jr);
-        }
+        fence_proxy_async_smem();  // this warp's reads and writes of the stage before the TMA write
+        issue(jr, next_id);
+        next_id = jr + 1 < nt ? tile_block(jr + 1) : -1;
         issued = jr + 1;
       }
     }
@@ -399,31 +414,34 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       for (int j = landed; j < issued; ++j) mbar_wait_bounded(full(j % ns), (j / ns) & 1, p.status);
     }
   } else if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
-    if (lane == 0) {
-      const bool is_k = warp == T::W_K;
-      const int ns = is_k ? T::NSK : T::NSV;
-      const CUtensorMap* map = is_k ? &kmap : &vmap;
-      const uint32_t area = base + (is_k ? T::K_OFF : T::V_OFF);
-      int issued = is_k ? 1 : 0;  // Q and K tile 0 were issued in the prologue
-      for (int j = issued; j < nt; ++j) {
-        const int s = j % ns, use = j / ns;
-        const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
-        const int i0 = j * T::BPT, i1 = min(nb, i0 + T::BPT);
-        int nvalid = 0;
-        for (int i = i0; i < i1; ++i) nvalid += ids[i] >= 0;
-        const uint32_t bytes = static_cast<uint32_t>(nvalid) * 2u * BS * 128u;
-        if (use > 0 && !mbar_wait_bounded(empty, (use - 1) & 1, p.status)) break;
+    // whole warp: lane i < BPT loads block i of each tile (both 64-dim halves); the block ids of
+    // the next tile are read from the table while the stage it needs is still in use
+    const bool is_k = warp == T::W_K;
+    const int ns = is_k ? T::NSK : T::NSV;
+    const CUtensorMap* map = is_k ? &kmap : &vmap;
+    const uint32_t area = base + (is_k ? T::K_OFF : T::V_OFF);
+    int issued = is_k ? 1 : 0;  // Q and K tile 0 were issued in the prologue
+    int id = issued < nt ? tile_block(issued) : -1;
+    for (int j = issued; j < nt; ++j) {
+      const int s = j % ns, use = j / ns;
+      const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
+      const unsigned vm = __ballot_sync(kFullMask, id >= 0);
+      if (use > 0 && !warp_wait_bounded(empty, (use - 1) & 1, p.status)) break;
+      if (lane == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(__popc(vm)) * 2u * BS * 128u;
         if (bytes) mbar_arrive_expect_tx(full, bytes); else mbar_arrive(full);
-        for (int i = i0; i < i1; ++i) {
-          const int id = ids[i];
-          if (id < 0) continue;
-          const uint32_t dst = area + s * T::TILE + (i - i0) * BS * 128;
-          tma_load_4d(dst, map, full, 0, hk, 0, id, policy);
-          tma_load_4d(dst + T::HALF, map, full, 64, hk, 0, id, policy);
-        }
-        issued = j + 1;
       }
-      // drain (bounded): the copies of the last stages have landed before exit
+      __syncwarp();
+      if (id >= 0) {
+        const uint32_t dst = area + s * T::TILE + lane * BS * 128;
+        tma_load_4d(dst, map, full, 0, hk, 0, id, policy);
+        tma_load_4d(dst + T::HALF, map, full, 64, hk, 0, id, policy);
+      }
+      issued = j + 1;
+      id = j + 1 < nt ? tile_block(j + 1) : -1;
+    }
+    // drain (bounded): the copies of the last stages have landed before exit
+    if (lane == 0) {
       if (is_k) mbar_wait_bounded(q_full, 0, p.status);
       for (int j = max(0, issued - ns); j < issued; ++j)
         mbar_wait_bounded(is_k ? k_full(j % ns) : v_full(j % ns), (j / ns) & 1, p.status);
@@ -513,18 +531,21 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       wait(v_full(j % T::NSV), (j / T::NSV) & 1);
       const int vr = 64 * h + 16 * quarter + (lane >> 1);
       const int t = tok_begin + j * T::TOK + vr;
-      if (t >= tok_end || (bad && ids[(t - tok_begin) / BS] < 0)) {
+      if (t >= tok_end || (bad && block_id((t - tok_begin) / BS) < 0)) {
         uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
     };
-    auto half_tile_bad = [&](int t0) {  // a block of this half tile with a bad id
-      bool bad = false;
+    // bit k set: block k of the half tile starting at token t0 has a bad id (t0 - tok_begin is a
+    // multiple of 64, so the half tile holds 64 / BS whole blocks)
+    auto half_tile_bad = [&](int t0) {
+      unsigned bad = 0u;
       if (any_bad) {
-        const int i0 = (t0 - tok_begin) / BS, i1 = min(nb, (t0 + 64 - tok_begin) / BS);
-        for (int i = i0; i < i1; ++i) bad |= ids[i] < 0;
+        const int i0 = (t0 - tok_begin) / BS;
+        for (int k = 0; k < 64 / BS && i0 + k < nb; ++k)
+          if (block_id(i0 + k) < 0) bad |= 1u << k;
       }
       return bad;
     };
@@ -541,7 +562,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        const bool bad = half_tile_bad(t0);
+        const bool bad = half_tile_bad(t0) != 0u;
         if (j > 0) wait(pv_done(h), (j - 1) & 1);
         if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
         tc_fence_before();
@@ -571,7 +592,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       if (lane == 0) mbar_arrive(s_free);
 
       // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
-      const bool bad = half_tile_bad(t0);
+      const unsigned bad_blocks = half_tile_bad(t0);
+      const bool bad = bad_blocks != 0u;
       const bool ragged = t0 + 64 > tok_end;  // tokens at or past tok_end in this half tile
       // row max of the raw scores (q_scale > 0 commutes with the max); masked scores -> -inf.
       // Eight independent partial maxima / sums: instruction-level parallelism hides latency.
@@ -582,7 +604,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         if (bad) {  // scores of blocks that were not loaded (stale tiles) never reach the max
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (ids[(t0 + c - tok_begin) / BS] < 0) sv[c] = -INFINITY;
+            if ((bad_blocks >> (c / BS)) & 1u) sv[c] = -INFINITY;
         }
         // column c is visible iff c <= last (causal position and the end of what is loaded)
         const int last = min(pos, tok_end - 1) - t0;

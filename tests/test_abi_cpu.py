@@ -108,6 +108,26 @@ def test_partition_choice_and_workspace_size():
         pk.decode_partition_tokens(1, 1, 1, 128, 16, 100, bf16, 40)
 
 
+def test_shared_prefix_partition_and_workspace():
+    # 32 groups x 40 heads over up to 1088 tokens: three partitions at least -> 512 tokens
+    assert pk.decode_shared_prefix_partition_tokens(32, 40, 16, 68) == 512
+    # the plain decode of the same batch (128 x 40 pairs) keeps one partition
+    assert pk.decode_partition_tokens(128, 40, 40, 128, 16, 68, torch.bfloat16) == 2048
+    assert pk.decode_shared_prefix_partition_tokens(32, 40, 16, 68, 256) == 256
+    assert pk.decode_shared_prefix_partition_tokens(2, 2, 16, 20) == 320   # <= 512 tokens: one partition
+    with pytest.raises(pk.PagedKVError):
+        pk.decode_shared_prefix_partition_tokens(32, 40, 16, 68, 24)
+    with pytest.raises(pk.PagedKVError):
+        pk.decode_shared_prefix_partition_tokens(32, 40, 8, 68)
+    # two slots (shared + own) per partition of the longest table, per (sequence, query head): m, l and 128 floats
+    P = 2 * -(-68 * 16 // 512)
+    rows = 128 * 40 * P
+    assert pk.decode_shared_prefix_workspace_bytes(128, 32, 40, 40, 128, 16, 68) == \
+        (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
+    assert pk.decode_shared_prefix_workspace_bytes(128, 32, 40, 40, 128, 16, 68, 512) == \
+        pk.decode_shared_prefix_workspace_bytes(128, 32, 40, 40, 128, 16, 68)
+
+
 def test_multiquery_partition_and_workspace():
     lib = _lib.load()
     BF, F8 = pk.DTYPE_BF16, pk.DTYPE_FP8_E4M3

@@ -235,6 +235,27 @@ def test_rows_past_the_context_are_never_used(spec):
         assert torch.isfinite(out.float()).all()
 
 
+@pytest.mark.parametrize("hkv", [1, 2, 3, 6])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_fp8_gqa8_kv_head_counts(hkv, bs):
+    """fp8 cache, 8 query heads per KV head (the tensor-core kernel) with odd and even KV-head
+    counts: the oracle's result, with the fused new-token write, at several partition lengths."""
+    spec = W.GQA_BATCH.with_(num_seqs=4, num_q_heads=8 * hkv, num_kv_heads=hkv, block_size=bs,
+                             ctx=("list", (1, 3 * bs + 5, 700, 2 * bs)))
+    w = W.make_decode_workload(spec, seed=20 + hkv + bs, device=DEV)
+    for pt in (0, bs, 4 * bs):
+        check_step(w, partition_tokens=pt, what=f"hkv={hkv} bs={bs} pt={pt}")
+    kc, vc = w.key_cache.clone(), w.value_cache.clone()
+    out = pk.paged_decode_append(w.q, w.new_k, w.new_v, kc, vc, w.block_tables, w.context_lens, w.scale,
+                                 k_scale=w.k_scale, v_scale=w.v_scale, partition_tokens=bs, validate=True)
+    torch.cuda.synchronize()
+    rk, rv, ref = oracle_step(w)
+    assert_cache_equal(kc, rk, "append key_cache")
+    assert_cache_equal(vc, rv, "append value_cache")
+    assert_close(f64(out), ref, *tol_for(w), what=f"fused append hkv={hkv} bs={bs}")
+    assert pk.device_status(clear=True) == 0
+
+
 def test_tensor_core_kernel_guards_bad_block_ids():
     w = W.make_decode_workload(W.GQA_BATCH.with_(num_seqs=3, ctx=("list", (40, 300, 7)), new_tokens=False), seed=13,
                                device=DEV)
