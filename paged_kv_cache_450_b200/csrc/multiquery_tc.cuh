@@ -64,10 +64,22 @@
 
 namespace pkv {
 
-template <int BS, bool F8 = false>
+// ROWS = 128 query rows per CTA (the MMA's M), or -- bf16 caches, at most
+// 64 rows per (sequence, KV head), as in grouped verification (5 queries x 8
+// heads = 40) -- ROWS = 64 *stacked*: MMA rows 64-127 repeat rows 0-63 (the Q
+// tile's first 64 rows are copied below them), so S holds every score twice;
+// the warps of TMEM lanes 0-63 write P's bf16 high part and those of lanes
+// 64-127 its residual for the same rows, and each P . V k-step is ONE M = 128
+// MMA whose accumulator rows 64-127 collect the residual's share (added back
+// in the epilogue).  The single issuing thread pays per MMA instruction (an
+// M = 64 MMA measured no faster than M = 128), so this takes a tile from 24
+// instructions to 16.
+template <int BS, bool F8 = false, int ROWS_ = 128>
 struct MqTcTraits {
   static constexpr int D = 128;
-  static constexpr int ROWS = 128;           // query rows per CTA (MMA M)
+  static constexpr int ROWS = ROWS_;         // query rows per CTA
+  static constexpr bool STACK = ROWS == 64;  // hi / lo parts of P stacked in the MMA's rows
+  static_assert(ROWS == 128 || (ROWS == 64 && !F8), "M = 128, or 64 rows stacked (bf16 caches)");
   static constexpr int TOK = 128;            // tokens per KV tile
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
@@ -83,13 +95,16 @@ struct MqTcTraits {
   static constexpr int BAR_OFF = V_OFF + NSV * TILE;
   // mbarriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free, p_full[2],
   // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, k_ready[NSK], v_ready[NSV]
-  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + NSK + NSV : 0);
+  // (stacked rows add q_ready: the copy of the Q rows is in place)
+  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   // float [4][128 rows]: m_0, m_1, l_0, l_1 of the epilogue, over the Q tile: every S has
   // completed before the epilogue starts (the last P . V, which it waits for, was issued after them)
   static constexpr int XCH_OFF = Q_OFF;
-  static constexpr int THREADS = 352;
-  static constexpr int W_K = 8, W_MMA = 9, W_V = 10;  // producer / issuer warps
+  // Warp w runs on sub-partition w % 4, the one whose TMEM lanes 32 (w % 4) .. it may access.
+  // The MMA issuer sits on sub-partition 3; warp 9 has no role.
+  static constexpr int THREADS = 384;
+  static constexpr int W_K = 8, W_MMA = 11, W_V = 10;  // producer / issuer warps
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or fp16 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
   // (block ids are read from the table as the tiles are issued: nothing depends on the partition length)
@@ -113,11 +128,40 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return d;
 }
 
+// Waits of this kernel: the thread sleeps inside mbarrier.try_wait (the hardware
+// wakes it when the phase completes, or after the hint of 20 us) instead of
+// polling.  Four to five warps share each sub-partition; a warp polling a
+// barrier takes issue slots from the softmax warps beside it (measured: the
+// softmax warps of the MMA issuer's sub-partition ran ~1000 cycles per tile
+// behind the others).  Still bounded: gives up after kWaitLimitNs in all.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, unsigned* status) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, PKV_STATUS_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Bounded wait taken by every lane of a warp; the result is the same on every
 // lane (false if any lane gave up), so the warp stays converged for the
 // .sync.aligned tensor-memory instructions that follow.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, unsigned* status) {
-  return __all_sync(kFullMask, mbar_wait_bounded(bar, parity, status));
+  return __all_sync(kFullMask, mbar_wait_sleep(bar, parity, status));
 }
 
 // Longest work first.  CTAs start roughly in grid order and one runs per SM,
@@ -189,13 +233,13 @@ __device__ __forceinline__ void widen_e4m3_tile_in_place(uint8_t* stage, int lan
   fence_proxy_async_smem();
 }
 
-template <int BS, int G, bool F8>
-__global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
+template <int BS, int G, bool F8, int ROWS = 128>
+__global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
     paged_multiquery_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap, const MultiQueryParams p) {
-  using T = MqTcTraits<BS, F8>;
+  using T = MqTcTraits<BS, F8, ROWS>;
   constexpr int D = T::D;
-  constexpr int QPT = T::ROWS / G;  // queries per CTA tile
+  constexpr int QPT = T::ROWS / G;  // queries per CTA tile (the Q box holds 128 / G; stacked: the first QPT)
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -301,6 +345,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
         for (int s = 0; s < T::NSV; ++s) mbar_init(v_ready(s), 1);
       }
+      if constexpr (T::STACK) mbar_init(q_ready, 4);
       fence_barrier_init();
       mbar_arrive_expect_tx(q_full, T::TILE);
       tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
@@ -381,7 +426,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     int landed = 0;
     for (int j = 0; j < nt; ++j) {
       const int st = j % ns;
-      if (!__all_sync(kFullMask, mbar_wait_bounded(full(st), (j / ns) & 1, p.status))) break;
+      if (!__all_sync(kFullMask, mbar_wait_sleep(full(st), (j / ns) & 1, p.status))) break;
       landed = j + 1;
       uint8_t* stage = data + area + st * T::TILE;
       const int tile0 = tok_begin + j * T::TOK;
@@ -399,7 +444,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       const int jr = j - 1 + ns;
       if (j >= 1 && jr < nt) {
         const int sp = (j - 1) % ns;
-        if (!__all_sync(kFullMask, mbar_wait_bounded(is_k ? k_empty(sp) : v_empty(sp), ((j - 1) / ns) & 1,
+        if (!__all_sync(kFullMask, mbar_wait_sleep(is_k ? k_empty(sp) : v_empty(sp), ((j - 1) / ns) & 1,
                                                      p.status)))
           break;
         fence_proxy_async_smem();  // this warp's reads and writes of the stage before the TMA write
@@ -410,8 +455,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     }
     // drain (bounded): the raw loads started have landed before exit
     if (lane == 0) {
-      if (is_k) mbar_wait_bounded(q_full, 0, p.status);
-      for (int j = landed; j < issued; ++j) mbar_wait_bounded(full(j % ns), (j / ns) & 1, p.status);
+      if (is_k) mbar_wait_sleep(q_full, 0, p.status);
+      for (int j = landed; j < issued; ++j) mbar_wait_sleep(full(j % ns), (j / ns) & 1, p.status);
     }
   } else if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
     // whole warp: lane i < BPT loads block i of each tile (both 64-dim halves); the block ids of
@@ -442,9 +487,9 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     }
     // drain (bounded): the copies of the last stages have landed before exit
     if (lane == 0) {
-      if (is_k) mbar_wait_bounded(q_full, 0, p.status);
+      if (is_k) mbar_wait_sleep(q_full, 0, p.status);
       for (int j = max(0, issued - ns); j < issued; ++j)
-        mbar_wait_bounded(is_k ? k_full(j % ns) : v_full(j % ns), (j / ns) & 1, p.status);
+        mbar_wait_sleep(is_k ? k_full(j % ns) : v_full(j % ns), (j / ns) & 1, p.status);
     }
   } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
     if (lane == 0) {
@@ -452,13 +497,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
-      bool ok = mbar_wait_bounded(F8 ? q_ready : q_full, 0, p.status);
+      bool ok = mbar_wait_sleep(F8 || T::STACK ? q_ready : q_full, 0, p.status);
       // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1)
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
           const int sk = j % T::NSK;
-          if (!(ok = mbar_wait_bounded(F8 ? k_ready(sk) : k_full(sk), (j / T::NSK) & 1, p.status))) break;
-          if (j > 0 && !(ok = mbar_wait_bounded(s_free, (j - 1) & 1, p.status))) break;
+          if (!(ok = mbar_wait_sleep(F8 ? k_ready(sk) : k_full(sk), (j / T::NSK) & 1, p.status))) break;
+          if (j > 0 && !(ok = mbar_wait_sleep(s_free, (j - 1) & 1, p.status))) break;
           tc_fence_after();
           // descriptors differ only in the start-address field (address >> 4 in the low bits, all
           // addresses below 256 KB): the base descriptors plus offsets
@@ -475,15 +520,15 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
           const int jj = j - 1, sv = jj % T::NSV;
           const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
           // the V tile (bf16: landed; fp8: widened)
-          if (!(ok = mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (jj / T::NSV) & 1, p.status))) break;
+          if (!(ok = mbar_wait_sleep(F8 ? v_ready(sv) : v_full(sv), (jj / T::NSV) & 1, p.status))) break;
           for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
-            if (!(ok = mbar_wait_bounded(p_full(h), jj & 1, p.status))) break;
+            if (!(ok = mbar_wait_sleep(p_full(h), jj & 1, p.status))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
               const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
               tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-              if constexpr (!F8) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+              if constexpr (!F8 && !T::STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
             }
             tc_commit(pv_done(h));
           }
@@ -493,14 +538,20 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       }
       // drain (bounded): no MMA may still read shared memory or write TMEM at exit
       tc_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, p.status);
+      mbar_wait_sleep(mma_done, 0, p.status);
     }
-  } else {  // ---------------- softmax warps 0-7 ------------------------------------------
+  } else if (warp < 8) {  // ---------------- softmax warps 0-7 --------------------------------------
     const int quarter = warp & 3, h = warp >> 2;  // TMEM lane quarter, token half of each tile
-    const int r = 32 * quarter + lane;            // this thread's row (TMEM lane)
+    const int tl = 32 * quarter + lane;           // this thread's TMEM lane
+    // its query row; stacked: lanes 64-127 repeat rows 0-63 and write the residual part of P
+    const bool lo_part = T::STACK && quarter >= 2;
+    const int r = T::STACK ? tl & 63 : tl;
     const int row = qt * T::ROWS + r;
     const bool valid = row < rows_total;
-    const int pos = valid ? base_pos + row / G : -1;  // an invalid row sees nothing
+    // an invalid row (its output is never written) sees what the CTA's last row sees, so that it
+    // takes the same path as its warp's valid rows (a row that saw nothing would take the masking
+    // path alone and hold the warp on it every tile); its P only feeds its own accumulator row
+    const int pos = base_pos + (valid ? row : row_last) / G;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float qk = p.q_scale;
     float m = -INFINITY, l = 0.f;  // this half's running reference max (log2 units) and row sum
@@ -554,7 +605,21 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
     // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
     // output rows nobody writes.
-    if (qt * T::ROWS + 32 * quarter >= rows_total) {
+    if constexpr (T::STACK) {  // Q rows 0-63 (both 64-dim halves) copied below themselves, same swizzle phase
+      if (lo_part) {
+        wait(q_full, 0);
+        // the two warps of half h copy the 64-dim half h: 64 threads x 8 x 16 bytes
+        const int i = 32 * (quarter - 2) + lane;
+        const uint4* src = reinterpret_cast<const uint4*>(data + T::Q_OFF + h * T::HALF);
+        uint4* dst = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + 64 * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[i + 64 * c] = src[i + 64 * c];
+        fence_proxy_async_smem();  // these writes before the MMA's reads (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_ready);
+      }
+    }
+    if (qt * T::ROWS + (T::STACK ? 32 * (quarter & 1) : 32 * quarter) >= rows_total) {
       for (int j = 0; j < nt; ++j) {
         const int t0 = tok_begin + j * T::TOK + 64 * h;
         wait(s_full, j & 1);
@@ -677,17 +742,18 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         }
       }
       if (!F8 && (ragged || bad)) zero_v_rows(j, bad);
-      // this half of row r of P into TMEM lane r
+      // this half of row r of P into TMEM lane r (stacked: the high part in lanes 0-63, the residual
+      // in lanes 64-127, both in P_h's columns)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pw[16], lw[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          pw[k] = ph[16 * c + k];
+          pw[k] = lo_part ? plo[16 * c + k] : ph[16 * c + k];
           lw[k] = plo[16 * c + k];
         }
         tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
-        if constexpr (!F8) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
+        if constexpr (!F8 && !T::STACK) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -697,17 +763,22 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     wait(pv_done(h), (nt - 1) & 1);
     tc_fence_after();
     // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 -----
-    float* xch = reinterpret_cast<float*>(data + T::XCH_OFF);  // [m_0, m_1, l_0, l_1][row]
-    xch[h * 128 + r] = m;
-    xch[(2 + h) * 128 + r] = l;
+    float* xch = reinterpret_cast<float*>(data + T::XCH_OFF);  // [m_0, m_1, l_0, l_1][TMEM lane]
+    xch[h * 128 + tl] = m;
+    xch[(2 + h) * 128 + tl] = l;
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");  // the two warps of this lane quarter
-    const float m_o = xch[(h ^ 1) * 128 + r], l_o = xch[(2 + (h ^ 1)) * 128 + r];
+    const float m_o = xch[(h ^ 1) * 128 + tl], l_o = xch[(2 + (h ^ 1)) * 128 + tl];
     const float M = fmaxf(l > 0.f ? m : -INFINITY, l_o > 0.f ? m_o : -INFINITY);
     const float w_self = l > 0.f ? fast_exp2(m - M) : 0.f, w_oth = l_o > 0.f ? fast_exp2(m_o - M) : 0.f;
     const float lsum = l * w_self + l_o * w_oth;
     const float inv = lsum > 0.f ? p.out_scale / lsum : 0.f;
     const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
     const int64_t orow = static_cast<int64_t>(q0 + row / G) * Hq + hk * G + row % G;
+    // stacked rows: the residual's share of this row's output (accumulator rows 64-127) goes from
+    // the warp of lanes 64-127 to the warp of the same row and half through the free K ring
+    float* xo = reinterpret_cast<float*>(data + T::K_OFF);  // [64 rows][128 dims]
+    const int pair_bar = 5 + 2 * (quarter & 1) + h;      // named barrier of the two warps of this row
+    if (T::STACK && !lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       const int d0 = 64 * h + 32 * c;
@@ -720,6 +791,22 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       float o[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u0[e]) * w0 + __uint_as_float(u1[e]) * w1;
+      if constexpr (T::STACK) {
+        float4* x4 = reinterpret_cast<float4*>(xo + r * 128 + d0);
+        if (lo_part) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) x4[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+          continue;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 v = x4[e / 4];
+          o[e] += v.x;
+          o[e + 1] += v.y;
+          o[e + 2] += v.z;
+          o[e + 3] += v.w;
+        }
+      }
       if (nparts == 1) {
         __nv_bfloat16* dst = out + orow * D + d0;
 #pragma unroll
@@ -738,7 +825,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
       }
     }
-    if (valid && ok && nparts > 1 && h == 0) {
+    if (T::STACK && lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+    if (valid && ok && nparts > 1 && h == 0 && !lo_part) {
       const int64_t srow = orow * p.max_partitions + part;
       p.ws_ml[srow * 2] = lsum > 0.f ? M * kLn2 : 0.f;
       p.ws_ml[srow * 2 + 1] = lsum;
