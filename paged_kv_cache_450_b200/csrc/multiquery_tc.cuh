@@ -168,21 +168,27 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 // so the tail of a launch is set by the long units that start last.  Grid z
 // index z therefore takes the sequence whose context is the z-th longest
 // (ties by index: a permutation of the sequences); every thread of the CTA
-// takes part (two CTA barriers).  More than 1024 sequences keep grid order.
-__device__ __forceinline__ int longest_first_sequence(const MultiQueryParams& p, int z, int* slot) {
+// takes part (three CTA barriers).  The context lengths are staged in
+// `scratch` (shared memory no load has reached yet) so that the B x B
+// comparisons read shared memory, not the cache hierarchy.  More than 1024
+// sequences keep grid order.
+__device__ __forceinline__ int longest_first_sequence(const MultiQueryParams& p, int z, int* slot, int* scratch) {
   const int B = p.num_seqs;
   if (B > 1024) return z;
   if (threadIdx.x == 0) *slot = z;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) scratch[i] = p.context_lens[i];
   __syncthreads();
   for (int t = threadIdx.x; t < B; t += blockDim.x) {
-    const int lt = p.context_lens[t];
+    const int lt = scratch[t];
     int rank = 0;
+#pragma unroll 4
     for (int j = 0; j < B; ++j) {
-      const int lj = p.context_lens[j];
+      const int lj = scratch[j];
       rank += (lj > lt) || (lj == lt && j < t);
     }
     if (rank == z) *slot = t;
   }
+  fence_proxy_async_smem();  // the scratch writes before the tile loads that later land there
   __syncthreads();
   return *slot;
 }
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
 
   const int Hkv = p.num_kv_heads;
   __shared__ int seq_slot;
-  const int b = longest_first_sequence(p, blockIdx.z, &seq_slot);
+  const int b = longest_first_sequence(p, blockIdx.z, &seq_slot, reinterpret_cast<int*>(data + T::V_OFF));
   // the last query tile of a sequence sees the most tokens: it goes first
   const int hk = blockIdx.x % Hkv, qt = gridDim.x / Hkv - 1 - blockIdx.x / Hkv, part = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -500,7 +500,8 @@ def test_multiquery_prefill_sized_tiles(bs, hq, hkv):
         _mq_check(mw, partition_tokens=pt, what=f"bs={bs} hq={hq} hkv={hkv} pt={pt}")
 
 
-@pytest.mark.parametrize("q_lens", [(5, 5, 5, 5), (200, 129, 64, 300)], ids=["verify", "prefill"])
+@pytest.mark.parametrize("q_lens", [(5, 5, 5, 5), (12, 9, 12, 3), (200, 129, 64, 300)],
+                         ids=["verify", "verify-stacked-tile", "prefill"])
 def test_multiquery_rows_past_the_context_are_never_used(q_lens):
     ctxs = (300, 129, 100, 700)
     spec = W.DecodeSpec("mqnan", len(ctxs), 8, 4, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
@@ -537,8 +538,8 @@ def test_multiquery_guards_bad_block_ids(q_lens):
 
 
 def test_multiquery_long_context_largest_partition():
-    # a 16384-token partition (1024 block ids of bs 16 in the tcgen05 kernel's shared memory) and a
-    # context split in two by it
+    # a 16384-token partition (1024 blocks of bs 16, their ids read tile by tile by the tcgen05 kernel's
+    # producers) and a context split in two by it
     ctxs = (20000, 16384, 300)
     spec = W.DecodeSpec("mqlong", len(ctxs), 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, ("list", ctxs),
                         ("slack", 1.05))
@@ -613,7 +614,7 @@ def test_multiquery_one_query_per_sequence_matches_decode():
     assert_close(f64(mq), f64(dec), *TOL_BF16, what="multi-query vs decode")
 
 
-@pytest.mark.parametrize("q_lens", [(4, 2, 3), (100, 200, 40)], ids=["verify", "prefill"])
+@pytest.mark.parametrize("q_lens", [(4, 2, 3), (12, 5, 9), (100, 200, 40)], ids=["verify", "verify-stacked-tile", "prefill"])
 @pytest.mark.parametrize("case", ["end_past_total", "negative_start", "q_len_above_max"])
 def test_multiquery_guards_bad_query_start_loc(q_lens, case):
     """query_start_loc entries outside [0, total_q] (or a q_len above max_q_len) reach the kernels only
