@@ -5,29 +5,30 @@
 
 namespace pkv {
 
-template <int BS, int G, bool F8, int ROWS>
-static cudaError_t launch_mq_tc_rows(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                                     const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
-  using T = MqTcTraits<BS, F8, ROWS>;
-  auto kern = paged_multiquery_tc_kernel<BS, G, F8, ROWS>;
-  const size_t smem = T::smem_bytes(p.partition_blocks);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.num_kv_heads) * n_qtiles, p.max_partitions, p.num_seqs);
-  e = launch_pdl(kern, grid, dim3(T::THREADS), smem, st, qmap, kmap, vmap, p);
-  if (e != cudaSuccess || !reduce) return e;
-  return launch_multiquery_reduce(p, st);
+// Persistent launch: one CTA per SM (fewer when there are fewer work units);
+// each CTA takes units c, c + CTAs, ... of the longest-first unit list.
+static int sm_count_of_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n;
 }
 
-// n_qtiles counts 128-row tiles.  bf16 caches with at most 64 rows per (sequence, KV head) run the
-// stacked 64-row tile (one MMA per P . V k-step instead of two).
 template <int BS, int G, bool F8>
 static cudaError_t launch_mq_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                                 const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
-  if constexpr (!F8) {
-    if (p.max_q_len * G <= 64) return launch_mq_tc_rows<BS, G, F8, 64>(qmap, kmap, vmap, p, 1, reduce, st);
-  }
-  return launch_mq_tc_rows<BS, G, F8, 128>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
+  using T = MqTcTraits<BS, F8>;
+  auto kern = paged_multiquery_tc_kernel<BS, G, F8>;
+  const size_t smem = T::smem_bytes(p.partition_blocks);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t units = static_cast<int64_t>(p.num_kv_heads) * n_qtiles * p.max_partitions * p.num_seqs;
+  const int64_t ctas = units < sm_count_of_device() ? units : sm_count_of_device();
+  if (ctas <= 0) return cudaSuccess;
+  e = launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(T::THREADS), smem, st, qmap, kmap, vmap, p);
+  if (e != cudaSuccess || !reduce) return e;
+  return launch_multiquery_reduce(p, st);
 }
 
 template <int BS, bool F8>

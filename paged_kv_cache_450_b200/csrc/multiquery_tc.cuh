@@ -5,15 +5,26 @@
 // Same operation as multiquery.cuh (causal over the paged cache, queries are
 // the sequence's last q_len positions), written for the Blackwell MMA:
 //
-//   one CTA = 128 query rows (query i, head g; g fastest) x one KV head x one
-//   split-context partition; KV tiles of 128 tokens (8 blocks of 16 or 4 of 32)
-//   from the partition's start (a partition that is not a multiple of 128
-//   tokens ends in a partial tile, masked like the context end).
+//   a work unit = 128 query rows (query i, head g; g fastest) x one KV head x
+//   one split-context partition; KV tiles of 128 tokens (8 blocks of 16 or 4
+//   of 32) from the partition's start (a partition that is not a multiple of
+//   128 tokens ends in a partial tile, masked like the context end).
 //   S = Q . K^T      M = 128 rows, N = 128 tokens, K = 128 dims -> TMEM columns [0, 128)
 //   O_h += P_h . V_h M = 128 rows, N = 128 dims,   K = 64 tokens (half h of the tile)
 //                    -> TMEM columns [128, 256) (h = 0) and [256, 384) (h = 1)
 // (Every MMA is as wide as the operands allow: the single issuing thread pays
-// about the same per instruction for N = 64 as for N = 128.)
+// per instruction, 80-125 cycles whatever M and N.)
+//
+// Persistent CTAs: one CTA per SM (the launch has min(units, SMs) CTAs) takes
+// one unit of every round of CTAs-many units of the unit list, which is ordered
+// longest context first (the last query tile of a sequence first): unit c of
+// even rounds, unit CTAs - 1 - c of odd rounds (a CTA that got one of the
+// longest units of a round gets one of the shortest of the next).  Barrier
+// phases and ring stages run on per-CTA counters across units, so the next
+// unit's Q and first K / V tiles load while the current unit finishes, and the
+// TMEM allocation, the barrier set-up and the CTA launch are paid once per SM
+// instead of once per unit (measured ~8 us per unit: a third of a prefill
+// unit of 8-9 tiles).
 //
 // Q, K and V sit in shared memory in the 128-byte-swizzled layout (two
 // 64-element halves of every 256-byte row) as TMA delivers them; Q and K are
@@ -25,34 +36,35 @@
 // costs up to ~3e-3 absolute on short contexts), packed with integer byte
 // permutes.  (One fp16 P over V converted to fp16 in shared memory halves the
 // P . V MMAs but measured 1.7x slower: the conversions compete with the
-// exponentials.)  Eleven warps:
-//   warps 0-7  softmax: warp w serves rows 32 (w & 3) .. +31 (the TMEM lanes
-//              its sub-partition may touch) and half h = w >> 2 of every KV
-//              tile's tokens.  The two halves are independent online
+// exponentials.)  Thirteen warps (warp w runs on sub-partition w % 4):
+//   warps 0-7  softmax: warp w serves the rows in TMEM lanes 32 (w & 3) .. +31
+//              (the lanes its sub-partition may touch) and half h = w >> 2 of
+//              every KV tile's tokens.  The two halves are independent online
 //              softmaxes -- each with its own running max, row sum and
 //              accumulator O_h -- so the two warps of a sub-partition never
 //              wait for each other and their special-function (exp) and
 //              integer / FMA (P packing) phases interleave; they are merged
-//              once, in the epilogue.  Per tile a thread reads its 64 scores
-//              from TMEM, applies the causal / context mask, keeps a
+//              once per unit, in the epilogue (the (m, l) exchange goes through
+//              TMEM columns of P, free by then).  Per tile a thread reads its 64
+//              scores from TMEM, applies the causal / context mask, keeps a
 //              reference max (O_h is rescaled only when a score passes it by
 //              more than 2^8), and writes its 64 probabilities into P_h.
-//   warp 8     TMA producer of Q (once) and the K tiles (three-stage ring; one
-//              4-D box per block and 64-dim half); owns the TMEM allocation.
-//   warp 10    TMA producer of the V tiles (two-stage ring), so that a K load
-//              never waits behind a V stage that P . V still holds.
-//   warp 9     MMA issuer: one thread issues S_j as soon as the softmax has
+//   warp 8     TMA producer of Q and the K tiles (three-stage ring; one 4-D box
+//              per block and 64-dim half); owns the TMEM allocation.
+//   warp 10    TMA producer of the V tiles (three-stage ring).
+//   warp 11    MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
 //              is signalled through tcgen05.commit on mbarriers.
-// Caches of fp8 (E4M3, F8 = true): the K and V producer warps TMA each tile's
-// raw codes (128 bytes per token row) into the upper half of the tile's own
-// ring stage and then, all 32 lanes, widen them exactly to fp16 in place (one
-// thread per token row reads the raw row whole, then writes its two fp16
-// halves; V rows that must not contribute are zeroed there) -- the rings have
-// the bf16 layout and depths, so widening overlaps the MMAs; the softmax warps
-// round their Q rows to fp16 once; both MMAs run on fp16 operands, and P is
-// one fp16 value (11 significant bits; columns [384, 448)).  The K scale is
-// folded into the logit scale, the V scale into the output.
+//   warps 9, 12  fp8 caches: widen the K (9) and V (12) tiles (bf16: warp 9 idles, no warp 12).
+// Caches of fp8 (E4M3, F8 = true): the producer warps TMA each tile's raw codes
+// (128 bytes per token row) into the upper half of the tile's own ring stage;
+// warps 9 and 12 then widen them exactly to fp16 in place (one thread per token
+// row reads the raw row whole, then writes its two fp16 halves; V rows that
+// must not contribute are zeroed there) -- the rings have the bf16 layout and
+// depths, so widening overlaps the MMAs; the softmax warps round their Q rows to
+// fp16 once per unit; both MMAs run on fp16 operands, and P is one fp16 value
+// (11 significant bits; columns [384, 448)).  The K scale is folded into the
+// logit scale, the V scale into the output.
 // Every wait is bounded (2 s); on a timeout the status bit is set, the
 // producer and issuer loops stop, the softmax warps skip their remaining
 // waits, in-flight work is drained with bounded waits and TMEM is freed.
@@ -64,22 +76,10 @@
 
 namespace pkv {
 
-// ROWS = 128 query rows per CTA (the MMA's M), or -- bf16 caches, at most
-// 64 rows per (sequence, KV head), as in grouped verification (5 queries x 8
-// heads = 40) -- ROWS = 64 *stacked*: MMA rows 64-127 repeat rows 0-63 (the Q
-// tile's first 64 rows are copied below them), so S holds every score twice;
-// the warps of TMEM lanes 0-63 write P's bf16 high part and those of lanes
-// 64-127 its residual for the same rows, and each P . V k-step is ONE M = 128
-// MMA whose accumulator rows 64-127 collect the residual's share (added back
-// in the epilogue).  The single issuing thread pays per MMA instruction (an
-// M = 64 MMA measured no faster than M = 128), so this takes a tile from 24
-// instructions to 16.
-template <int BS, bool F8 = false, int ROWS_ = 128>
+template <int BS, bool F8 = false>
 struct MqTcTraits {
   static constexpr int D = 128;
-  static constexpr int ROWS = ROWS_;         // query rows per CTA
-  static constexpr bool STACK = ROWS == 64;  // hi / lo parts of P stacked in the MMA's rows
-  static_assert(ROWS == 128 || (ROWS == 64 && !F8), "M = 128, or 64 rows stacked (bf16 caches)");
+  static constexpr int ROWS = 128;           // query rows per unit (MMA M)
   static constexpr int TOK = 128;            // tokens per KV tile
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
@@ -93,23 +93,23 @@ struct MqTcTraits {
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
   static constexpr int BAR_OFF = V_OFF + NSV * TILE;
-  // mbarriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free, p_full[2],
-  // pv_done[2], mma_done (the pairs: one per token half); fp8 caches add q_ready, k_ready[NSK], v_ready[NSV]
-  // (stacked rows add q_ready: the copy of the Q rows is in place)
-  static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 7 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
+  // mbarriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free,
+  // p_full[2], pv_done[2] (one per token half), o_free, mma_done; fp8 caches add q_ready, k_ready[NSK],
+  // v_ready[NSV]
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
-  // float [4][128 rows]: m_0, m_1, l_0, l_1 of the epilogue, over the Q tile: every S has
-  // completed before the epilogue starts (the last P . V, which it waits for, was issued after them)
-  static constexpr int XCH_OFF = Q_OFF;
-  // Warp w runs on sub-partition w % 4, the one whose TMEM lanes 32 (w % 4) .. it may access.
-  // The MMA issuer sits on sub-partition 3; warp 9 has no role.
-  static constexpr int THREADS = 384;
-  static constexpr int W_K = 8, W_MMA = 11, W_V = 10;  // producer / issuer warps
+  // the sequence of each of the CTA's first MAX_UNITS units (longest-first rank -> sequence)
+  static constexpr int MAX_UNITS = 64;
+  static constexpr int UNIT_OFF = SLOT_OFF + 16;
+  // 13 warps with fp8 caches (the two widening warps), 12 otherwise: each sub-partition's registers
+  // hold at most three warps of the bf16 kernel's ~140 registers (four would cap them at 128)
+  static constexpr int THREADS = F8 ? 416 : 384;
+  static constexpr int W_K = 8, W_KWIDEN = 9, W_V = 10, W_MMA = 11, W_VWIDEN = 12;
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or fp16 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
   // (block ids are read from the table as the tiles are issued: nothing depends on the partition length)
-  static constexpr size_t smem_bytes(int /*partition_blocks*/) { return 1024 + SLOT_OFF + 16; }
-  static_assert(1024 + SLOT_OFF + 16 + 64 <= 232448, "shared memory of one CTA");
+  static constexpr size_t smem_bytes(int /*partition_blocks*/) { return 1024 + UNIT_OFF + 4 * MAX_UNITS; }
+  static_assert(1024 + UNIT_OFF + 4 * MAX_UNITS + 64 <= 232448, "shared memory of one CTA");
 };
 
 // 3-D tiled TMA load (coordinates innermost first; c0 is 0 or 64 elements).
@@ -164,33 +164,102 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
   return __all_sync(kFullMask, mbar_wait_sleep(bar, parity, status));
 }
 
-// Longest work first.  CTAs start roughly in grid order and one runs per SM,
-// so the tail of a launch is set by the long units that start last.  Grid z
-// index z therefore takes the sequence whose context is the z-th longest
-// (ties by index: a permutation of the sequences); every thread of the CTA
-// takes part (three CTA barriers).  The context lengths are staged in
-// `scratch` (shared memory no load has reached yet) so that the B x B
-// comparisons read shared memory, not the cache hierarchy.  More than 1024
-// sequences keep grid order.
-__device__ __forceinline__ int longest_first_sequence(const MultiQueryParams& p, int z, int* slot, int* scratch) {
+// One work unit: (query tile qt, KV head hk) = x, partition = y, longest-first
+// rank = z of the unit list (x fastest), its sequence b.  Every thread of the
+// CTA computes the same description from the same global data.
+struct MqUnit {
+  int b, hk, qt, part;
+  int q0, q_len, rows_total, base_pos, row_last;
+  int tok_begin, tok_end, nt, nb, nparts;
+  const int32_t* table;  // the partition's block ids
+  int kind;              // kRun, kSkip (nothing to do), kZero (write zero rows, then nothing), kBadQuery
+};
+enum { kRun = 0, kSkip = 1, kZero = 2, kBadQuery = 3 };
+
+template <int BS, int G>
+__device__ __forceinline__ MqUnit mq_unit(const MultiQueryParams& p, int64_t u, int b, int gx, int gy) {
+  MqUnit U;
+  const int x = static_cast<int>(u % gx), y = static_cast<int>((u / gx) % gy);
+  const int Hkv = p.num_kv_heads, n_qt = gx / Hkv;
+  U.b = b;
+  U.hk = x % Hkv;
+  U.qt = n_qt - 1 - x / Hkv;  // the last query tile of a sequence sees the most tokens: it goes first
+  U.part = y;
+  U.table = nullptr;
+  U.nt = U.nb = U.nparts = 0;
+  if (!query_rows_ok(p, b, U.q0, U.q_len)) {  // before any load or store
+    U.kind = kBadQuery;
+    return U;
+  }
+  U.rows_total = U.q_len * G;
+  U.kind = kSkip;
+  if (U.q_len <= 0 || U.qt * 128 >= U.rows_total) return U;
+  const int max_ctx = p.max_blocks_per_seq * BS;
+  int ctx = p.context_lens[b];
+  if (ctx < 0 || ctx > max_ctx) {
+    if (threadIdx.x == 0 && U.hk == 0 && U.part == 0 && U.qt == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
+    ctx = ctx < 0 ? 0 : max_ctx;
+  }
+  const int nblk = (ctx + BS - 1) / BS;
+  const int pb = p.partition_blocks;
+  const int nparts = (nblk + pb - 1) / pb;
+  U.nparts = nparts;
+  U.base_pos = ctx - U.q_len;
+  U.row_last = min(U.rows_total, (U.qt + 1) * 128) - 1;
+  const int pos_last = U.base_pos + U.row_last / G;
+  if (nparts == 0 || pos_last < 0) {  // nothing to attend: zero rows (partition 0 writes them)
+    if (U.part == 0) U.kind = kZero;
+    return U;
+  }
+  if (U.part >= nparts) return U;
+  U.tok_begin = U.part * pb * BS;
+  // tokens this unit's rows can see in the partition: [tok_begin, tok_end)
+  U.tok_end = min(min(ctx, U.tok_begin + pb * BS), pos_last + 1);
+  if (U.tok_end <= U.tok_begin) return U;  // every row sits before this partition (never merged)
+  U.nt = (U.tok_end - U.tok_begin + 127) / 128;
+  U.nb = (U.tok_end - U.tok_begin + BS - 1) / BS;
+  U.table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + U.part * pb;
+  U.kind = kRun;
+  return U;
+}
+
+// Unit k of this CTA: round k, position c or CTAs - 1 - c (see above); may be
+// past the last unit (n_all) in the last round.
+__device__ __forceinline__ int64_t cta_unit(int k) {
+  const int64_t c = (k & 1) ? gridDim.x - 1 - blockIdx.x : blockIdx.x;
+  return static_cast<int64_t>(k) * gridDim.x + c;
+}
+
+// Longest work first.  Unit rank z takes the sequence whose context is the
+// z-th longest (ties by index: a permutation of the sequences), so that the
+// units that start last are the short ones.  Each thread ranks whole
+// sequences from the context lengths staged in `scratch` (shared memory no
+// load has reached yet) and records the sequence of every unit of this CTA
+// with that rank.  Fewer than 1025 sequences and MAX_UNITS rounds; otherwise
+// units keep the sequences' order (unit_b unused).
+__device__ __forceinline__ void rank_units(const MultiQueryParams& p, int gxy, int n_rounds, int* scratch,
+                                           int* unit_b) {
   const int B = p.num_seqs;
-  if (B > 1024) return z;
-  if (threadIdx.x == 0) *slot = z;
   for (int i = threadIdx.x; i < B; i += blockDim.x) scratch[i] = p.context_lens[i];
   __syncthreads();
   for (int t = threadIdx.x; t < B; t += blockDim.x) {
     const int lt = scratch[t];
-    int rank = 0;
+    int r = 0;
 #pragma unroll 4
     for (int j = 0; j < B; ++j) {
       const int lj = scratch[j];
-      rank += (lj > lt) || (lj == lt && j < t);
+      r += (lj > lt) || (lj == lt && j < t);
     }
-    if (rank == z) *slot = t;
+    // this CTA's units u with u / gxy == r lie in rounds u_lo / CTAs .. (u_hi - 1) / CTAs
+    const int64_t u_lo = static_cast<int64_t>(r) * gxy, u_hi = u_lo + gxy;  // [u_lo, u_hi)
+    const int64_t k_hi = min(static_cast<int64_t>(n_rounds) - 1, (u_hi - 1) / gridDim.x);
+    for (int64_t k = u_lo / gridDim.x; k <= k_hi; ++k) {
+      const int64_t u = cta_unit(static_cast<int>(k));
+      if (u >= u_lo && u < u_hi) unit_b[k] = t;
+    }
   }
   fence_proxy_async_smem();  // the scratch writes before the tile loads that later land there
   __syncthreads();
-  return *slot;
 }
 
 // Widens one KV tile of raw E4M3 codes in place.  The raw codes of token row
@@ -239,158 +308,96 @@ __device__ __forceinline__ void widen_e4m3_tile_in_place(uint8_t* stage, int lan
   fence_proxy_async_smem();
 }
 
-template <int BS, int G, bool F8, int ROWS = 128>
-__global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
+template <int BS, int G, bool F8>
+__global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     paged_multiquery_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap, const MultiQueryParams p) {
-  using T = MqTcTraits<BS, F8, ROWS>;
+  using T = MqTcTraits<BS, F8>;
   constexpr int D = T::D;
-  constexpr int QPT = T::ROWS / G;  // queries per CTA tile (the Q box holds 128 / G; stacked: the first QPT)
+  constexpr int QPT = T::ROWS / G;  // queries per unit
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* data = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  const int Hkv = p.num_kv_heads;
-  __shared__ int seq_slot;
-  const int b = longest_first_sequence(p, blockIdx.z, &seq_slot, reinterpret_cast<int*>(data + T::V_OFF));
-  // the last query tile of a sequence sees the most tokens: it goes first
-  const int hk = blockIdx.x % Hkv, qt = gridDim.x / Hkv - 1 - blockIdx.x / Hkv, part = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int q0, q_len;
-  if (!query_rows_ok(p, b, q0, q_len)) {  // before any load or store
-    if (threadIdx.x == 0) set_status(p.status, PKV_STATUS_BAD_QUERY_LOC);
-    return;
-  }
-  const int rows_total = q_len * G;
-  if (q_len <= 0 || qt * T::ROWS >= rows_total) return;
-  const int max_ctx = p.max_blocks_per_seq * BS;
-  int ctx = p.context_lens[b];
-  if (ctx < 0 || ctx > max_ctx) {
-    if (threadIdx.x == 0 && hk == 0 && part == 0 && qt == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
-    ctx = ctx < 0 ? 0 : max_ctx;
-  }
-  const int nblk = (ctx + BS - 1) / BS;
-  const int pb = p.partition_blocks;
-  const int nparts = (nblk + pb - 1) / pb;
-  const int Hq = p.num_q_heads;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-  const int base_pos = ctx - q_len;
-  const int row_last = min(rows_total, (qt + 1) * T::ROWS) - 1;
-  const int pos_last = base_pos + row_last / G;
-  if (nparts == 0 || pos_last < 0) {  // nothing to attend: zero rows (partition 0 writes them)
-    if (part == 0 && threadIdx.x < T::ROWS) {
-      const int row = qt * T::ROWS + threadIdx.x;
-      if (row < rows_total) {
-        const int64_t orow = static_cast<int64_t>(q0 + row / G) * Hq + hk * G + row % G;
-        for (int d = 0; d < D; d += 8)
-          *reinterpret_cast<uint4*>(out + orow * D + d) = make_uint4(0u, 0u, 0u, 0u);
-      }
+  const int Hkv = p.num_kv_heads, Hq = p.num_q_heads;
+  const int n_qt = (p.max_q_len * G + T::ROWS - 1) / T::ROWS;
+  const int gx = Hkv * n_qt, gy = p.max_partitions;
+  const int64_t n_all = static_cast<int64_t>(gx) * gy * p.num_seqs;
+  const int n_units = static_cast<int>((n_all + gridDim.x - 1) / gridDim.x);  // rounds (the last may miss this CTA)
+  int* unit_b = reinterpret_cast<int*>(data + T::UNIT_OFF);
+  const bool ranked = p.num_seqs <= 1024 && n_units <= T::MAX_UNITS;
+  if (ranked) rank_units(p, gx * gy, n_units, reinterpret_cast<int*>(data + T::V_OFF), unit_b);
+  // unit k of this CTA (kind kSkip past the last unit)
+  auto unit_at = [&](int k) {
+    const int64_t u = cta_unit(k);
+    if (u >= n_all) {
+      MqUnit U;
+      U.kind = kSkip;
+      U.nt = 0;
+      return U;
     }
-    return;
-  }
-  if (part >= nparts) return;
-  const int tok_begin = part * pb * BS;
-  // tokens this CTA's rows can see in the partition: [tok_begin, tok_end)
-  const int tok_end = min(min(ctx, tok_begin + pb * BS), pos_last + 1);
-  if (tok_end <= tok_begin) return;  // every row sits before this partition (never merged)
-  const int nt = (tok_end - tok_begin + T::TOK - 1) / T::TOK;
-  const int nb = (tok_end - tok_begin + BS - 1) / BS;
+    const int z = static_cast<int>(u / (static_cast<int64_t>(gx) * gy));
+    return mq_unit<BS, G>(p, u, ranked ? unit_b[k] : z, gx, gy);
+  };
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 
   const uint32_t base = smem_u32(data);
   const uint32_t bar0 = base + T::BAR_OFF;
-  const uint32_t q_full = bar0;
-  auto k_full = [&](int s) { return bar0 + 8 * (1 + s); };
-  auto k_empty = [&](int s) { return bar0 + 8 * (1 + T::NSK + s); };
-  auto v_full = [&](int s) { return bar0 + 8 * (1 + 2 * T::NSK + s); };
-  auto v_empty = [&](int s) { return bar0 + 8 * (1 + 2 * T::NSK + T::NSV + s); };
-  // P-full and P.V-done barriers per token half h (each completes once per tile)
-  constexpr int B2 = 1 + 2 * T::NSK + 2 * T::NSV;
-  const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1), mma_done = bar0 + 8 * (B2 + 6);
+  const uint32_t q_full = bar0, q_empty = bar0 + 8;
+  auto k_full = [&](int s) { return bar0 + 8 * (2 + s); };
+  auto k_empty = [&](int s) { return bar0 + 8 * (2 + T::NSK + s); };
+  auto v_full = [&](int s) { return bar0 + 8 * (2 + 2 * T::NSK + s); };
+  auto v_empty = [&](int s) { return bar0 + 8 * (2 + 2 * T::NSK + T::NSV + s); };
+  constexpr int B2 = 2 + 2 * T::NSK + 2 * T::NSV;
+  const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1);
   auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
   auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
+  const uint32_t o_free = bar0 + 8 * (B2 + 6), mma_done = bar0 + 8 * (B2 + 7);
   // fp8 caches: Q rounded to fp16, K / V stages widened (k_full / v_full: their raw codes landed)
-  constexpr int B3 = B2 + 7;
+  constexpr int B3 = B2 + 8;
   const uint32_t q_ready = bar0 + 8 * B3;
   auto k_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
   auto v_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NSK + s); };
   const uint64_t policy = l2_policy_evict_first();
-  const int* table = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + part * pb;
-  // physical id of the partition's block i (i < nb), -1 when outside the pool
-  auto block_id = [&](int i) {
-    const int id = table[i];
+  // physical id of block i of the unit's partition (i < nb), -1 when outside the pool
+  auto block_id = [&](const MqUnit& U, int i) {
+    const int id = U.table[i];
     return id < 0 || id >= p.num_blocks ? -1 : id;
   };
   // producers: lane i < BPT takes block i of tile j (-1 past the partition's blocks or outside the pool)
-  auto tile_block = [&](int j) {
+  auto tile_block = [&](const MqUnit& U, int j) {
     const int i = j * T::BPT + lane;
-    return lane < T::BPT && i < nb ? block_id(i) : -1;
+    return lane < T::BPT && i < U.nb ? block_id(U, i) : -1;
   };
-  if (warp == T::W_K) {
-    // The K producer starts the first loads before the CTA-wide set-up: it
-    // initialises the barriers (no other thread touches them before the
-    // barrier below), then fetches Q and the first K tile itself.
-    if (lane == 0) {
-      mbar_init(q_full, 1);
-      for (int s = 0; s < T::NSK; ++s) {
-        mbar_init(k_full(s), 1);
-        mbar_init(k_empty(s), 1);
-      }
-      for (int s = 0; s < T::NSV; ++s) {
-        mbar_init(v_full(s), 1);
-        mbar_init(v_empty(s), 1);
-      }
-      mbar_init(s_full, 1);
-      mbar_init(s_free, 8);
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(p_full(h), 4);
-        mbar_init(pv_done(h), 1);
-      }
-      mbar_init(mma_done, 1);
-      if constexpr (F8) {
-        mbar_init(q_ready, 8);
-        for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
-        for (int s = 0; s < T::NSV; ++s) mbar_init(v_ready(s), 1);
-      }
-      if constexpr (T::STACK) mbar_init(q_ready, 4);
-      fence_barrier_init();
-      mbar_arrive_expect_tx(q_full, T::TILE);
-      tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, hk * G, q0 + qt * QPT);
-      tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, hk * G, q0 + qt * QPT);
-    }
-    // K tile 0: lane i < blocks of the tile reads block id i
-    int id = -1;
-    if (lane < min(nb, T::BPT)) {
-      id = table[lane];
-      if (id < 0 || id >= p.num_blocks) id = -1;  // (reported by the scan below)
-    }
-    const unsigned valid = __ballot_sync(kFullMask, id >= 0);
-    // bf16: the tile into K stage 0; fp8: the raw codes into the stage's upper half
-    if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(__popc(valid)) * (F8 ? 1u : 2u) * BS * 128u;
-      if (bytes) mbar_arrive_expect_tx(k_full(0), bytes); else mbar_arrive(k_full(0));
-    }
-    __syncwarp();
-    if (id >= 0) {
-      if constexpr (F8) {
-        tma_load_4d(base + T::K_OFF + T::HALF + lane * BS * 128, &kmap, k_full(0), 0, hk, 0, id, policy);
-      } else {
-        const uint32_t dst = base + T::K_OFF + lane * BS * 128;
-        tma_load_4d(dst, &kmap, k_full(0), 0, hk, 0, id, policy);
-        tma_load_4d(dst + T::HALF, &kmap, k_full(0), 64, hk, 0, id, policy);
-      }
-    }
-  }
 
-  int local_bad = 0;
-  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-    if (block_id(i) < 0) {
-      set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
-      local_bad = 1;
+  if (threadIdx.x == T::W_K * 32) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < T::NSK; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
     }
+    for (int s = 0; s < T::NSV; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(p_full(h), 4);
+      mbar_init(pv_done(h), 1);
+    }
+    mbar_init(o_free, 8);
+    mbar_init(mma_done, 1);
+    if constexpr (F8) {
+      mbar_init(q_ready, 8);
+      for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
+      for (int s = 0; s < T::NSV; ++s) mbar_init(v_ready(s), 1);
+    }
+    fence_barrier_init();
   }
-  const bool any_bad = __syncthreads_or(local_bad) != 0;
+  __syncthreads();
   if (warp == T::W_K) {
-    __syncwarp();
     tmem_alloc(base + T::SLOT_OFF, T::TMEM_COLS);
     tmem_relinquish();
   }
@@ -403,99 +410,87 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
   auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };    // tokens 64h .. 64h+63 packed in pairs: hi / fp16
   auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };  // bf16 caches: the residual
 
-  if (F8 && (warp == T::W_K || warp == T::W_V)) {  // ---------- fp8: TMA raw codes, widen in place ----------
-    const bool is_k = warp == T::W_K;
-    const CUtensorMap* map = is_k ? &kmap : &vmap;
-    const int ns = is_k ? T::NSK : T::NSV;
-    const int area = is_k ? T::K_OFF : T::V_OFF;
-    auto full = [&](int st) { return is_k ? k_full(st) : v_full(st); };
-    // whole warp: tile j's raw codes into the upper half of stage j % ns, lane i loading block i;
-    // `id` is tile_block(j), read one issue ahead so that the table's latency is off the path
-    auto issue = [&](int j, int id) {
-      const int st = j % ns;
-      const unsigned vm = __ballot_sync(kFullMask, id >= 0);
-      if (lane == 0) {
-        const uint32_t bytes = static_cast<uint32_t>(__popc(vm)) * BS * 128u;
-        if (bytes) mbar_arrive_expect_tx(full(st), bytes); else mbar_arrive(full(st));
-      }
-      __syncwarp();
-      if (id >= 0)
-        tma_load_4d(base + area + st * T::TILE + T::HALF + lane * BS * 128, map, full(st), 0, hk, 0, id, policy);
-    };
-    int issued = min(nt, ns);
-    int next = is_k ? 1 : 0;  // (K tile 0 went out in the prologue)
-    int next_id = next < nt ? tile_block(next) : -1;
-    for (; next < issued; ++next) {
-      issue(next, next_id);
-      next_id = next + 1 < nt ? tile_block(next + 1) : -1;
-    }
-    int landed = 0;
-    for (int j = 0; j < nt; ++j) {
-      const int st = j % ns;
-      if (!__all_sync(kFullMask, mbar_wait_sleep(full(st), (j / ns) & 1, p.status))) break;
-      landed = j + 1;
-      uint8_t* stage = data + area + st * T::TILE;
-      const int tile0 = tok_begin + j * T::TOK;
-      if (is_k) {  // scores of rows that are not loaded are masked, whatever these rows hold
-        widen_e4m3_tile_in_place(stage, lane, [](int) { return false; });
-      } else {     // V rows that must not contribute (past tok_end, bad blocks) are zeroed
-        widen_e4m3_tile_in_place(stage, lane, [&](int t) {
-          return tile0 + t >= tok_end || (any_bad && block_id((tile0 + t - tok_begin) / BS) < 0);
-        });
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(is_k ? k_ready(st) : v_ready(st));
-      // refill the stage of tile j - 1 with tile j - 1 + ns once its MMA has read it (by now it
-      // usually has: S(j-1) / P.V(j-1) were issued before tile j landed)
-      const int jr = j - 1 + ns;
-      if (j >= 1 && jr < nt) {
-        const int sp = (j - 1) % ns;
-        if (!__all_sync(kFullMask, mbar_wait_sleep(is_k ? k_empty(sp) : v_empty(sp), ((j - 1) / ns) & 1,
-                                                     p.status)))
-          break;
-        fence_proxy_async_smem();  // this warp's reads and writes of the stage before the TMA write
-        issue(jr, next_id);
-        next_id = jr + 1 < nt ? tile_block(jr + 1) : -1;
-        issued = jr + 1;
-      }
-    }
-    // drain (bounded): the raw loads started have landed before exit
-    if (lane == 0) {
-      if (is_k) mbar_wait_sleep(q_full, 0, p.status);
-      for (int j = landed; j < issued; ++j) mbar_wait_sleep(full(j % ns), (j / ns) & 1, p.status);
-    }
-  } else if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of K and of V ----------
-    // whole warp: lane i < BPT loads block i of each tile (both 64-dim halves); the block ids of
-    // the next tile are read from the table while the stage it needs is still in use
+  if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of Q and K, and of V --------
+    // whole warp: lane i < BPT loads block i of each tile; ring stages and phases run on the tile
+    // count g across the CTA's units
     const bool is_k = warp == T::W_K;
     const int ns = is_k ? T::NSK : T::NSV;
     const CUtensorMap* map = is_k ? &kmap : &vmap;
     const uint32_t area = base + (is_k ? T::K_OFF : T::V_OFF);
-    int issued = is_k ? 1 : 0;  // Q and K tile 0 were issued in the prologue
-    int id = issued < nt ? tile_block(issued) : -1;
-    for (int j = issued; j < nt; ++j) {
-      const int s = j % ns, use = j / ns;
-      const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
-      const unsigned vm = __ballot_sync(kFullMask, id >= 0);
-      if (use > 0 && !warp_wait_bounded(empty, (use - 1) & 1, p.status)) break;
-      if (lane == 0) {
-        const uint32_t bytes = static_cast<uint32_t>(__popc(vm)) * 2u * BS * 128u;
-        if (bytes) mbar_arrive_expect_tx(full, bytes); else mbar_arrive(full);
+    int g = 0, ku = 0;
+    bool ok = true;
+    for (int k = 0; ok && k < n_units; ++k) {
+      const MqUnit U = unit_at(k);
+      if (U.kind != kRun) continue;
+      if (is_k) {  // Q of this unit once the previous unit's S MMAs are done with the Q tile
+        if (ku > 0 && !(ok = warp_wait_bounded(q_empty, (ku - 1) & 1, p.status))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, T::TILE);
+          tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, U.hk * G, U.q0 + U.qt * QPT);
+          tma_load_3d(base + T::Q_OFF + T::HALF, &qmap, q_full, 64, U.hk * G, U.q0 + U.qt * QPT);
+        }
+        ++ku;
       }
-      __syncwarp();
-      if (id >= 0) {
-        const uint32_t dst = area + s * T::TILE + lane * BS * 128;
-        tma_load_4d(dst, map, full, 0, hk, 0, id, policy);
-        tma_load_4d(dst + T::HALF, map, full, 64, hk, 0, id, policy);
+      for (int j = 0; j < U.nt; ++j, ++g) {
+        const int s = g % ns, use = g / ns;
+        const int id = tile_block(U, j);  // (its latency overlaps the wait)
+        if (use > 0 && !(ok = warp_wait_bounded(is_k ? k_empty(s) : v_empty(s), (use - 1) & 1, p.status))) break;
+        const unsigned vm = __ballot_sync(kFullMask, id >= 0);
+        if (is_k && lane == 0 && __popc(vm) < min(T::BPT, U.nb - j * T::BPT))
+          set_status(p.status, PKV_STATUS_BAD_BLOCK_ID);
+        const uint32_t full = is_k ? k_full(s) : v_full(s);
+        if (lane == 0) {
+          const uint32_t bytes = static_cast<uint32_t>(__popc(vm)) * (F8 ? 1u : 2u) * BS * 128u;
+          if (bytes) mbar_arrive_expect_tx(full, bytes); else mbar_arrive(full);
+        }
+        __syncwarp();
+        if (id >= 0) {
+          if constexpr (F8) {  // the raw codes into the stage's upper half
+            tma_load_4d(area + s * T::TILE + T::HALF + lane * BS * 128, map, full, 0, U.hk, 0, id, policy);
+          } else {
+            const uint32_t dst = area + s * T::TILE + lane * BS * 128;
+            tma_load_4d(dst, map, full, 0, U.hk, 0, id, policy);
+            tma_load_4d(dst + T::HALF, map, full, 64, U.hk, 0, id, policy);
+          }
+        }
       }
-      issued = j + 1;
-      id = j + 1 < nt ? tile_block(j + 1) : -1;
     }
-    // drain (bounded): the copies of the last stages have landed before exit
+    // drain (bounded): the copies of the last stages (and the last Q) have landed before exit
     if (lane == 0) {
-      if (is_k) mbar_wait_sleep(q_full, 0, p.status);
-      for (int j = max(0, issued - ns); j < issued; ++j)
-        mbar_wait_sleep(is_k ? k_full(j % ns) : v_full(j % ns), (j / ns) & 1, p.status);
+      if (is_k && ku > 0) mbar_wait_sleep(q_full, (ku - 1) & 1, p.status);
+      for (int i = max(0, g - ns); i < g; ++i)
+        mbar_wait_sleep(is_k ? k_full(i % ns) : v_full(i % ns), (i / ns) & 1, p.status);
+    }
+  } else if (F8 && (warp == T::W_KWIDEN || warp == T::W_VWIDEN)) {  // ---- fp8: widen the landed tiles ----
+    const bool is_k = warp == T::W_KWIDEN;
+    const int ns = is_k ? T::NSK : T::NSV;
+    const int area = is_k ? T::K_OFF : T::V_OFF;
+    int g = 0;
+    bool ok = true;
+    for (int k = 0; ok && k < n_units; ++k) {
+      const MqUnit U = unit_at(k);
+      if (U.kind != kRun) continue;
+      // blocks of the unit with a bad id: their V rows are zeroed
+      bool any_bad = false;
+      if (!is_k) {
+        for (int i = lane; i < U.nb; i += 32) any_bad |= block_id(U, i) < 0;
+        any_bad = __any_sync(kFullMask, any_bad);
+      }
+      for (int j = 0; j < U.nt; ++j, ++g) {
+        const int st = g % ns;
+        if (!(ok = warp_wait_bounded(is_k ? k_full(st) : v_full(st), (g / ns) & 1, p.status))) break;
+        uint8_t* stage = data + area + st * T::TILE;
+        const int tile0 = U.tok_begin + j * T::TOK;
+        if (is_k) {  // scores of rows that are not loaded are masked, whatever these rows hold
+          widen_e4m3_tile_in_place(stage, lane, [](int) { return false; });
+        } else {     // V rows that must not contribute (past tok_end, bad blocks) are zeroed
+          widen_e4m3_tile_in_place(stage, lane, [&](int t) {
+            return tile0 + t >= U.tok_end || (any_bad && block_id(U, (tile0 + t - U.tok_begin) / BS) < 0);
+          });
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(is_k ? k_ready(st) : v_ready(st));
+      }
     }
   } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
     if (lane == 0) {
@@ -503,44 +498,56 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
       constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
-      bool ok = mbar_wait_sleep(F8 || T::STACK ? q_ready : q_full, 0, p.status);
-      // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1)
-      for (int j = 0; ok && j <= nt; ++j) {
-        if (j < nt) {
-          const int sk = j % T::NSK;
-          if (!(ok = mbar_wait_sleep(F8 ? k_ready(sk) : k_full(sk), (j / T::NSK) & 1, p.status))) break;
-          if (j > 0 && !(ok = mbar_wait_sleep(s_free, (j - 1) & 1, p.status))) break;
-          tc_fence_after();
-          // descriptors differ only in the start-address field (address >> 4 in the low bits, all
-          // addresses below 256 KB): the base descriptors plus offsets
-          const uint64_t kd0 = qd0 + ((T::K_OFF - T::Q_OFF + sk * T::TILE) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = ((kk >> 2) * T::HALF + (kk & 3) * 32) >> 4;
-            tc_mma_bf16(tmem_s, qd0 + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(s_full);
-          tc_commit(k_empty(sk));
-        }
-        if (j > 0) {
-          const int jj = j - 1, sv = jj % T::NSV;
-          const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
-          // the V tile (bf16: landed; fp8: widened)
-          if (!(ok = mbar_wait_sleep(F8 ? v_ready(sv) : v_full(sv), (jj / T::NSV) & 1, p.status))) break;
-          for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(j-1) . V_h(j-1)
-            if (!(ok = mbar_wait_sleep(p_full(h), jj & 1, p.status))) break;
+      int g = 0, ku = 0;  // tiles whose S was issued; units
+      bool ok = true;
+      for (int k = 0; ok && k < n_units; ++k) {
+        const MqUnit U = unit_at(k);
+        if (U.kind != kRun) continue;
+        if (!(ok = mbar_wait_sleep(F8 ? q_ready : q_full, ku & 1, p.status))) break;
+        // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1); tile j is tile g0 + j of the CTA
+        const int g0 = g;
+        for (int j = 0; ok && j <= U.nt; ++j) {
+          if (j < U.nt) {
+            const int gj = g0 + j, sk = gj % T::NSK;
+            if (!(ok = mbar_wait_sleep(F8 ? k_ready(sk) : k_full(sk), (gj / T::NSK) & 1, p.status))) break;
+            if (gj > 0 && !(ok = mbar_wait_sleep(s_free, (gj - 1) & 1, p.status))) break;
             tc_fence_after();
+            // descriptors differ only in the start-address field (address >> 4 in the low bits, all
+            // addresses below 256 KB): the base descriptors plus offsets
+            const uint64_t kd0 = qd0 + ((T::K_OFF - T::Q_OFF + sk * T::TILE) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
-              const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
-              tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-              if constexpr (!F8 && !T::STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = ((kk >> 2) * T::HALF + (kk & 3) * 32) >> 4;
+              tc_mma_bf16(tmem_s, qd0 + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
             }
-            tc_commit(pv_done(h));
+            tc_commit(s_full);
+            tc_commit(k_empty(sk));
+            if (j == U.nt - 1) tc_commit(q_empty);  // the unit's S MMAs are its only readers of Q
+            ++g;
           }
-          if (!ok) break;
-          tc_commit(v_empty(sv));
+          if (j > 0) {
+            const int jj = j - 1, gjj = g0 + jj, sv = gjj % T::NSV;
+            const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
+            // the V tile (bf16: landed; fp8: widened)
+            if (!(ok = mbar_wait_sleep(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status))) break;
+            // the unit's first P . V overwrites O: the previous unit's epilogue must have read it
+            if (jj == 0 && ku > 0 && !(ok = mbar_wait_sleep(o_free, (ku - 1) & 1, p.status))) break;
+            for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
+              if (!(ok = mbar_wait_sleep(p_full(h), gjj & 1, p.status))) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
+                const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
+                tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (!F8) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+              }
+              tc_commit(pv_done(h));
+            }
+            if (!ok) break;
+            tc_commit(v_empty(sv));
+          }
         }
+        ++ku;
       }
       // drain (bounded): no MMA may still read shared memory or write TMEM at exit
       tc_commit(mma_done);
@@ -548,294 +555,304 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, ROWS>::THREADS, 1)
     }
   } else if (warp < 8) {  // ---------------- softmax warps 0-7 --------------------------------------
     const int quarter = warp & 3, h = warp >> 2;  // TMEM lane quarter, token half of each tile
-    const int tl = 32 * quarter + lane;           // this thread's TMEM lane
-    // its query row; stacked: lanes 64-127 repeat rows 0-63 and write the residual part of P
-    const bool lo_part = T::STACK && quarter >= 2;
-    const int r = T::STACK ? tl & 63 : tl;
-    const int row = qt * T::ROWS + r;
-    const bool valid = row < rows_total;
-    // an invalid row (its output is never written) sees what the CTA's last row sees, so that it
-    // takes the same path as its warp's valid rows (a row that saw nothing would take the masking
-    // path alone and hold the warp on it every tile); its P only feeds its own accumulator row
-    const int pos = base_pos + (valid ? row : row_last) / G;
+    const int r = 32 * quarter + lane;            // this thread's row of a unit (TMEM lane)
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float qk = p.q_scale;
-    float m = -INFINITY, l = 0.f;  // this half's running reference max (log2 units) and row sum
     // After a timed-out wait the warp stops waiting (every later wait fails at
-    // once) but still runs every iteration, so the two warps of a pair meet at
-    // the epilogue's named barrier; the status bit reports the failure.
+    // once) but still runs every unit and iteration, so the two warps of a pair
+    // meet at the epilogue's named barriers; the status bit reports the failure.
     bool ok = true;
     auto wait = [&](uint32_t bar, uint32_t parity) {
       if (ok) ok = warp_wait_bounded(bar, parity, p.status);
       return ok;
     };
-    if constexpr (F8) {  // this thread's Q row half to fp16, in place (exact for |q| in [2^-14, 65504])
-      wait(q_full, 0);
-      uint4* qrow = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + r * 128);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w = qrow[c];
-        qrow[c] = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
+    int g = 0, ku = 0;  // tiles consumed; units
+    for (int k = 0; k < n_units; ++k) {
+      const MqUnit U = unit_at(k);
+      if (U.kind == kBadQuery) {
+        if (threadIdx.x == 0) set_status(p.status, PKV_STATUS_BAD_QUERY_LOC);
+        continue;
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_ready);
-    }
-    // bf16 caches: V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed:
-    // 0 * NaN would poison O.  The 64 rows of this half: thread (quarter, lane) takes row
-    // 16 quarter + lane / 2, dims half lane & 1.  (fp8 caches: the V producer zeroed them.)
-    auto zero_v_rows = [&](int j, bool bad) {
-      wait(v_full(j % T::NSV), (j / T::NSV) & 1);
-      const int vr = 64 * h + 16 * quarter + (lane >> 1);
-      const int t = tok_begin + j * T::TOK + vr;
-      if (t >= tok_end || (bad && block_id((t - tok_begin) / BS) < 0)) {
-        uint8_t* vrow = data + T::V_OFF + (j % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+      if (U.kind == kZero) {  // nothing to attend: zero rows
+        if (warp < 4) {
+          const int row = U.qt * T::ROWS + r;
+          if (row < U.rows_total) {
+            const int64_t orow = static_cast<int64_t>(U.q0 + row / G) * Hq + U.hk * G + row % G;
+            for (int d = 0; d < D; d += 8)
+              *reinterpret_cast<uint4*>(out + orow * D + d) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
       }
-      fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
-    };
-    // bit k set: block k of the half tile starting at token t0 has a bad id (t0 - tok_begin is a
-    // multiple of 64, so the half tile holds 64 / BS whole blocks)
-    auto half_tile_bad = [&](int t0) {
-      unsigned bad = 0u;
-      if (any_bad) {
-        const int i0 = (t0 - tok_begin) / BS;
-        for (int k = 0; k < 64 / BS && i0 + k < nb; ++k)
-          if (block_id(i0 + k) < 0) bad |= 1u << k;
-      }
-      return bad;
-    };
-    // A warp whose 32 rows all lie past the CTA's query rows (grouped verification uses 40 of 128)
-    // computes nothing: it keeps every barrier step -- including the wait for the previous tile's
-    // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
-    // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
-    // output rows nobody writes.
-    if constexpr (T::STACK) {  // Q rows 0-63 (both 64-dim halves) copied below themselves, same swizzle phase
-      if (lo_part) {
-        wait(q_full, 0);
-        // the two warps of half h copy the 64-dim half h: 64 threads x 8 x 16 bytes
-        const int i = 32 * (quarter - 2) + lane;
-        const uint4* src = reinterpret_cast<const uint4*>(data + T::Q_OFF + h * T::HALF);
-        uint4* dst = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + 64 * 128);
+      if (U.kind != kRun) continue;
+      const int tok_begin = U.tok_begin, tok_end = U.tok_end, nt = U.nt, nb = U.nb;
+      const int row = U.qt * T::ROWS + r;
+      const bool valid = row < U.rows_total;
+      // an invalid row (its output is never written) sees what the unit's last row sees, so that it
+      // takes the same path as its warp's valid rows (a row that saw nothing would take the masking
+      // path alone and hold the warp on it every tile); its P only feeds its own accumulator row
+      const int pos = U.base_pos + (valid ? row : U.row_last) / G;
+      float m = -INFINITY, l = 0.f;  // this half's running reference max (log2 units) and row sum
+      if constexpr (F8) {  // this thread's Q row half to fp16, in place (exact for |q| in [2^-14, 65504])
+        wait(q_full, ku & 1);
+        uint4* qrow = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + r * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) dst[i + 64 * c] = src[i + 64 * c];
-        fence_proxy_async_smem();  // these writes before the MMA's reads (async proxy)
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = qrow[c];
+          qrow[c] = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
+        }
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
       }
-    }
-    if (qt * T::ROWS + (T::STACK ? 32 * (quarter & 1) : 32 * quarter) >= rows_total) {
+      // blocks of the unit with a bad id (reported by the K producer): masked, their V rows zeroed
+      bool any_bad = false;
+      for (int i = lane; i < nb; i += 32) any_bad |= block_id(U, i) < 0;
+      any_bad = __any_sync(kFullMask, any_bad);
+      // bf16 caches: V rows of tokens that must not contribute (past tok_end, bad blocks) are zeroed:
+      // 0 * NaN would poison O.  The 64 rows of this half: thread (quarter, lane) takes row
+      // 16 quarter + lane / 2, dims half lane & 1.  (fp8 caches: the widening warp zeroed them.)
+      auto zero_v_rows = [&](int j, bool bad) {
+        const int gj = g + j;
+        wait(v_full(gj % T::NSV), (gj / T::NSV) & 1);
+        const int vr = 64 * h + 16 * quarter + (lane >> 1);
+        const int t = tok_begin + j * T::TOK + vr;
+        if (t >= tok_end || (bad && block_id(U, (t - tok_begin) / BS) < 0)) {
+          uint8_t* vrow = data + T::V_OFF + (gj % T::NSV) * T::TILE + (lane & 1) * T::HALF + vr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // the zeroed rows before the MMA reads them
+      };
+      // bit k set: block k of the half tile starting at token t0 has a bad id (t0 - tok_begin is a
+      // multiple of 64, so the half tile holds 64 / BS whole blocks)
+      auto half_tile_bad = [&](int t0) {
+        unsigned bad = 0u;
+        if (any_bad) {
+          const int i0 = (t0 - tok_begin) / BS;
+          for (int kb = 0; kb < 64 / BS && i0 + kb < nb; ++kb)
+            if (block_id(U, i0 + kb) < 0) bad |= 1u << kb;
+        }
+        return bad;
+      };
+      // A warp whose 32 rows all lie past the unit's query rows (grouped verification uses 40 of 128)
+      // computes nothing: it keeps every barrier step -- including the wait for the previous tile's
+      // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
+      // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
+      // output rows nobody writes.
+      if (U.qt * T::ROWS + 32 * quarter >= U.rows_total) {
+        for (int j = 0; j < nt; ++j) {
+          const int t0 = tok_begin + j * T::TOK + 64 * h;
+          wait(s_full, (g + j) & 1);
+          tc_fence_after();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+          const bool bad = half_tile_bad(t0) != 0u;
+          if (j > 0) wait(pv_done(h), (g + j - 1) & 1);
+          if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full(h));
+        }
+      } else
       for (int j = 0; j < nt; ++j) {
-        const int t0 = tok_begin + j * T::TOK + 64 * h;
-        wait(s_full, j & 1);
+        const int t0 = tok_begin + j * T::TOK + 64 * h;  // first token of this half of the tile
+        wait(s_full, (g + j) & 1);
         tc_fence_after();
+        float sv[64];
+        {
+          uint32_t u[2][32];
+          tmem_ld32(tmem_s + lane_off + 64 * h, u[0]);
+          tmem_ld32(tmem_s + lane_off + 64 * h + 32, u[1]);
+          tmem_ld_wait(u[0]);
+          tmem_ld_wait(u[1]);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[e] = __uint_as_float(u[0][e]);
+            sv[32 + e] = __uint_as_float(u[1][e]);
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        const bool bad = half_tile_bad(t0) != 0u;
-        if (j > 0) wait(pv_done(h), (j - 1) & 1);
-        if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
+
+        // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
+        const unsigned bad_blocks = half_tile_bad(t0);
+        const bool bad = bad_blocks != 0u;
+        const bool ragged = t0 + 64 > tok_end;  // tokens at or past tok_end in this half tile
+        // row max of the raw scores (q_scale > 0 commutes with the max); masked scores -> -inf.
+        // Eight independent partial maxima / sums: instruction-level parallelism hides latency.
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+        if (t0 + 63 > pos || ragged || bad) {
+          if (bad) {  // scores of blocks that were not loaded (stale tiles) never reach the max
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if ((bad_blocks >> (c / BS)) & 1u) sv[c] = -INFINITY;
+          }
+          // column c is visible iff c <= last (causal position and the end of what is loaded)
+          const int last = min(pos, tok_end - 1) - t0;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            sv[c] = c > last ? -INFINITY : sv[c];
+            mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) mx8[(c >> 1) & 7] = fmax3f(mx8[(c >> 1) & 7], sv[c], sv[c + 1]);
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qk;
+        // reference max: move it (and rescale) only when a score passes it by more than 8 (log2 units)
+        float alpha = 1.f;
+        if (mx > m + 8.f) {
+          alpha = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+          l *= alpha;
+          m = mx;
+        }
+        const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
+        // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add, and at once the
+        // row's half of P as packed pairs (tokens 2k, 2k+1 in word k).  bf16 caches: a high part (the
+        // top 16 bits of the fp32 value: truncation) and the residual (exact in fp32, then truncated to
+        // its top 16 bits), ~16 significant bits per probability, with integer ops only.  fp8 caches:
+        // one fp16 value (round to nearest; p <= 2^8).  One loop, so the special-function unit (ex2)
+        // and the integer / FMA pipes (packing) work side by side; the stores to TMEM wait below.
+        const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
+        float2 sum4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
+        uint32_t ph[32], plo[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
+          const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
+          sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
+          if constexpr (F8) {
+            const __half2 hp = __floats2half2_rn(a, bb);  // token 2k in the low half
+            ph[k] = *reinterpret_cast<const uint32_t*>(&hp);
+            plo[k] = 0u;
+          } else {
+            const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
+            // residual = value - its truncation (the negated truncation is one logic op)
+            const float2 rr = __fadd2_rn(make_float2(a, bb),
+                                         make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
+                                                     __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
+            ph[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
+            plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+          }
+        }
+        const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
+        l += s2.x + s2.y;
+        // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
+        if (j > 0) {
+          wait(pv_done(h), (g + j - 1) & 1);
+          tc_fence_after();
+          if (__any_sync(kFullMask, alpha != 1.f)) {  // a moved reference: rescale this row of O_h
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t u[32];
+              const uint32_t oa = tmem_o(h) + lane_off + 32 * c;
+              tmem_ld32(oa, u);
+              tmem_ld_wait(u);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+              tmem_st32(oa, u);
+            }
+          }
+        }
+        if (!F8 && (ragged || bad)) zero_v_rows(j, bad);
+        // this half of row r of P into TMEM lane r
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pw[16], lw[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            pw[k] = ph[16 * c + k];
+            lw[k] = plo[16 * c + k];
+          }
+          tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
+          if constexpr (!F8) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
+        }
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full(h));
       }
-    } else
-    for (int j = 0; j < nt; ++j) {
-      const int t0 = tok_begin + j * T::TOK + 64 * h;  // first token of this half of the tile
-      wait(s_full, j & 1);
+      g += nt;
+      wait(pv_done(h), (g - 1) & 1);
       tc_fence_after();
-      float sv[64];
+      // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 ---
+      // (m, l) of this half go to the partner warp through TMEM columns of P_h (its P . V is done)
       {
-        uint32_t u[2][32];
-        tmem_ld32(tmem_s + lane_off + 64 * h, u[0]);
-        tmem_ld32(tmem_s + lane_off + 64 * h + 32, u[1]);
-        tmem_ld_wait(u[0]);
-        tmem_ld_wait(u[1]);
+        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          sv[e] = __uint_as_float(u[0][e]);
-          sv[32 + e] = __uint_as_float(u[1][e]);
-        }
+        for (int c = 0; c < 16; ++c) w[c] = 0u;
+        w[0] = __float_as_uint(m);
+        w[1] = __float_as_uint(l);
+        tmem_st16(tmem_p(h) + lane_off, w);
+        tmem_st_wait();
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-
-      // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
-      const unsigned bad_blocks = half_tile_bad(t0);
-      const bool bad = bad_blocks != 0u;
-      const bool ragged = t0 + 64 > tok_end;  // tokens at or past tok_end in this half tile
-      // row max of the raw scores (q_scale > 0 commutes with the max); masked scores -> -inf.
-      // Eight independent partial maxima / sums: instruction-level parallelism hides latency.
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
-      if (t0 + 63 > pos || ragged || bad) {
-        if (bad) {  // scores of blocks that were not loaded (stale tiles) never reach the max
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if ((bad_blocks >> (c / BS)) & 1u) sv[c] = -INFINITY;
-        }
-        // column c is visible iff c <= last (causal position and the end of what is loaded)
-        const int last = min(pos, tok_end - 1) - t0;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          sv[c] = c > last ? -INFINITY : sv[c];
-          mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) mx8[(c >> 1) & 7] = fmax3f(mx8[(c >> 1) & 7], sv[c], sv[c + 1]);
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");  // the two warps of this lane quarter
+      tc_fence_after();
+      float m_o, l_o;
+      {
+        uint32_t x[32];
+        tmem_ld32(tmem_p(h ^ 1) + lane_off, x);
+        tmem_ld_wait(x);
+        m_o = __uint_as_float(x[0]);
+        l_o = __uint_as_float(x[1]);
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qk;
-      // reference max: move it (and rescale) only when a score passes it by more than 8 (log2 units)
-      float alpha = 1.f;
-      if (mx > m + 8.f) {
-        alpha = m == -INFINITY ? 0.f : fast_exp2(m - mx);
-        l *= alpha;
-        m = mx;
-      }
-      const float neg_m = m == -INFINITY ? 0.f : -m;  // m = -inf: every score is -inf, p = 0
-      // p = 2^(s * q_scale - m), pairs of values through the packed fp32x2 FMA / add, and at once the
-      // row's half of P as packed pairs (tokens 2k, 2k+1 in word k).  bf16 caches: a high part (the
-      // top 16 bits of the fp32 value: truncation) and the residual (exact in fp32, then truncated to
-      // its top 16 bits), ~16 significant bits per probability, with integer ops only.  fp8 caches:
-      // one fp16 value (round to nearest; p <= 2^8).  One loop, so the special-function unit (ex2)
-      // and the integer / FMA pipes (packing) work side by side; the stores to TMEM wait below.
-      const float2 qk2 = make_float2(qk, qk), nm2 = make_float2(neg_m, neg_m);
-      float2 sum4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
-      uint32_t ph[32], plo[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
-        const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
-        sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
-        if constexpr (F8) {
-          const __half2 hp = __floats2half2_rn(a, bb);  // token 2k in the low half
-          ph[k] = *reinterpret_cast<const uint32_t*>(&hp);
-          plo[k] = 0u;
-        } else {
-          const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
-          // residual = value - its truncation (the negated truncation is one logic op)
-          const float2 rr = __fadd2_rn(make_float2(a, bb),
-                                       make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
-                                                   __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
-          ph[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
-          plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
-        }
-      }
-      const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
-      l += s2.x + s2.y;
-      // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
-      if (j > 0) {
-        wait(pv_done(h), (j - 1) & 1);
-        tc_fence_after();
-        if (__any_sync(kFullMask, alpha != 1.f)) {  // a moved reference: rescale this row of O_h
+      const float M = fmaxf(l > 0.f ? m : -INFINITY, l_o > 0.f ? m_o : -INFINITY);
+      const float w_self = l > 0.f ? fast_exp2(m - M) : 0.f, w_oth = l_o > 0.f ? fast_exp2(m_o - M) : 0.f;
+      const float lsum = l * w_self + l_o * w_oth;
+      const float inv = lsum > 0.f ? p.out_scale / lsum : 0.f;
+      const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
+      const int64_t orow = static_cast<int64_t>(U.q0 + row / G) * Hq + U.hk * G + row % G;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t u[32];
-            const uint32_t oa = tmem_o(h) + lane_off + 32 * c;
-            tmem_ld32(oa, u);
-            tmem_ld_wait(u);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(oa, u);
-          }
-        }
-      }
-      if (!F8 && (ragged || bad)) zero_v_rows(j, bad);
-      // this half of row r of P into TMEM lane r (stacked: the high part in lanes 0-63, the residual
-      // in lanes 64-127, both in P_h's columns)
-#pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t pw[16], lw[16];
+        const int d0 = 64 * h + 32 * c;
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tmem_o(0) + lane_off + d0, u0);
+        tmem_ld32(tmem_o(1) + lane_off + d0, u1);
+        tmem_ld_wait(u0);
+        tmem_ld_wait(u1);
+        if (!valid || !ok) continue;
+        float o[32];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          pw[k] = lo_part ? plo[16 * c + k] : ph[16 * c + k];
-          lw[k] = plo[16 * c + k];
-        }
-        tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
-        if constexpr (!F8 && !T::STACK) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(h));
-    }
-    wait(pv_done(h), (nt - 1) & 1);
-    tc_fence_after();
-    // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 -----
-    float* xch = reinterpret_cast<float*>(data + T::XCH_OFF);  // [m_0, m_1, l_0, l_1][TMEM lane]
-    xch[h * 128 + tl] = m;
-    xch[(2 + h) * 128 + tl] = l;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");  // the two warps of this lane quarter
-    const float m_o = xch[(h ^ 1) * 128 + tl], l_o = xch[(2 + (h ^ 1)) * 128 + tl];
-    const float M = fmaxf(l > 0.f ? m : -INFINITY, l_o > 0.f ? m_o : -INFINITY);
-    const float w_self = l > 0.f ? fast_exp2(m - M) : 0.f, w_oth = l_o > 0.f ? fast_exp2(m_o - M) : 0.f;
-    const float lsum = l * w_self + l_o * w_oth;
-    const float inv = lsum > 0.f ? p.out_scale / lsum : 0.f;
-    const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
-    const int64_t orow = static_cast<int64_t>(q0 + row / G) * Hq + hk * G + row % G;
-    // stacked rows: the residual's share of this row's output (accumulator rows 64-127) goes from
-    // the warp of lanes 64-127 to the warp of the same row and half through the free K ring
-    float* xo = reinterpret_cast<float*>(data + T::K_OFF);  // [64 rows][128 dims]
-    const int pair_bar = 5 + 2 * (quarter & 1) + h;      // named barrier of the two warps of this row
-    if (T::STACK && !lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      const int d0 = 64 * h + 32 * c;
-      uint32_t u0[32], u1[32];
-      tmem_ld32(tmem_o(0) + lane_off + d0, u0);
-      tmem_ld32(tmem_o(1) + lane_off + d0, u1);
-      tmem_ld_wait(u0);
-      tmem_ld_wait(u1);
-      if (!valid || !ok) continue;
-      float o[32];
+        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u0[e]) * w0 + __uint_as_float(u1[e]) * w1;
+        if (U.nparts == 1) {
+          __nv_bfloat16* dst = out + orow * D + d0;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u0[e]) * w0 + __uint_as_float(u1[e]) * w1;
-      if constexpr (T::STACK) {
-        float4* x4 = reinterpret_cast<float4*>(xo + r * 128 + d0);
-        if (lo_part) {
+          for (int e = 0; e < 32; e += 8) {
+            uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) x4[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
-          continue;
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 v = x4[e / 4];
-          o[e] += v.x;
-          o[e + 1] += v.y;
-          o[e + 2] += v.z;
-          o[e + 3] += v.w;
-        }
-      }
-      if (nparts == 1) {
-        __nv_bfloat16* dst = out + orow * D + d0;
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            __nv_bfloat162 hv = __floats2bfloat162_rn(o[e + 2 * k], o[e + 2 * k + 1]);
-            w[k] = *reinterpret_cast<uint32_t*>(&hv);
+            for (int kq = 0; kq < 4; ++kq) {
+              __nv_bfloat162 hv = __floats2bfloat162_rn(o[e + 2 * kq], o[e + 2 * kq + 1]);
+              w[kq] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      } else {
-        float* dst = p.ws_o + (orow * p.max_partitions + part) * D + d0;
+        } else {
+          float* dst = p.ws_o + (orow * p.max_partitions + U.part) * D + d0;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        }
       }
-    }
-    if (T::STACK && lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-    if (valid && ok && nparts > 1 && h == 0 && !lo_part) {
-      const int64_t srow = orow * p.max_partitions + part;
-      p.ws_ml[srow * 2] = lsum > 0.f ? M * kLn2 : 0.f;
-      p.ws_ml[srow * 2 + 1] = lsum;
+      if (valid && ok && U.nparts > 1 && h == 0) {
+        const int64_t srow = orow * p.max_partitions + U.part;
+        p.ws_ml[srow * 2] = lsum > 0.f ? M * kLn2 : 0.f;
+        p.ws_ml[srow * 2 + 1] = lsum;
+      }
+      // both warps of the pair have read the exchanged (m, l) before either writes the next unit's P,
+      // and every softmax warp has read O before the next unit's first P . V overwrites it
+      tc_fence_before();
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+      if (lane == 0) mbar_arrive(o_free);
+      ++ku;
     }
   }
   tc_fence_before();
