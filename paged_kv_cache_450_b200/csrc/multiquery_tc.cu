@@ -15,11 +15,11 @@ static int sm_count_of_device() {
   return n;
 }
 
-template <int BS, int G, bool F8>
-static cudaError_t launch_mq_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                                const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
-  using T = MqTcTraits<BS, F8>;
-  auto kern = paged_multiquery_tc_kernel<BS, G, F8>;
+template <int BS, int G, bool F8, bool STACK>
+static cudaError_t launch_mq_tc_kind(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                     const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
+  using T = MqTcTraits<BS, F8, STACK>;
+  auto kern = paged_multiquery_tc_kernel<BS, G, F8, STACK>;
   const size_t smem = T::smem_bytes(p.partition_blocks);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -29,6 +29,16 @@ static cudaError_t launch_mq_tc(const CUtensorMap& qmap, const CUtensorMap& kmap
   e = launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(T::THREADS), smem, st, qmap, kmap, vmap, p);
   if (e != cudaSuccess || !reduce) return e;
   return launch_multiquery_reduce(p, st);
+}
+
+// bf16 caches with at most 64 query rows per (sequence, KV head): the stacked tile
+template <int BS, int G, bool F8>
+static cudaError_t launch_mq_tc(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                const MultiQueryParams& p, int n_qtiles, bool reduce, cudaStream_t st) {
+  if constexpr (!F8) {
+    if (p.max_q_len * G <= 64) return launch_mq_tc_kind<BS, G, F8, true>(qmap, kmap, vmap, p, 1, reduce, st);
+  }
+  return launch_mq_tc_kind<BS, G, F8, false>(qmap, kmap, vmap, p, n_qtiles, reduce, st);
 }
 
 template <int BS, bool F8>

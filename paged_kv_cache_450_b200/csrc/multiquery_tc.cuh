@@ -76,10 +76,22 @@
 
 namespace pkv {
 
-template <int BS, bool F8 = false>
+// STACK (bf16 caches, at most 64 query rows per (sequence, KV head), as in
+// grouped verification: 5 queries x 8 heads = 40): MMA rows 64-127 repeat rows
+// 0-63 (the softmax warps of TMEM lanes 64-127 copy the Q tile's first 64 rows
+// below them), so S holds every score twice; the warps of lanes 0-63 write P's
+// bf16 high part and those of lanes 64-127 its residual for the same rows, and
+// each P . V k-step is ONE M = 128 MMA whose accumulator rows 64-127 collect the
+// residual's share -- 16 MMAs per tile instead of 24 for the single issuing
+// thread.  The epilogue adds the residual's share back through the Q tile, so
+// the next unit's Q loads once the epilogue is done (o_free) rather than once
+// the unit's S MMAs are (q_empty).
+template <int BS, bool F8 = false, bool STACK_ = false>
 struct MqTcTraits {
   static constexpr int D = 128;
-  static constexpr int ROWS = 128;           // query rows per unit (MMA M)
+  static constexpr bool STACK = STACK_;
+  static_assert(!(STACK && F8), "stacked rows: bf16 caches");
+  static constexpr int ROWS = STACK ? 64 : 128;  // query rows per unit
   static constexpr int TOK = 128;            // tokens per KV tile
   static constexpr int BPT = TOK / BS;       // blocks per KV tile
   static constexpr int HALF = 128 * 128;     // 128 rows x 128 bytes (64 bf16 / fp16)
@@ -96,7 +108,7 @@ struct MqTcTraits {
   // mbarriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free,
   // p_full[2], pv_done[2] (one per token half), o_free, mma_done; fp8 caches add q_ready, k_ready[NSK],
   // v_ready[NSV]
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : 0);
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   // the sequence of each of the CTA's first MAX_UNITS units (longest-first rank -> sequence)
   static constexpr int MAX_UNITS = 64;
@@ -308,11 +320,11 @@ __device__ __forceinline__ void widen_e4m3_tile_in_place(uint8_t* stage, int lan
   fence_proxy_async_smem();
 }
 
-template <int BS, int G, bool F8>
-__global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
+template <int BS, int G, bool F8, bool STACK = false>
+__global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     paged_multiquery_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap, const MultiQueryParams p) {
-  using T = MqTcTraits<BS, F8>;
+  using T = MqTcTraits<BS, F8, STACK>;
   constexpr int D = T::D;
   constexpr int QPT = T::ROWS / G;  // queries per unit
   pdl_wait_and_release();
@@ -394,6 +406,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
       for (int s = 0; s < T::NSV; ++s) mbar_init(v_ready(s), 1);
     }
+    if constexpr (STACK) mbar_init(q_ready, 4);
     fence_barrier_init();
   }
   __syncthreads();
@@ -422,8 +435,9 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     for (int k = 0; ok && k < n_units; ++k) {
       const MqUnit U = unit_at(k);
       if (U.kind != kRun) continue;
-      if (is_k) {  // Q of this unit once the previous unit's S MMAs are done with the Q tile
-        if (ku > 0 && !(ok = warp_wait_bounded(q_empty, (ku - 1) & 1, p.status))) break;
+      if (is_k) {  // Q of this unit once the previous unit is done with the Q tile (its S MMAs; stacked:
+                   // its epilogue too)
+        if (ku > 0 && !(ok = warp_wait_bounded(STACK ? o_free : q_empty, (ku - 1) & 1, p.status))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full, T::TILE);
           tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, U.hk * G, U.q0 + U.qt * QPT);
@@ -503,7 +517,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       for (int k = 0; ok && k < n_units; ++k) {
         const MqUnit U = unit_at(k);
         if (U.kind != kRun) continue;
-        if (!(ok = mbar_wait_sleep(F8 ? q_ready : q_full, ku & 1, p.status))) break;
+        if (!(ok = mbar_wait_sleep(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
         // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1); tile j is tile g0 + j of the CTA
         const int g0 = g;
         for (int j = 0; ok && j <= U.nt; ++j) {
@@ -539,7 +553,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
               for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
                 const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
                 tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                if constexpr (!F8) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+                if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
               }
               tc_commit(pv_done(h));
             }
@@ -555,7 +569,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
     }
   } else if (warp < 8) {  // ---------------- softmax warps 0-7 --------------------------------------
     const int quarter = warp & 3, h = warp >> 2;  // TMEM lane quarter, token half of each tile
-    const int r = 32 * quarter + lane;            // this thread's row of a unit (TMEM lane)
+    const int tl = 32 * quarter + lane;           // this thread's TMEM lane
+    // its row of a unit; stacked: lanes 64-127 repeat rows 0-63 and write the residual part of P
+    const bool lo_part = STACK && quarter >= 2;
+    const int r = STACK ? (tl & 63) : tl;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float qk = p.q_scale;
     // After a timed-out wait the warp stops waiting (every later wait fails at
@@ -575,7 +592,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       }
       if (U.kind == kZero) {  // nothing to attend: zero rows
         if (warp < 4) {
-          const int row = U.qt * T::ROWS + r;
+          const int row = U.qt * T::ROWS + tl;
           if (row < U.rows_total) {
             const int64_t orow = static_cast<int64_t>(U.q0 + row / G) * Hq + U.hk * G + row % G;
             for (int d = 0; d < D; d += 8)
@@ -604,6 +621,19 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
+      }
+      if constexpr (STACK) {  // Q rows 0-63 (this warp's 64-dim half) copied below themselves, same phase
+        if (lo_part) {
+          wait(q_full, ku & 1);
+          const int i = 32 * (quarter - 2) + lane;  // 64 threads x 8 x 16 bytes of the half
+          const uint4* src = reinterpret_cast<const uint4*>(data + T::Q_OFF + h * T::HALF);
+          uint4* dst = reinterpret_cast<uint4*>(data + T::Q_OFF + h * T::HALF + 64 * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) dst[i + 64 * c] = src[i + 64 * c];
+          fence_proxy_async_smem();  // these writes before the MMA's reads (async proxy)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_ready);
+        }
       }
       // blocks of the unit with a bad id (reported by the K producer): masked, their V rows zeroed
       bool any_bad = false;
@@ -640,7 +670,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
       // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
       // output rows nobody writes.
-      if (U.qt * T::ROWS + 32 * quarter >= U.rows_total) {
+      if (U.qt * T::ROWS + 32 * (STACK ? (quarter & 1) : quarter) >= U.rows_total) {
         for (int j = 0; j < nt; ++j) {
           const int t0 = tok_begin + j * T::TOK + 64 * h;
           wait(s_full, (g + j) & 1);
@@ -769,11 +799,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
           uint32_t pw[16], lw[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            pw[k] = ph[16 * c + k];
+            pw[k] = lo_part ? plo[16 * c + k] : ph[16 * c + k];
             lw[k] = plo[16 * c + k];
           }
           tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
-          if constexpr (!F8) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
+          if constexpr (!F8 && !STACK) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -811,6 +841,12 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
       const float inv = lsum > 0.f ? p.out_scale / lsum : 0.f;
       const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
       const int64_t orow = static_cast<int64_t>(U.q0 + row / G) * Hq + U.hk * G + row % G;
+      // stacked: the residual's share of this row's output (accumulator rows 64-127) goes from the warp
+      // of lanes 64-127 to the warp of the same row and half through the Q tile (free: the next unit's
+      // Q waits for o_free)
+      float* xo = reinterpret_cast<float*>(data + T::Q_OFF);  // [64 rows][128 dims]
+      const int pair_bar = 5 + 2 * (quarter & 1) + h;       // named barrier of the two warps of this row
+      if (STACK && !lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         const int d0 = 64 * h + 32 * c;
@@ -823,6 +859,22 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
         float o[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u0[e]) * w0 + __uint_as_float(u1[e]) * w1;
+        if constexpr (STACK) {
+          float4* x4 = reinterpret_cast<float4*>(xo + r * 128 + d0);
+          if (lo_part) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) x4[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            continue;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 v = x4[e / 4];
+            o[e] += v.x;
+            o[e + 1] += v.y;
+            o[e + 2] += v.z;
+            o[e + 3] += v.w;
+          }
+        }
         if (U.nparts == 1) {
           __nv_bfloat16* dst = out + orow * D + d0;
 #pragma unroll
@@ -842,7 +894,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8>::THREADS, 1)
             *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
       }
-      if (valid && ok && U.nparts > 1 && h == 0) {
+      if (STACK && lo_part) {
+        fence_proxy_async_smem();  // these writes before the next unit's Q load (async proxy)
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      }
+      if (valid && ok && U.nparts > 1 && h == 0 && !lo_part) {
         const int64_t srow = orow * p.max_partitions + U.part;
         p.ws_ml[srow * 2] = lsum > 0.f ? M * kLn2 : 0.f;
         p.ws_ml[srow * 2 + 1] = lsum;
