@@ -445,9 +445,9 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         }
         ++ku;
       }
+      int id = tile_block(U, 0);  // the block ids of tile j + 1 are read while tile j is issued
       for (int j = 0; j < U.nt; ++j, ++g) {
         const int s = g % ns, use = g / ns;
-        const int id = tile_block(U, j);  // (its latency overlaps the wait)
         if (use > 0 && !(ok = warp_wait_bounded(is_k ? k_empty(s) : v_empty(s), (use - 1) & 1, p.status))) break;
         const unsigned vm = __ballot_sync(kFullMask, id >= 0);
         if (is_k && lane == 0 && __popc(vm) < min(T::BPT, U.nb - j * T::BPT))
@@ -467,6 +467,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             tma_load_4d(dst + T::HALF, map, full, 64, U.hk, 0, id, policy);
           }
         }
+        id = j + 1 < U.nt ? tile_block(U, j + 1) : -1;
       }
     }
     // drain (bounded): the copies of the last stages (and the last Q) have landed before exit
