@@ -457,6 +457,9 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   auto slot = [&](int i) { return i < n0 ? i : s1 + (i - n0); };
   const float* ml = p.ws_ml + row * p.max_partitions * 2;
   const float* o = p.ws_o + row * p.max_partitions * D;
+  // Partitions are taken 32 at a time: lane i loads (m, l) of partition c + i at once, the weights
+  // l e^{m - M} go to the other lanes by shuffle, and the partial outputs are read four at a time,
+  // so the loads of a row overlap instead of following one another.
   float M = -INFINITY;
   for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[2 * slot(i)]);
 #pragma unroll
@@ -465,15 +468,39 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
 #pragma unroll
   for (int e = 0; e < PVV; ++e) acc[e] = 0.f;
   float W = 0.f;
-  for (int k = 0; k < nparts; ++k) {
-    const int i = slot(k);
-    const float li = ml[2 * i + 1];
-    const float w = li > 0.f ? li * fast_exp2((ml[2 * i] - M) * kLog2e) : 0.f;
-    W += w;
-    const float* oi = o + static_cast<int64_t>(i) * D + lane * PVV;
+  for (int c = 0; c < nparts; c += 32) {
+    const int n = min(32, nparts - c);
+    float wl = 0.f;  // this lane's partition c + lane
+    if (lane < n) {
+      const int i = slot(c + lane);
+      const float li = ml[2 * i + 1];
+      wl = li > 0.f ? li * fast_exp2((ml[2 * i] - M) * kLog2e) : 0.f;
+    }
+    W += wl;
+    int k = 0;
+    for (; k + 4 <= n; k += 4) {
+      float w4[4], v[4][PVV];
 #pragma unroll
-    for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w, oi[e], acc[e]);
+      for (int q = 0; q < 4; ++q) {
+        w4[q] = __shfl_sync(kFullMask, wl, k + q);
+        const float* oi = o + static_cast<int64_t>(slot(c + k + q)) * D + lane * PVV;
+#pragma unroll
+        for (int e = 0; e < PVV; ++e) v[q][e] = oi[e];
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w4[q], v[q][e], acc[e]);
+    }
+    for (; k < n; ++k) {
+      const float w = __shfl_sync(kFullMask, wl, k);
+      const float* oi = o + static_cast<int64_t>(slot(c + k)) * D + lane * PVV;
+#pragma unroll
+      for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w, oi[e], acc[e]);
+    }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(kFullMask, W, off);
   TQ* out = static_cast<TQ*>(p.out) + row * D + lane * PVV;
 #pragma unroll
   for (int e = 0; e < PVV; ++e) out[e] = Elem<TQ>::from_float(W > 0.f ? acc[e] / W : 0.f);
