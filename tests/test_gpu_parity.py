@@ -603,6 +603,34 @@ def test_multiquery_full_size_sampled(name):
     _mq_check(mw, rows=rows, what=name)
 
 
+@pytest.mark.parametrize("case", ["rounds-ranked", "over-1024-sequences", "over-64-rounds"])
+def test_multiquery_persistent_many_units(case):
+    """The tcgen05 kernel's persistent CTAs over many units: about 8 units per CTA with the
+    longest-first ranking; more than 1024 sequences and more than 64 units per CTA, where units keep
+    the sequences' order; empty query sets and sequences whose rows span two 128-row units among
+    them.  Sampled rows against the oracle."""
+    rng = np.random.default_rng({"rounds-ranked": 31, "over-1024-sequences": 32, "over-64-rounds": 33}[case])
+    if case == "rounds-ranked":
+        B, hq, hkv = 300, 8, 2
+        q_lens = [int(x) if x > 3 else 0 for x in rng.integers(0, 41, B)]      # up to 160 rows: two units
+        ctxs = [int(max(q, c)) for q, c in zip(q_lens, rng.integers(50, 601, B))]
+    elif case == "over-1024-sequences":
+        B, hq, hkv = 1100, 4, 4
+        q_lens = [int(x) for x in rng.integers(17, 25, B)]                      # 17-24 rows: stacked tile
+        ctxs = [int(max(q, c)) for q, c in zip(q_lens, rng.integers(30, 201, B))]
+    else:
+        B, hq, hkv = 1000, 32, 16
+        q_lens = [int(x) for x in rng.integers(9, 11, B)]                       # 18-20 rows, 16000 units
+        ctxs = [int(max(q, c)) for q, c in zip(q_lens, rng.integers(20, 81, B))]
+    spec = W.DecodeSpec("mqpers", B, hq, hkv, 128, 16, torch.bfloat16, torch.bfloat16, ("list", tuple(ctxs)),
+                        ("slack", 1.1))
+    mw = W.make_multiquery_workload(spec, q_lens, seed=int(rng.integers(1 << 30)), device=DEV)
+    T = int(mw.query_start_loc[-1])
+    rows = np.unique(np.concatenate([rng.choice(T * hq, 600, replace=False), np.arange(hq),
+                                     T * hq - 1 - np.arange(hq)]))
+    _mq_check(mw, rows=rows, what=case)
+
+
 def test_multiquery_one_query_per_sequence_matches_decode():
     spec = W.LLAMA7B.with_(num_seqs=5, num_q_heads=16, num_kv_heads=2, ctx=("list", (1, 40, 300, 17, 1000)))
     mw = W.make_multiquery_workload(spec, (1,) * 5, seed=4, device=DEV)
