@@ -13,7 +13,9 @@
 //   O_h += P_h . V_h M = 128 rows, N = 128 dims,   K = 64 tokens (half h of the tile)
 //                    -> TMEM columns [128, 256) (h = 0) and [256, 384) (h = 1)
 // (Every MMA is as wide as the operands allow: the single issuing thread pays
-// per instruction, 80-125 cycles whatever M and N.)
+// ~64 cycles per instruction whatever M and N -- an N = 128 MMA executes in
+// ~81 -- and ~50-100 per barrier wait, fence or commit, so it waits on as few
+// barriers per tile as the data flow allows.)
 //
 // Persistent CTAs: one CTA per SM (the launch has min(units, SMs) CTAs) takes
 // one unit of every round of CTAs-many units of the unit list, which is ordered
@@ -41,9 +43,10 @@
 //              (the lanes its sub-partition may touch) and half h = w >> 2 of
 //              every KV tile's tokens.  The two halves are independent online
 //              softmaxes -- each with its own running max, row sum and
-//              accumulator O_h -- so the two warps of a sub-partition never
-//              wait for each other and their special-function (exp) and
-//              integer / FMA (P packing) phases interleave; they are merged
+//              accumulator O_h -- so the two warps of a sub-partition wait for
+//              each other only through the tile's P barrier, and their
+//              special-function (exp) and integer / FMA (P packing) phases
+//              interleave; they are merged
 //              once per unit, in the epilogue (the (m, l) exchange goes through
 //              TMEM columns of P, free by then).  Per tile a thread reads its 64
 //              scores from TMEM, applies the causal / context mask, keeps a
@@ -106,9 +109,9 @@ struct MqTcTraits {
   static constexpr int V_OFF = K_OFF + NSK * TILE;
   static constexpr int BAR_OFF = V_OFF + NSV * TILE;
   // mbarriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free,
-  // p_full[2], pv_done[2] (one per token half), o_free, mma_done; fp8 caches add q_ready, k_ready[NSK],
+  // p_full, pv_done (both token halves), o_free, mma_done; fp8 caches add q_ready, k_ready[NSK],
   // v_ready[NSV]
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 6 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   // the sequence of each of the CTA's first MAX_UNITS units (longest-first rank -> sequence)
   static constexpr int MAX_UNITS = 64;
@@ -362,11 +365,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
   auto v_empty = [&](int s) { return bar0 + 8 * (2 + 2 * T::NSK + T::NSV + s); };
   constexpr int B2 = 2 + 2 * T::NSK + 2 * T::NSV;
   const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1);
-  auto p_full = [&](int h) { return bar0 + 8 * (B2 + 2 + h); };
-  auto pv_done = [&](int h) { return bar0 + 8 * (B2 + 4 + h); };
-  const uint32_t o_free = bar0 + 8 * (B2 + 6), mma_done = bar0 + 8 * (B2 + 7);
+  // P of both token halves stored (8 softmax warps); both halves' P . V of the tile complete
+  const uint32_t p_full = bar0 + 8 * (B2 + 2), pv_done = bar0 + 8 * (B2 + 3);
+  const uint32_t o_free = bar0 + 8 * (B2 + 4), mma_done = bar0 + 8 * (B2 + 5);
   // fp8 caches: Q rounded to fp16, K / V stages widened (k_full / v_full: their raw codes landed)
-  constexpr int B3 = B2 + 8;
+  constexpr int B3 = B2 + 6;
   const uint32_t q_ready = bar0 + 8 * B3;
   auto k_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
   auto v_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NSK + s); };
@@ -395,10 +398,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(p_full(h), 4);
-      mbar_init(pv_done(h), 1);
-    }
+    mbar_init(p_full, 8);
+    mbar_init(pv_done, 1);
     mbar_init(o_free, 8);
     mbar_init(mma_done, 1);
     if constexpr (F8) {
@@ -518,14 +519,14 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       for (int k = 0; ok && k < n_units; ++k) {
         const MqUnit U = unit_at(k);
         if (U.kind != kRun) continue;
-        if (!(ok = mbar_wait_sleep(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
+        if (!(ok = mbar_wait_bounded(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
         // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1); tile j is tile g0 + j of the CTA
         const int g0 = g;
         for (int j = 0; ok && j <= U.nt; ++j) {
           if (j < U.nt) {
             const int gj = g0 + j, sk = gj % T::NSK;
-            if (!(ok = mbar_wait_sleep(F8 ? k_ready(sk) : k_full(sk), (gj / T::NSK) & 1, p.status))) break;
-            if (gj > 0 && !(ok = mbar_wait_sleep(s_free, (gj - 1) & 1, p.status))) break;
+            if (!(ok = mbar_wait_bounded(F8 ? k_ready(sk) : k_full(sk), (gj / T::NSK) & 1, p.status))) break;
+            if (gj > 0 && !(ok = mbar_wait_bounded(s_free, (gj - 1) & 1, p.status))) break;
             tc_fence_after();
             // descriptors differ only in the start-address field (address >> 4 in the low bits, all
             // addresses below 256 KB): the base descriptors plus offsets
@@ -544,21 +545,21 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             const int jj = j - 1, gjj = g0 + jj, sv = gjj % T::NSV;
             const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
             // the V tile (bf16: landed; fp8: widened)
-            if (!(ok = mbar_wait_sleep(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status))) break;
+            if (!(ok = mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status))) break;
             // the unit's first P . V overwrites O: the previous unit's epilogue must have read it
-            if (jj == 0 && ku > 0 && !(ok = mbar_wait_sleep(o_free, (ku - 1) & 1, p.status))) break;
-            for (int h = 0; ok && h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
-              if (!(ok = mbar_wait_sleep(p_full(h), gjj & 1, p.status))) break;
-              tc_fence_after();
+            if (jj == 0 && ku > 0 && !(ok = mbar_wait_bounded(o_free, (ku - 1) & 1, p.status))) break;
+            if (!(ok = mbar_wait_bounded(p_full, gjj & 1, p.status))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
                 const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
                 tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                 if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
               }
-              tc_commit(pv_done(h));
             }
-            if (!ok) break;
+            tc_commit(pv_done);
             tc_commit(v_empty(sv));
           }
         }
@@ -566,7 +567,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       }
       // drain (bounded): no MMA may still read shared memory or write TMEM at exit
       tc_commit(mma_done);
-      mbar_wait_sleep(mma_done, 0, p.status);
+      mbar_wait_bounded(mma_done, 0, p.status);
     }
   } else if (warp < 8) {  // ---------------- softmax warps 0-7 --------------------------------------
     const int quarter = warp & 3, h = warp >> 2;  // TMEM lane quarter, token half of each tile
@@ -680,11 +681,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
           const bool bad = half_tile_bad(t0) != 0u;
-          if (j > 0) wait(pv_done(h), (g + j - 1) & 1);
+          if (j > 0) wait(pv_done, (g + j - 1) & 1);
           if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(p_full(h));
+          if (lane == 0) mbar_arrive(p_full);
         }
       } else
       for (int j = 0; j < nt; ++j) {
@@ -778,7 +779,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         l += s2.x + s2.y;
         // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
         if (j > 0) {
-          wait(pv_done(h), (g + j - 1) & 1);
+          wait(pv_done, (g + j - 1) & 1);
           tc_fence_after();
           if (__any_sync(kFullMask, alpha != 1.f)) {  // a moved reference: rescale this row of O_h
 #pragma unroll 1
@@ -809,10 +810,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(h));
+        if (lane == 0) mbar_arrive(p_full);
       }
       g += nt;
-      wait(pv_done(h), (g - 1) & 1);
+      wait(pv_done, (g - 1) & 1);
       tc_fence_after();
       // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 ---
       // (m, l) of this half go to the partner warp through TMEM columns of P_h (its P . V is done)
