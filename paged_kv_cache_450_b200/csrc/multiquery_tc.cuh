@@ -109,9 +109,14 @@ struct MqTcTraits {
   static constexpr int V_OFF = K_OFF + NSK * TILE;
   static constexpr int BAR_OFF = V_OFF + NSV * TILE;
   // mbarriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free,
-  // p_full, pv_done (both token halves), o_free, mma_done; fp8 caches add q_ready, k_ready[NSK],
+  // p_full[NPB], pv_done[NPB] (both token halves of a tile; by tile parity), o_free, mma_done; fp8 caches add
+  // q_ready, k_ready[NSK],
   // v_ready[NSV]
-  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 6 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
+  // P buffers in TMEM: two (tile parity) when P is one 16-bit value per probability row (stacked rows,
+  // fp8 caches), so the softmax writes P of tile t while P . V of tile t - 1 still reads the other; one
+  // (hi and residual parts) for bf16 caches otherwise
+  static constexpr int NPB = (STACK || F8) ? 2 : 1;
+  static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
   // the sequence of each of the CTA's first MAX_UNITS units (longest-first rank -> sequence)
   static constexpr int MAX_UNITS = 64;
@@ -120,7 +125,8 @@ struct MqTcTraits {
   // hold at most three warps of the bf16 kernel's ~140 registers (four would cap them at 128)
   static constexpr int THREADS = F8 ? 416 : 384;
   static constexpr int W_K = 8, W_KWIDEN = 9, W_V = 10, W_MMA = 11, W_VWIDEN = 12;
-  // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or fp16 0,1 (32 + 32)
+  // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or (stacked bf16, fp16)
+  // buffer 0: halves 0,1 (32 + 32), buffer 1: halves 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
   // (block ids are read from the table as the tiles are issued: nothing depends on the partition length)
   static constexpr size_t smem_bytes(int /*partition_blocks*/) { return 1024 + UNIT_OFF + 4 * MAX_UNITS; }
@@ -365,11 +371,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
   auto v_empty = [&](int s) { return bar0 + 8 * (2 + 2 * T::NSK + T::NSV + s); };
   constexpr int B2 = 2 + 2 * T::NSK + 2 * T::NSV;
   const uint32_t s_full = bar0 + 8 * B2, s_free = bar0 + 8 * (B2 + 1);
-  // P of both token halves stored (8 softmax warps); both halves' P . V of the tile complete
-  const uint32_t p_full = bar0 + 8 * (B2 + 2), pv_done = bar0 + 8 * (B2 + 3);
-  const uint32_t o_free = bar0 + 8 * (B2 + 4), mma_done = bar0 + 8 * (B2 + 5);
+  // tile t: P of both token halves stored (8 softmax warps) on p_full(t & 1), phase t >> 1; both halves'
+  // P . V of the tile complete on pv_done(t & 1), phase t >> 1
+  auto p_full = [&](int t) { return bar0 + 8 * (B2 + 2 + (t & 1)); };
+  auto pv_done = [&](int t) { return bar0 + 8 * (B2 + 4 + (t & 1)); };
+  const uint32_t o_free = bar0 + 8 * (B2 + 6), mma_done = bar0 + 8 * (B2 + 7);
   // fp8 caches: Q rounded to fp16, K / V stages widened (k_full / v_full: their raw codes landed)
-  constexpr int B3 = B2 + 6;
+  constexpr int B3 = B2 + 8;
   const uint32_t q_ready = bar0 + 8 * B3;
   auto k_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + s); };
   auto v_ready = [&](int s) { return bar0 + 8 * (B3 + 1 + T::NSK + s); };
@@ -398,8 +406,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
-    mbar_init(p_full, 8);
-    mbar_init(pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(p_full(b), 8);
+      mbar_init(pv_done(b), 1);
+    }
     mbar_init(o_free, 8);
     mbar_init(mma_done, 1);
     if constexpr (F8) {
@@ -421,7 +431,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(data + T::SLOT_OFF);
   const uint32_t tmem_s = tmem;
   auto tmem_o = [&](int h) { return tmem + 128 + 128 * h; };
-  auto tmem_p = [&](int h) { return tmem + 384 + 32 * h; };    // tokens 64h .. 64h+63 packed in pairs: hi / fp16
+  // P of tile t, tokens 64h .. 64h+63 packed in pairs: hi / fp16
+  auto tmem_p = [&](int h, int t) { return tmem + 384 + 64 * (T::NPB == 2 ? (t & 1) : 0) + 32 * h; };
   auto tmem_plo = [&](int h) { return tmem + 448 + 32 * h; };  // bf16 caches: the residual
 
   if (warp == T::W_K || warp == T::W_V) {  // ---------------- TMA producers of Q and K, and of V --------
@@ -548,18 +559,18 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             if (!(ok = mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status))) break;
             // the unit's first P . V overwrites O: the previous unit's epilogue must have read it
             if (jj == 0 && ku > 0 && !(ok = mbar_wait_bounded(o_free, (ku - 1) & 1, p.status))) break;
-            if (!(ok = mbar_wait_bounded(p_full, gjj & 1, p.status))) break;
+            if (!(ok = mbar_wait_bounded(p_full(gjj), (gjj >> 1) & 1, p.status))) break;
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
                 const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
-                tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h, gjj) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                 if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
               }
             }
-            tc_commit(pv_done);
+            tc_commit(pv_done(gjj));
             tc_commit(v_empty(sv));
           }
         }
@@ -667,11 +678,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         }
         return bad;
       };
+      // P of tile t goes into a buffer last read by the P . V of tile t - NPB: that one must be complete
+      // (and so the warp never arrives on p_full ahead of the phase)
+      auto wait_p_buffer = [&](int t) {
+        const int tw = t - T::NPB;
+        if (tw >= 0) wait(pv_done(tw), (tw >> 1) & 1);
+      };
       // A warp whose 32 rows all lie past the unit's query rows (grouped verification uses 40 of 128)
-      // computes nothing: it keeps every barrier step -- including the wait for the previous tile's
-      // P . V, so that it never arrives on p_full ahead of the phase -- and its share of the V-row
-      // zeroing (that share is by token, not by query row).  Its P rows stay stale: they only feed
-      // output rows nobody writes.
+      // computes nothing: it keeps every barrier step -- including the wait for the P buffer -- and its
+      // share of the V-row zeroing (that share is by token, not by query row).  Its P rows stay stale:
+      // they only feed output rows nobody writes.
       if (U.qt * T::ROWS + 32 * (STACK ? (quarter & 1) : quarter) >= U.rows_total) {
         for (int j = 0; j < nt; ++j) {
           const int t0 = tok_begin + j * T::TOK + 64 * h;
@@ -681,11 +697,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
           const bool bad = half_tile_bad(t0) != 0u;
-          if (j > 0) wait(pv_done, (g + j - 1) & 1);
+          wait_p_buffer(g + j);
           if (!F8 && (t0 + 64 > tok_end || bad)) zero_v_rows(j, bad);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(p_full);
+          if (lane == 0) mbar_arrive(p_full(g + j));
         }
       } else
       for (int j = 0; j < nt; ++j) {
@@ -777,11 +793,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         }
         const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
         l += s2.x + s2.y;
-        // P_h . V_h of the previous tile must be complete: P_h is rewritten, and O_h may be rescaled
+        // the P buffer of this tile must be free; O_h is rescaled (rarely) once the previous tile's
+        // P . V is complete
+        wait_p_buffer(g + j);
+        tc_fence_after();
         if (j > 0) {
-          wait(pv_done, (g + j - 1) & 1);
-          tc_fence_after();
           if (__any_sync(kFullMask, alpha != 1.f)) {  // a moved reference: rescale this row of O_h
+            if constexpr (T::NPB == 2) {
+              wait(pv_done(g + j - 1), ((g + j - 1) >> 1) & 1);
+              tc_fence_after();
+            }
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               uint32_t u[32];
@@ -804,16 +825,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             pw[k] = lo_part ? plo[16 * c + k] : ph[16 * c + k];
             lw[k] = plo[16 * c + k];
           }
-          tmem_st16(tmem_p(h) + lane_off + 16 * c, pw);
+          tmem_st16(tmem_p(h, g + j) + lane_off + 16 * c, pw);
           if constexpr (!F8 && !STACK) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(p_full(g + j));
       }
       g += nt;
-      wait(pv_done, (g - 1) & 1);
+      wait(pv_done(g - 1), ((g - 1) >> 1) & 1);  // (and so every earlier P . V)
       tc_fence_after();
       // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 ---
       // (m, l) of this half go to the partner warp through TMEM columns of P_h (its P . V is done)
@@ -823,7 +844,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         for (int c = 0; c < 16; ++c) w[c] = 0u;
         w[0] = __float_as_uint(m);
         w[1] = __float_as_uint(l);
-        tmem_st16(tmem_p(h) + lane_off, w);
+        tmem_st16(tmem_p(h, 0) + lane_off, w);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -832,7 +853,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       float m_o, l_o;
       {
         uint32_t x[32];
-        tmem_ld32(tmem_p(h ^ 1) + lane_off, x);
+        tmem_ld32(tmem_p(h ^ 1, 0) + lane_off, x);
         tmem_ld_wait(x);
         m_o = __uint_as_float(x[0]);
         l_o = __uint_as_float(x[1]);
