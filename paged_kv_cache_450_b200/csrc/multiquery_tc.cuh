@@ -56,9 +56,12 @@
 //              per block and 64-dim half); owns the TMEM allocation.
 //   warp 10    TMA producer of the V tiles (three-stage ring).
 //   warp 11    MMA issuer: one thread issues S_j as soon as the softmax has
-//              taken S_{j-1} into registers, then P_{j-1} . V_{j-1}; completion
-//              is signalled through tcgen05.commit on mbarriers.
-//   warps 9, 12  fp8 caches: widen the K (9) and V (12) tiles (bf16: warp 9 idles, no warp 12).
+//              taken S_{j-1} into registers; completion is signalled through
+//              tcgen05.commit on mbarriers.
+//   warp 9     bf16 caches: the P_j . V_j issuer (its own waits and commits, so
+//              the two issuing threads' barrier work overlaps the other's MMAs).
+//   warps 9, 12  fp8 caches: widen the K (9) and V (12) tiles; warp 11 issues
+//              both MMA streams (S_j, then P_{j-1} . V_{j-1}).
 // Caches of fp8 (E4M3, F8 = true): the producer warps TMA each tile's raw codes
 // (128 bytes per token row) into the upper half of the tile's own ring stage;
 // warps 9 and 12 then widen them exactly to fp16 in place (one thread per token
@@ -125,6 +128,9 @@ struct MqTcTraits {
   // hold at most three warps of the bf16 kernel's ~140 registers (four would cap them at 128)
   static constexpr int THREADS = F8 ? 416 : 384;
   static constexpr int W_K = 8, W_KWIDEN = 9, W_V = 10, W_MMA = 11, W_VWIDEN = 12;
+  // the P . V issuer: warp 9 with bf16 caches (idle otherwise), the S issuer itself with fp8 caches
+  static constexpr int W_PV = F8 ? W_MMA : 9;
+  static constexpr int N_ISSUERS = W_PV == W_MMA ? 1 : 2;
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or (stacked bf16, fp16)
   // buffer 0: halves 0,1 (32 + 32), buffer 1: halves 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       mbar_init(pv_done(b), 1);
     }
     mbar_init(o_free, 8);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, T::N_ISSUERS);
     if constexpr (F8) {
       mbar_init(q_ready, 8);
       for (int s = 0; s < T::NSK; ++s) mbar_init(k_ready(s), 1);
@@ -519,64 +525,79 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         if (lane == 0) mbar_arrive(is_k ? k_ready(st) : v_ready(st));
       }
     }
-  } else if (warp == T::W_MMA) {  // ---------------- MMA issuer ------------------------------
+  } else if (warp == T::W_MMA || warp == T::W_PV) {  // ---------------- MMA issuers ----------------------
+    // bf16 caches: warp 11 issues the S MMAs and warp 9 the P . V MMAs, each with its own waits and
+    // commits, so one thread's barrier work overlaps the other's MMAs in the tensor pipe (the two
+    // streams touch disjoint TMEM columns; their order is set by the barriers alone).  fp8 caches
+    // (warp 9 widens K): warp 11 issues both, S(j) then P . V(j - 1).
     if (lane == 0) {
       constexpr uint32_t idesc_s = F8 ? idesc_f16_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
-      int g = 0, ku = 0;  // tiles whose S was issued; units
+      const bool do_s = warp == T::W_MMA, do_pv = warp == T::W_PV;
+      // S of tile j of the unit (tile gj of the CTA)
+      auto issue_s = [&](const MqUnit& U, int j, int gj) -> bool {
+        const int sk = gj % T::NSK;
+        if (!mbar_wait_bounded(F8 ? k_ready(sk) : k_full(sk), (gj / T::NSK) & 1, p.status)) return false;
+        if (gj > 0 && !mbar_wait_bounded(s_free, (gj - 1) & 1, p.status)) return false;
+        tc_fence_after();
+        // descriptors differ only in the start-address field (address >> 4 in the low bits, all
+        // addresses below 256 KB): the base descriptors plus offsets
+        const uint64_t kd0 = qd0 + ((T::K_OFF - T::Q_OFF + sk * T::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * T::HALF + (kk & 3) * 32) >> 4;
+          tc_mma_bf16(tmem_s, qd0 + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        tc_commit(k_empty(sk));
+        if (j == U.nt - 1) tc_commit(q_empty);  // the unit's S MMAs are its only readers of Q
+        return true;
+      };
+      // P . V of tile jj of unit ku (tile gjj of the CTA)
+      auto issue_pv = [&](int jj, int gjj, int ku) -> bool {
+        const int sv = gjj % T::NSV;
+        const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
+        // the V tile (bf16: landed; fp8: widened)
+        if (!mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status)) return false;
+        // the unit's first P . V overwrites O: the previous unit's epilogue must have read it
+        if (jj == 0 && ku > 0 && !mbar_wait_bounded(o_free, (ku - 1) & 1, p.status)) return false;
+        if (!mbar_wait_bounded(p_full(gjj), (gjj >> 1) & 1, p.status)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
+            const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
+            tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h, gjj) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
+          }
+        }
+        tc_commit(pv_done(gjj));
+        tc_commit(v_empty(sv));
+        return true;
+      };
+      int g = 0, ku = 0;  // tiles of the CTA so far; units
       bool ok = true;
       for (int k = 0; ok && k < n_units; ++k) {
         const MqUnit U = unit_at(k);
         if (U.kind != kRun) continue;
-        if (!(ok = mbar_wait_bounded(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
-        // per iteration j: S(j), then P_0.V_0(j-1) and P_1.V_1(j-1); tile j is tile g0 + j of the CTA
-        const int g0 = g;
-        for (int j = 0; ok && j <= U.nt; ++j) {
-          if (j < U.nt) {
-            const int gj = g0 + j, sk = gj % T::NSK;
-            if (!(ok = mbar_wait_bounded(F8 ? k_ready(sk) : k_full(sk), (gj / T::NSK) & 1, p.status))) break;
-            if (gj > 0 && !(ok = mbar_wait_bounded(s_free, (gj - 1) & 1, p.status))) break;
-            tc_fence_after();
-            // descriptors differ only in the start-address field (address >> 4 in the low bits, all
-            // addresses below 256 KB): the base descriptors plus offsets
-            const uint64_t kd0 = qd0 + ((T::K_OFF - T::Q_OFF + sk * T::TILE) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = ((kk >> 2) * T::HALF + (kk & 3) * 32) >> 4;
-              tc_mma_bf16(tmem_s, qd0 + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(s_full);
-            tc_commit(k_empty(sk));
-            if (j == U.nt - 1) tc_commit(q_empty);  // the unit's S MMAs are its only readers of Q
-            ++g;
+        if (do_s && !(ok = mbar_wait_bounded(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
+        if (do_s && do_pv) {  // one issuer: per iteration j, S(j) then P . V(j - 1)
+          for (int j = 0; ok && j <= U.nt; ++j) {
+            if (j < U.nt) ok = issue_s(U, j, g + j);
+            if (ok && j > 0) ok = issue_pv(j - 1, g + j - 1, ku);
           }
-          if (j > 0) {
-            const int jj = j - 1, gjj = g0 + jj, sv = gjj % T::NSV;
-            const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
-            // the V tile (bf16: landed; fp8: widened)
-            if (!(ok = mbar_wait_bounded(F8 ? v_ready(sv) : v_full(sv), (gjj / T::NSV) & 1, p.status))) break;
-            // the unit's first P . V overwrites O: the previous unit's epilogue must have read it
-            if (jj == 0 && ku > 0 && !(ok = mbar_wait_bounded(o_free, (ku - 1) & 1, p.status))) break;
-            if (!(ok = mbar_wait_bounded(p_full(gjj), (gjj >> 1) & 1, p.status))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
-                const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
-                tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h, gjj) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
-              }
-            }
-            tc_commit(pv_done(gjj));
-            tc_commit(v_empty(sv));
-          }
+        } else if (do_s) {
+          for (int j = 0; ok && j < U.nt; ++j) ok = issue_s(U, j, g + j);
+        } else {
+          for (int j = 0; ok && j < U.nt; ++j) ok = issue_pv(j, g + j, ku);
         }
+        g += U.nt;
         ++ku;
       }
-      // drain (bounded): no MMA may still read shared memory or write TMEM at exit
+      // drain (bounded): no MMA of this thread may still read shared memory or write TMEM at exit
       tc_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, p.status);
     }
