@@ -106,11 +106,21 @@ struct MqTcTraits {
   // are widened to fp16 in place).  Three V stages: a V tile is issued once the
   // P . V two tiles back has read its stage, so it has about two tiles' time
   // to land.
-  static constexpr int NSK = 3, NSV = 3;
+  // (stacked rows: two K stages -- K is read by the S MMAs alone, issued as soon as it lands -- and the
+  // third stage's space holds the P exchange buffers below)
+  static constexpr int NSK = STACK ? 2 : 3, NSV = 3;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
-  static constexpr int BAR_OFF = V_OFF + NSV * TILE;
+  // stacked rows: the two warps of a row pair (TMEM lanes r and r + 64) split each tile's exponentials
+  // and swap what the other stores -- 16 words per thread, two buffers by tile parity -- plus one float
+  // per thread for the row-sum parts at the end of a unit
+  static constexpr int XCH_OFF = V_OFF + NSV * TILE;
+  static constexpr int XCH_TILE = 256 * 16 * 4;
+  static constexpr int XCH_BYTES = STACK ? 2 * XCH_TILE + 256 * 4 : 0;
+  // (the epilogue's residual shares, 64 rows x 128 fp32, reuse the two exchange buffers)
+  static_assert(!STACK || 2 * XCH_TILE >= 64 * 128 * 4, "exchange buffers hold the residual shares");
+  static constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
   // mbarriers: q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full, s_free,
   // p_full[NPB], pv_done[NPB] (both token halves of a tile; by tile parity), o_free, mma_done; fp8 caches add
   // q_ready, k_ready[NSK],
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       if (U.kind != kRun) continue;
       if (is_k) {  // Q of this unit once the previous unit is done with the Q tile (its S MMAs; stacked:
                    // its epilogue too)
-        if (ku > 0 && !(ok = warp_wait_bounded(STACK ? o_free : q_empty, (ku - 1) & 1, p.status))) break;
+        if (ku > 0 && !(ok = warp_wait_bounded(q_empty, (ku - 1) & 1, p.status))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full, T::TILE);
           tma_load_3d(base + T::Q_OFF, &qmap, q_full, 0, U.hk * G, U.q0 + U.qt * QPT);
@@ -609,6 +619,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     const int r = STACK ? (tl & 63) : tl;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float qk = p.q_scale;
+    const int pair_bar = 5 + 2 * (quarter & 1) + h;  // stacked: named barrier of the two warps of a row
     // After a timed-out wait the warp stops waiting (every later wait fails at
     // once) but still runs every unit and iteration, so the two warps of a pair
     // meet at the epilogue's named barriers; the status bit reports the failure.
@@ -793,6 +804,49 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) sum4[e] = make_float2(0.f, 0.f);
         uint32_t ph[32], plo[32];
+        if constexpr (STACK) {
+          // The row's two warps hold the same scores: the high-part warp takes token pairs 0-15 of the
+          // half tile, the residual warp pairs 16-31; each sends the other the part it stores (the
+          // residuals of pairs 0-15, the high parts of pairs 16-31) and keeps its share of the row sum.
+          uint32_t own[16], send[16], recv[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float x0 = lo_part ? sv[32 + 2 * k] : sv[2 * k], x1 = lo_part ? sv[33 + 2 * k] : sv[2 * k + 1];
+            const float2 x = __ffma2_rn(make_float2(x0, x1), qk2, nm2);
+            const float a = fast_exp2(x.x), bb = fast_exp2(x.y);
+            sum4[k & 3] = __fadd2_rn(sum4[k & 3], make_float2(a, bb));
+            const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(bb);
+            const float2 rr = __fadd2_rn(make_float2(a, bb),
+                                         make_float2(__uint_as_float((ua & 0xFFFF0000u) ^ 0x80000000u),
+                                                     __uint_as_float((ub & 0xFFFF0000u) ^ 0x80000000u)));
+            const uint32_t hi = __byte_perm(ua, ub, 0x7632);
+            const uint32_t lo = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+            own[k] = lo_part ? lo : hi;
+            send[k] = lo_part ? hi : lo;
+          }
+          // thread (warp, lane) and its partner (warp ^ 2, lane): word group c of thread i at c * 256 + i
+          uint4* xs = reinterpret_cast<uint4*>(data + T::XCH_OFF + ((g + j) & 1) * T::XCH_TILE);
+          const int me = warp * 32 + lane, other = (warp ^ 2) * 32 + lane;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            xs[c * 256 + me] = make_uint4(send[4 * c], send[4 * c + 1], send[4 * c + 2], send[4 * c + 3]);
+          asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = xs[c * 256 + other];
+            recv[4 * c] = v.x;
+            recv[4 * c + 1] = v.y;
+            recv[4 * c + 2] = v.z;
+            recv[4 * c + 3] = v.w;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {  // high parts for the high-part warp, residuals for the other
+            ph[k] = own[k];
+            ph[16 + k] = recv[k];
+            plo[k] = recv[k];
+            plo[16 + k] = own[k];
+          }
+        } else {
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const float2 x = __ffma2_rn(make_float2(sv[2 * k], sv[2 * k + 1]), qk2, nm2);
@@ -811,6 +865,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             ph[k] = __byte_perm(ua, ub, 0x7632);  // {b.hi16, a.hi16}: token 2k in the low half
             plo[k] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
           }
+        }
         }
         const float2 s2 = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
         l += s2.x + s2.y;
@@ -857,6 +912,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       g += nt;
       wait(pv_done(g - 1), ((g - 1) >> 1) & 1);  // (and so every earlier P . V)
       tc_fence_after();
+      if constexpr (STACK) {  // the row sum: this warp's share plus its partner's (high-part share first)
+        float* lx = reinterpret_cast<float*>(data + T::XCH_OFF + 2 * T::XCH_TILE);
+        lx[warp * 32 + lane] = l;
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        const float lp = lx[(warp ^ 2) * 32 + lane];
+        l = lo_part ? lp + l : l + lp;
+      }
       // ---- epilogue: merge the two halves' (m, l, O_h); this warp writes output dims 64h .. 64h+63 ---
       // (m, l) of this half go to the partner warp through TMEM columns of P_h (its P . V is done)
       {
@@ -886,10 +948,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       const float w0 = (h == 0 ? w_self : w_oth) * inv, w1 = (h == 0 ? w_oth : w_self) * inv;  // O_0, O_1 weights
       const int64_t orow = static_cast<int64_t>(U.q0 + row / G) * Hq + U.hk * G + row % G;
       // stacked: the residual's share of this row's output (accumulator rows 64-127) goes from the warp
-      // of lanes 64-127 to the warp of the same row and half through the Q tile (free: the next unit's
-      // Q waits for o_free)
-      float* xo = reinterpret_cast<float*>(data + T::Q_OFF);  // [64 rows][128 dims]
-      const int pair_bar = 5 + 2 * (quarter & 1) + h;       // named barrier of the two warps of this row
+      // of lanes 64-127 to the warp of the same row and half through the P exchange buffers (the
+      // unit's last exchange was read before the row-sum barrier above), so the next unit's Q can
+      // load while this epilogue runs
+      float* xo = reinterpret_cast<float*>(data + T::XCH_OFF);  // [64 rows][128 dims]
       if (STACK && !lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
@@ -938,8 +1000,11 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
       }
-      if (STACK && lo_part) {
-        fence_proxy_async_smem();  // these writes before the next unit's Q load (async proxy)
+      if constexpr (STACK) {
+        // the residual warp's writes are complete (its arrival pairs with the wait before the loop);
+        // then both wait until the high-part warp has read them: the next unit's exchanges reuse the
+        // buffers
+        if (lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
         asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
       }
       if (valid && ok && U.nparts > 1 && h == 0 && !lo_part) {
