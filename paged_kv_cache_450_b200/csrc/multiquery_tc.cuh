@@ -224,7 +224,10 @@ __device__ __forceinline__ MqUnit mq_unit(const MultiQueryParams& p, int64_t u, 
   U.part = y;
   U.table = nullptr;
   U.nt = U.nb = U.nparts = 0;
-  if (!query_rows_ok(p, b, U.q0, U.q_len)) {  // before any load or store
+  // the sequence's context length is loaded beside its query range (b < num_seqs: in bounds), so the
+  // unit's description costs one memory latency, not two -- it sits between units on every warp's path
+  const int ctx_loaded = p.context_lens[b];
+  if (!query_rows_ok(p, b, U.q0, U.q_len)) {  // before any access through the query range
     U.kind = kBadQuery;
     return U;
   }
@@ -232,7 +235,7 @@ __device__ __forceinline__ MqUnit mq_unit(const MultiQueryParams& p, int64_t u, 
   U.kind = kSkip;
   if (U.q_len <= 0 || U.qt * 128 >= U.rows_total) return U;
   const int max_ctx = p.max_blocks_per_seq * BS;
-  int ctx = p.context_lens[b];
+  int ctx = ctx_loaded;
   if (ctx < 0 || ctx > max_ctx) {
     if (threadIdx.x == 0 && U.hk == 0 && U.part == 0 && U.qt == 0) set_status(p.status, PKV_STATUS_BAD_CONTEXT);
     ctx = ctx < 0 ? 0 : max_ctx;
@@ -952,7 +955,6 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       // unit's last exchange was read before the row-sum barrier above), so the next unit's Q can
       // load while this epilogue runs
       float* xo = reinterpret_cast<float*>(data + T::XCH_OFF);  // [64 rows][128 dims]
-      if (STACK && !lo_part) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         const int d0 = 64 * h + 32 * c;
@@ -961,6 +963,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         tmem_ld32(tmem_o(1) + lane_off + d0, u1);
         tmem_ld_wait(u0);
         tmem_ld_wait(u1);
+        // (the high-part warp's first accumulator reads overlap the residual warp's writes)
+        if (STACK && !lo_part && c == 0) asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
         if (!valid || !ok) continue;
         float o[32];
 #pragma unroll
