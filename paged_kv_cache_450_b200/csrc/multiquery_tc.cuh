@@ -158,6 +158,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
+// 32-byte global store of eight 32-bit words (sm_100); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // max(a, b, c) in one instruction (sm_100).
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
@@ -380,6 +387,9 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     return mq_unit<BS, G>(p, u, ranked ? unit_b[k] : z, gx, gy);
   };
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  // 32-byte output stores need 32-byte aligned rows (rows are 256 bytes; the bases only promise 16)
+  const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;
+  const bool ws_v8 = (reinterpret_cast<uintptr_t>(p.ws_o) & 31) == 0;
 
   const uint32_t base = smem_u32(data);
   const uint32_t bar0 = base + T::BAR_OFF;
@@ -985,23 +995,41 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
             o[e + 3] += v.w;
           }
         }
+        // Each lane writes its own row: 32-byte stores (whole sectors, half the store transactions of
+        // 16-byte ones) where the base allows, 16-byte ones otherwise.
         if (U.nparts == 1) {
           __nv_bfloat16* dst = out + orow * D + d0;
+          uint32_t w[2][8];
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t w[4];
+          for (int kq = 0; kq < 16; ++kq) {
+            __nv_bfloat162 hv = __floats2bfloat162_rn(o[2 * kq], o[2 * kq + 1]);
+            w[kq >> 3][kq & 7] = *reinterpret_cast<uint32_t*>(&hv);
+          }
+          if (out_v8) {
+            st_global_v8(dst, w[0]);
+            st_global_v8(dst + 16, w[1]);
+          } else {
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              __nv_bfloat162 hv = __floats2bfloat162_rn(o[e + 2 * kq], o[e + 2 * kq + 1]);
-              w[kq] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e)
+              *reinterpret_cast<uint4*>(dst + 8 * e) =
+                  make_uint4(w[e >> 1][4 * (e & 1)], w[e >> 1][4 * (e & 1) + 1], w[e >> 1][4 * (e & 1) + 2],
+                             w[e >> 1][4 * (e & 1) + 3]);
           }
         } else {
           float* dst = p.ws_o + (orow * p.max_partitions + U.part) * D + d0;
+          if (ws_v8) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t w8[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) w8[q] = __float_as_uint(o[e + q]);
+              st_global_v8(dst + e, w8);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+          }
         }
       }
       if constexpr (STACK) {
