@@ -227,10 +227,11 @@ __device__ __forceinline__ void finish_partition(const float* c_m, const float* 
       out[(out_row0 + g) * D + e] = Elem<TQ>::from_float(o);
     } else {
       const int64_t slot = (out_row0 + g) * p.max_partitions + part;
-      p.ws_o[slot * D + e] = o;
+      const uint64_t keep = l2_policy_evict_last();
+      st_global_hint(p.ws_o + slot * D + e, o, keep);
       if (e == 0) {
-        p.ws_ml[slot * 2] = M * kLn2;
-        p.ws_ml[slot * 2 + 1] = L;
+        st_global_hint(p.ws_ml + slot * 2, M * kLn2, keep);
+        st_global_hint(p.ws_ml + slot * 2 + 1, L, keep);
       }
     }
   }

@@ -91,6 +91,11 @@ __device__ __forceinline__ void store8(float* dst, const float (&v)[8]) {
   reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
+// (split-context partials: with an L2 policy)
+__device__ __forceinline__ void store8(float* dst, const float (&v)[8], uint64_t policy) {
+  st_global_hint(dst, make_float4(v[0], v[1], v[2], v[3]), policy);
+  st_global_hint(dst + 4, make_float4(v[4], v[5], v[6], v[7]), policy);
+}
 
 // Byte offset of logical 16-byte chunk q of row t in a 128-byte-swizzled tile.
 __device__ __forceinline__ int swz(int t, int q) { return t * 128 + ((q ^ (t & 7)) << 4); }
@@ -399,6 +404,7 @@ __global__ void __launch_bounds__(32, MINB)
     }
   } else {
     const int64_t slot_a = row_a * p.max_partitions + part, slot_b = row_b * p.max_partitions + part;
+    const uint64_t keep = l2_policy_evict_last();
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float va[8], vb[8];
@@ -407,14 +413,14 @@ __global__ void __launch_bounds__(32, MINB)
         va[i] = o[i][2 * h] * f0;
         vb[i] = o[i][2 * h + 1] * f1;
       }
-      store8(p.ws_o + slot_a * D + 8 * r + 64 * h, va);
-      store8(p.ws_o + slot_b * D + 8 * r + 64 * h, vb);
+      store8(p.ws_o + slot_a * D + 8 * r + 64 * h, va, keep);
+      store8(p.ws_o + slot_b * D + 8 * r + 64 * h, vb, keep);
     }
     if (r == 0) {
-      p.ws_ml[slot_a * 2] = m0 * kLn2;
-      p.ws_ml[slot_a * 2 + 1] = l0;
-      p.ws_ml[slot_b * 2] = m1 * kLn2;
-      p.ws_ml[slot_b * 2 + 1] = l1;
+      st_global_hint(p.ws_ml + slot_a * 2, m0 * kLn2, keep);
+      st_global_hint(p.ws_ml + slot_a * 2 + 1, l0, keep);
+      st_global_hint(p.ws_ml + slot_b * 2, m1 * kLn2, keep);
+      st_global_hint(p.ws_ml + slot_b * 2 + 1, l1, keep);
     }
   }
 }

@@ -401,26 +401,27 @@ __global__ void __launch_bounds__(32, MINB)
   } else {
     const int64_t slot_a = (ha < cols ? row_of(ha) : 0) * p.max_partitions + slot0 + part;
     const int64_t slot_b = (hb < cols ? row_of(hb) : 0) * p.max_partitions + slot0 + part;
+    const uint64_t keep = l2_policy_evict_last();
 #pragma unroll
     for (int mi = 0; mi < 8; ++mi) {
       const int d0 = 16 * mi + r, d1 = d0 + 8;
       if (ha < cols) {
-        p.ws_o[slot_a * D + d0] = o[mi][0] * f0;
-        p.ws_o[slot_a * D + d1] = o[mi][2] * f0;
+        st_global_hint(p.ws_o + slot_a * D + d0, o[mi][0] * f0, keep);
+        st_global_hint(p.ws_o + slot_a * D + d1, o[mi][2] * f0, keep);
       }
       if (hb < cols) {
-        p.ws_o[slot_b * D + d0] = o[mi][1] * f1;
-        p.ws_o[slot_b * D + d1] = o[mi][3] * f1;
+        st_global_hint(p.ws_o + slot_b * D + d0, o[mi][1] * f1, keep);
+        st_global_hint(p.ws_o + slot_b * D + d1, o[mi][3] * f1, keep);
       }
     }
     if (r == 0) {
       if (ha < cols) {
-        p.ws_ml[slot_a * 2] = m0 * kLn2;
-        p.ws_ml[slot_a * 2 + 1] = l0;
+        st_global_hint(p.ws_ml + slot_a * 2, m0 * kLn2, keep);
+        st_global_hint(p.ws_ml + slot_a * 2 + 1, l0, keep);
       }
       if (hb < cols) {
-        p.ws_ml[slot_b * 2] = m1 * kLn2;
-        p.ws_ml[slot_b * 2 + 1] = l1;
+        st_global_hint(p.ws_ml + slot_b * 2, m1 * kLn2, keep);
+        st_global_hint(p.ws_ml + slot_b * 2 + 1, l1, keep);
       }
     }
   }
