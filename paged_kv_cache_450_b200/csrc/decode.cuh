@@ -428,8 +428,29 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   finish_partition<TQ, D, G, T::NW>(c_m, c_l, c_acc, p, out_row0, part, nparts);
 }
 
-// Merge of split-context partials, one warp per (sequence, query head).
-template <typename TQ, int D>
+// PVV consecutive floats of a partial output (16- or 8-byte aligned: offsets are multiples of PVV).
+template <int PVV>
+__device__ __forceinline__ void load_partial(const float* src, float (&v)[PVV]) {
+  if constexpr (PVV == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(src);
+    v[0] = x.x;
+    v[1] = x.y;
+    v[2] = x.z;
+    v[3] = x.w;
+  } else if constexpr (PVV == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(src);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < PVV; ++e) v[e] = src[e];
+  }
+}
+
+// Merge of split-context partials, one warp per (sequence, query head).  BATCH partial outputs are
+// loaded at once (8 or 16: the registers they take set how many CTAs share an SM, so launches whose
+// rows have at most 8 partitions use 8).
+template <typename TQ, int D, int BATCH = 16>
 __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeParams p) {
   constexpr int PVV = D / 32;
   pdl_wait_and_release();
@@ -458,6 +479,56 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   auto slot = [&](int i) { return i < n0 ? i : s1 + (i - n0); };
   const float* ml = p.ws_ml + row * p.max_partitions * 2;
   const float* o = p.ws_o + row * p.max_partitions * D;
+  TQ* out = static_cast<TQ*>(p.out) + row * D + lane * PVV;
+  if (nparts <= 64) {
+    // Lane i holds (m, l) of partitions i and i + 32; the partial outputs are read BATCH partitions
+    // at a time, every load of a batch in flight at once, the first batch beside the (m, l) loads.
+    // The arithmetic and its order are those of the general loop below (the same results).
+    float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
+    if (lane < nparts) {
+      const float2 x = *reinterpret_cast<const float2*>(ml + 2 * slot(lane));
+      m0 = x.x;
+      l0 = x.y;
+    }
+    if (lane + 32 < nparts) {
+      const float2 x = *reinterpret_cast<const float2*>(ml + 2 * slot(lane + 32));
+      m1 = x.x;
+      l1 = x.y;
+    }
+    float v[BATCH][PVV];
+    auto load_batch = [&](int c) {
+#pragma unroll
+      for (int q = 0; q < BATCH; ++q)
+        if (c + q < nparts) load_partial<PVV>(o + static_cast<int64_t>(slot(c + q)) * D + lane * PVV, v[q]);
+    };
+    load_batch(0);
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+    const float w0 = l0 > 0.f ? l0 * fast_exp2((m0 - M) * kLog2e) : 0.f;
+    const float w1 = l1 > 0.f ? l1 * fast_exp2((m1 - M) * kLog2e) : 0.f;
+    float acc[PVV];
+#pragma unroll
+    for (int e = 0; e < PVV; ++e) acc[e] = 0.f;
+    for (int c = 0; c < nparts; c += BATCH) {
+      if (c > 0) load_batch(c);
+      const float wsrc = c < 32 ? w0 : w1;  // (a batch never straddles partition 32)
+#pragma unroll
+      for (int q = 0; q < BATCH; ++q) {
+        if (c + q < nparts) {
+          const float w = __shfl_sync(kFullMask, wsrc, (c + q) & 31);
+#pragma unroll
+          for (int e = 0; e < PVV; ++e) acc[e] = fmaf(w, v[q][e], acc[e]);
+        }
+      }
+    }
+    float W = w0 + w1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(kFullMask, W, off);
+#pragma unroll
+    for (int e = 0; e < PVV; ++e) out[e] = Elem<TQ>::from_float(W > 0.f ? acc[e] / W : 0.f);
+    return;
+  }
   // Partitions are taken 32 at a time: lane i loads (m, l) of partition c + i at once, the weights
   // l e^{m - M} go to the other lanes by shuffle, and the partial outputs are read four at a time,
   // so the loads of a row overlap instead of following one another.
@@ -502,7 +573,6 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(kFullMask, W, off);
-  TQ* out = static_cast<TQ*>(p.out) + row * D + lane * PVV;
 #pragma unroll
   for (int e = 0; e < PVV; ++e) out[e] = Elem<TQ>::from_float(W > 0.f ? acc[e] / W : 0.f);
 }

@@ -69,6 +69,9 @@ static cudaError_t launch_mma_bf16_grouped(const CUtensorMap& kmap, const CUtens
 template <typename TQ, int D>
 static cudaError_t launch_reduce(const DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_q_heads;
+  if (p.max_partitions <= 8)
+    return launch_pdl(paged_decode_reduce_kernel<TQ, D, 8>, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0,
+                      st, p);
   return launch_pdl(paged_decode_reduce_kernel<TQ, D>, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, st,
                     p);
 }
