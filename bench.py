@@ -263,9 +263,10 @@ def unique_kv_bytes(w) -> int:
     return int(sum(rows.values())) * s.num_kv_heads * s.head_dim * W.elem_size(s.cache_dtype) * 2
 
 
-def step_inputs_bytes(w) -> tuple[int, int]:
+def step_inputs_bytes(w, grouped: bool = False) -> tuple[int, int]:
     """Bytes of one step's per-step inputs (host -> device) and result (device -> host)."""
-    ts = [w.q, w.new_k, w.new_v, w.slot_mapping, w.block_tables, w.context_lens, w.copy_pairs]
+    ts = [w.q, w.new_k, w.new_v, w.block_tables, w.context_lens, w.copy_pairs]
+    ts += [w.group_start, w.shared_blocks] if grouped else [w.slot_mapping]
     h2d = sum(t.numel() * t.element_size() for t in ts if t is not None)
     return h2d, w.q.numel() * w.q.element_size()
 
@@ -367,15 +368,26 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
 
     # ---- end to end through the public API with pinned host buffers ----------
     host = {k: (getattr(w, k).cpu().pin_memory() if getattr(w, k) is not None else None)
-            for k in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens", "copy_pairs")}
+            for k in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens", "copy_pairs",
+                      "group_start", "shared_blocks")}
     # two steps in flight: the copies in of step i+1 overlap the kernels of step i
-    pipe = pk.HostStepPipeline(host["q"], host["new_k"], w.key_cache, host["block_tables"], host["copy_pairs"],
-                               partition_tokens=pt, depth=2, compute_stream=stream)
+    if grouped:  # the same shared-prefix decode, its inputs and output in host memory
+        pipe = pk.SharedPrefixHostStepPipeline(host["q"], w.key_cache, host["block_tables"], host["group_start"],
+                                               host["copy_pairs"], partition_tokens=pt, depth=2,
+                                               compute_stream=stream)
 
-    def e2e_step():
-        pipe.step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
-                  host["context_lens"], w.key_cache, w.value_cache, w.scale, copy_pairs=host["copy_pairs"],
-                  k_scale=w.k_scale, v_scale=w.v_scale)
+        def e2e_step():
+            pipe.step(host["q"], host["new_k"], host["new_v"], host["block_tables"], host["context_lens"],
+                      host["group_start"], host["shared_blocks"], w.key_cache, w.value_cache, w.scale,
+                      max_group_size=max_group, copy_pairs=host["copy_pairs"])
+    else:
+        pipe = pk.HostStepPipeline(host["q"], host["new_k"], w.key_cache, host["block_tables"], host["copy_pairs"],
+                                   partition_tokens=pt, depth=2, compute_stream=stream)
+
+        def e2e_step():
+            pipe.step(host["q"], host["new_k"], host["new_v"], host["slot_mapping"], host["block_tables"],
+                      host["context_lens"], w.key_cache, w.value_cache, w.scale, copy_pairs=host["copy_pairs"],
+                      k_scale=w.k_scale, v_scale=w.v_scale)
 
     e2e_steps = max(1, args.e2e_steps)  # its own count: the two-deep pipeline's fill and drain amortised
     for _ in range(min(args.warmup, 10)):
@@ -402,7 +414,7 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
     decode_ms = max_over_ranks(decode_ms, dev)
     total_kv = sum_over_ranks(kv_bytes, dev)
     total_seqs = sum_over_ranks(s.num_seqs, dev)
-    h2d, d2h = step_inputs_bytes(w)
+    h2d, d2h = step_inputs_bytes(w, grouped)
     peak, peak_kind = hbm_peak()
     value = total_kv / (step_ms * 1e-3) / 1e9
     shared = w.copy_pairs is not None
@@ -438,10 +450,11 @@ def measure_decode(spec, args, dev, rank, world, clocks, *, headline: bool):
                      "traffic": traffic},
         "e2e": {"value": round(total_kv / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async (pinned host "
-                       "inputs and output every step; two steps in flight: copies in, kernels, copies out on "
-                       "three streams)" + ("; the host step decodes per sequence (it takes no groups)"
-                                           if grouped else "")},
+                "api": ("paged_kv_cache_450_b200.SharedPrefixHostStepPipeline -> "
+                        "pkv_decode_step_host_shared_prefix_async" if grouped else
+                        "paged_kv_cache_450_b200.HostStepPipeline -> pkv_decode_step_host_async")
+                       + " (pinned host inputs and output every step; two steps in flight: copies in, kernels, "
+                         "copies out on three streams)"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }

@@ -519,6 +519,52 @@ int pkv_decode_step_host_async(void* out_host, const void* q_host, const void* k
                                void* copy_out_stream, void* staging_free_event, void* done_event);
 
 /*
+ * pkv_decode_step_host_async for groups of sequences that share their
+ * prompt's blocks: the decode is pkv_paged_attention_decode_shared_prefix
+ * (each shared block read once for the whole group), with each sequence's new
+ * token written first inside it.
+ *
+ * Source: "vLLM — 把操作系统的分页搬进 GPU KV cache", 实践案例 2 (n candidates
+ * share the prompt's blocks) and 核心要点 (copy-on-write before the write);
+ * the step with host buffers is this library's.
+ * Enqueued in order: the host -> device copies (on copy_in_stream, after
+ * staging_free_event); pkv_kv_block_copy of copy_pairs (if num_pairs > 0);
+ * the shared-prefix decode with the new tokens fused in (on compute_stream);
+ * the device -> host copy of the output (on copy_out_stream), then done_event.
+ *
+ * k_new_host,          host [num_seqs][num_kv_heads][head_dim] of q_dtype: the
+ * v_new_host           token each sequence appends at position
+ *                      context_lens[b] - 1 (both, or both NULL for none).
+ * group_start_host,    host int32 [num_groups + 1] and [num_groups]: the groups
+ * shared_blocks_host   (see pkv_paged_attention_decode_shared_prefix).
+ * max_group_size       the largest group.
+ * staging              device scratch of at least
+ *                      pkv_decode_step_shared_prefix_staging_bytes(...) bytes,
+ *                      256-byte aligned, caller-owned.
+ * Other arguments, errors and the stream / event contract: as
+ * pkv_decode_step_host_async and pkv_paged_attention_decode_shared_prefix
+ * (bf16 only; no validation).  Argument errors are returned before anything
+ * is enqueued.
+ */
+int pkv_decode_step_host_shared_prefix_async(void* out_host, const void* q_host, const void* k_new_host,
+                                             const void* v_new_host, const int32_t* block_tables_host,
+                                             const int32_t* context_lens_host, const int32_t* group_start_host,
+                                             const int32_t* shared_blocks_host, int num_groups, int max_group_size,
+                                             const int64_t* copy_pairs_host, int64_t num_pairs, void* key_cache,
+                                             void* value_cache, int num_seqs, int num_q_heads, int num_kv_heads,
+                                             int head_dim, int block_size, int max_blocks_per_seq,
+                                             int64_t num_blocks, float scale, int q_dtype, int cache_dtype,
+                                             int partition_tokens, void* staging, size_t staging_bytes,
+                                             void* copy_in_stream, void* compute_stream, void* copy_out_stream,
+                                             void* staging_free_event, void* done_event);
+
+/* Staging bytes pkv_decode_step_host_shared_prefix_async needs for these
+ * arguments (0 for unsupported ones; a sizing helper of this library). */
+size_t pkv_decode_step_shared_prefix_staging_bytes(int num_seqs, int num_groups, int num_q_heads, int num_kv_heads,
+                                                   int head_dim, int block_size, int max_blocks_per_seq,
+                                                   int q_dtype, int partition_tokens, int64_t num_pairs);
+
+/*
  * Prefix caching by hash chain (host side; no device work).
  *
  * Source: "vLLM KV Cache 实现机制", 4.2 -- a full block is identified by a hash

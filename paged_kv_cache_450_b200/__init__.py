@@ -36,6 +36,7 @@ __all__ = ["paged_kv_write", "paged_attention_decode", "paged_decode_append", "p
            "decode_shared_prefix_workspace_bytes", "decode_shared_prefix_partition_tokens",
            "paged_attention_multiquery", "multiquery_workspace_bytes", "kv_block_copy", "swap_blocks", "fp8_scale_from_amax",
            "prefix_block_hashes", "PrefixCache", "decode_step", "decode_step_staging_bytes",
+           "HostStepPipeline", "SharedPrefixHostStepPipeline", "decode_step_shared_prefix_staging_bytes",
            "decode_workspace_bytes",
            "decode_partition_tokens", "decode_max_partitions", "decode_table_scan", "device_status", "launch_count", "PagedKVError",
            "library_path"]
@@ -516,6 +517,81 @@ class HostStepPipeline:
                 ctypes.c_void_p(self.copy_out.cuda_stream),
                 ctypes.c_void_p(self.done[k].cuda_event if self.used[k] else 0),
                 ctypes.c_void_p(self.done[k].cuda_event)), "decode_step_pipelined")
+        self.used[k] = True
+        self.i += 1
+        return out, self.done[k]
+
+    def synchronize(self):
+        for e in self.done:
+            e.synchronize()
+
+
+def decode_step_shared_prefix_staging_bytes(q, key_cache, block_tables, num_groups: int, copy_pairs=None,
+                                            partition_tokens: int = 0) -> int:
+    """Device staging bytes of a shared-prefix host step for inputs of these shapes."""
+    B, Hq, d = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+    return int(_lib.load().pkv_decode_step_shared_prefix_staging_bytes(B, int(num_groups), Hq, Hkv, d, bs,
+                                                                       block_tables.shape[1], _dtype(q),
+                                                                       partition_tokens, n_pairs))
+
+
+class SharedPrefixHostStepPipeline:
+    """HostStepPipeline for groups of sequences sharing their prompt's blocks
+    (pkv_decode_step_host_shared_prefix_async): per step the copy-on-write
+    copies, then the shared-prefix decode with each sequence's new token
+    (``new_k``/``new_v``, [num_seqs][num_kv_heads][head_dim], at position
+    context_lens - 1) written inside it.  ``depth`` steps in flight, as
+    HostStepPipeline; ``step(...)`` returns ``(out, done)`` the same way."""
+
+    def __init__(self, q, key_cache, block_tables, group_start, copy_pairs=None, partition_tokens: int = 0,
+                 depth: int = 2, compute_stream=None):
+        dev = key_cache.device
+        self.depth = int(depth)
+        self.partition_tokens = int(partition_tokens)
+        self.num_groups = int(group_start.shape[0]) - 1
+        need = decode_step_shared_prefix_staging_bytes(q, key_cache, block_tables, self.num_groups, copy_pairs,
+                                                       partition_tokens)
+        if need == 0 and q.shape[0] > 0:
+            raise ValueError("unsupported shapes or dtypes for the shared-prefix step")
+        self.staging = [torch.empty(max(need, 1), dtype=torch.uint8, device=dev) for _ in range(self.depth)]
+        self.outs = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(self.depth)]
+        self.compute = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev)
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.done = [torch.cuda.Event() for _ in range(self.depth)]
+        for e in self.done:  # create the events (torch makes them on first record)
+            e.record(self.compute)
+        self.used = [False] * self.depth
+        self.i = 0
+
+    def step(self, q, new_k, new_v, block_tables, context_lens, group_start, shared_blocks, key_cache, value_cache,
+             scale: float, *, max_group_size: int, copy_pairs=None):
+        host = [t for t in (q, new_k, new_v, block_tables, context_lens, group_start, shared_blocks, copy_pairs)
+                if t is not None]
+        if any(t.device.type != "cpu" or not t.is_contiguous() for t in host):
+            raise ValueError("host inputs must all be contiguous CPU tensors")
+        if (new_k is None) != (new_v is None):
+            raise ValueError("new_k and new_v: both or neither")
+        _cuda(key_cache, value_cache)
+        k = self.i % self.depth
+        B, Hq, d = q.shape
+        NB, bs, Hkv, _ = key_cache.shape
+        n_groups = int(group_start.shape[0]) - 1
+        n_pairs = 0 if copy_pairs is None else copy_pairs.shape[0]
+        ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        out, st = self.outs[k], self.staging[k]
+        with torch.cuda.device(key_cache.device):
+            _check(_lib.load().pkv_decode_step_host_shared_prefix_async(
+                out.data_ptr(), q.data_ptr(), ptr(new_k), ptr(new_v), block_tables.data_ptr(),
+                context_lens.data_ptr(), group_start.data_ptr(), shared_blocks.data_ptr(), n_groups,
+                int(max_group_size), ptr(copy_pairs), n_pairs, key_cache.data_ptr(), value_cache.data_ptr(), B, Hq,
+                Hkv, d, bs, block_tables.shape[1], NB, float(scale), _dtype(q), _dtype(key_cache),
+                self.partition_tokens, st.data_ptr(), st.numel(), ctypes.c_void_p(self.copy_in.cuda_stream),
+                ctypes.c_void_p(self.compute.cuda_stream), ctypes.c_void_p(self.copy_out.cuda_stream),
+                ctypes.c_void_p(self.done[k].cuda_event if self.used[k] else 0),
+                ctypes.c_void_p(self.done[k].cuda_event)), "decode_step_shared_prefix")
         self.used[k] = True
         self.i += 1
         return out, self.done[k]

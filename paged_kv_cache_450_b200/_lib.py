@@ -33,6 +33,9 @@ SIGNATURES = {
     "pkv_decode_step_staging_bytes": (SZ, [I, I, I, I, I, I, I, I, I, I64, I64]),
     "pkv_decode_step_host_async": (I, [P, P, P, P, P, I64, P, P, P, I64, P, P, I, I, I, I, I, I, I64, F, F, F, I, I,
                                        I, P, SZ, P, P, P, P, P]),
+    "pkv_decode_step_host_shared_prefix_async": (I, [P, P, P, P, P, P, P, P, I, I, P, I64, P, P, I, I, I, I, I, I, I64,
+                                                     F, I, I, I, P, SZ, P, P, P, P, P]),
+    "pkv_decode_step_shared_prefix_staging_bytes": (SZ, [I, I, I, I, I, I, I, I, I, I64]),
     "pkv_decode_partition_tokens": (I, [I, I, I, I, I, I, I, I]),
     "pkv_decode_max_partitions": (I, [I, I, I, I, I, I, I, I]),
     "pkv_decode_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),

@@ -128,6 +128,35 @@ def test_shared_prefix_partition_and_workspace():
         pk.decode_shared_prefix_workspace_bytes(128, 32, 40, 40, 128, 16, 68)
 
 
+def test_shared_prefix_host_step_staging_and_argument_errors():
+    lib = _lib.load()
+    BF = pk.DTYPE_BF16
+    # 128 sequences in 32 groups, 40 heads, d 128, bs 16, 68 blocks, 96 copy pairs: the staged inputs
+    # (each piece 256-byte aligned) followed by the shared-prefix workspace
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    qb, kb = 128 * 40 * 128 * 2, 128 * 40 * 128 * 2
+    pieces = [qb, qb, kb, kb, 128 * 68 * 4, 128 * 4, 33 * 4, 32 * 4, 96 * 16]
+    ws = pk.decode_shared_prefix_workspace_bytes(128, 32, 40, 40, 128, 16, 68)
+    want = a(sum(a(x) for x in pieces) + ws)
+    assert lib.pkv_decode_step_shared_prefix_staging_bytes(128, 32, 40, 40, 128, 16, 68, BF, 0, 96) == want
+    assert lib.pkv_decode_step_shared_prefix_staging_bytes(128, 32, 40, 40, 128, 8, 68, BF, 0, 96) == 0  # bs 8
+    # argument errors come back before anything is enqueued (no GPU needed)
+    buf = ctypes.create_string_buffer(1024)
+    p = ctypes.addressof(buf)
+    aligned = (p + 255) // 256 * 256
+    call = lambda out, k, v, staging: lib.pkv_decode_step_host_shared_prefix_async(  # noqa: E731
+        out, p, k, v, p, p, p, p, 1, 1, None, 0, p, p, 1, 8, 8, 128, 16, 4, 16, 0.1, BF, BF, 0, staging, 512,
+        None, None, None, None, None)
+    ERR_NULL_POINTER, ERR_WORKSPACE, ERR_MISALIGNED = -1, -6, -10
+    assert call(None, None, None, aligned) == ERR_NULL_POINTER       # no output buffer
+    assert call(p, p, None, aligned) == ERR_NULL_POINTER             # k_new without v_new
+    assert call(p, None, None, aligned + 16) == ERR_MISALIGNED       # staging not 256-byte aligned
+    assert call(p, None, None, aligned) == ERR_WORKSPACE             # staging too small
+    assert lib.pkv_decode_step_host_shared_prefix_async(
+        None, None, None, None, None, None, None, None, 0, 0, None, 0, p, p, 0, 8, 8, 128, 16, 4, 16, 0.1, BF, BF, 0,
+        aligned, 512, None, None, None, None, None) == 0                     # nothing to do
+
+
 def test_multiquery_partition_and_workspace():
     lib = _lib.load()
     BF, F8 = pk.DTYPE_BF16, pk.DTYPE_FP8_E4M3

@@ -178,3 +178,59 @@ def test_kernel_skips_a_group_past_the_batch():
     torch.cuda.synchronize()
     assert pk.device_status(clear=True) & pk.STATUS_BAD_GROUP
     assert_close(f64(out)[:4], ref[:4], *tol_for(w), what="the well-formed group")
+
+
+@pytest.mark.parametrize("depth", [1, 2])
+def test_shared_prefix_host_step_pipeline(depth):
+    """pkv_decode_step_host_shared_prefix_async through SharedPrefixHostStepPipeline: host inputs
+    copied in, the copy-on-write copies, the shared-prefix decode with the new tokens fused in, the
+    output copied out -- every step equal to the device-side calls on the same inputs; one step's
+    caches equal to the oracle's and its output within tolerance of it."""
+    spec = W.PARALLEL_SAMPLING.with_(name="sph", num_seqs=12, num_q_heads=8, num_kv_heads=4,
+                                     sampling=(3, 4, 150, 1, 70))
+    w = W.make_decode_workload(spec, seed=23, device=DEV)
+    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+    host = {k: pin(getattr(w, k)) for k in ("new_k", "new_v", "block_tables", "context_lens", "group_start",
+                                            "shared_blocks", "copy_pairs")}
+    max_group = int((w.group_start[1:] - w.group_start[:-1]).max().item())
+    steps = 4
+    g = torch.Generator(device="cpu").manual_seed(23)
+    qs = [torch.randn(w.q.shape, generator=g).to(w.q.dtype).pin_memory() for _ in range(steps)]
+    kc_h, vc_h = w.key_cache.clone(), w.value_cache.clone()
+    pipe = pk.SharedPrefixHostStepPipeline(qs[0], kc_h, host["block_tables"], host["group_start"],
+                                           host["copy_pairs"], depth=depth)
+    got = []
+    for i in range(steps):
+        pipe.step(qs[i], host["new_k"], host["new_v"], host["block_tables"], host["context_lens"],
+                  host["group_start"], host["shared_blocks"], kc_h, vc_h, w.scale, max_group_size=max_group,
+                  copy_pairs=host["copy_pairs"])
+        if i >= depth - 1:
+            j = i - depth + 1
+            pipe.done[j % depth].synchronize()
+            got.append(pipe.outs[j % depth].clone())
+    pipe.synchronize()
+    for j in range(steps - depth + 1, steps):
+        got.append(pipe.outs[j % depth].clone())
+    assert pk.device_status(clear=True) == 0
+    # the same steps on the device (the copies and the write are idempotent, only q changes)
+    kc_d, vc_d = w.key_cache.clone(), w.value_cache.clone()
+    for i in range(steps):
+        pk.kv_block_copy(w.copy_pairs, kc_d, vc_d)
+        ref = pk.paged_attention_decode_shared_prefix(qs[i].to(DEV), kc_d, vc_d, w.block_tables, w.context_lens,
+                                                      w.group_start, w.shared_blocks, w.scale, k_new=w.new_k,
+                                                      v_new=w.new_v, max_group_size=max_group)
+        torch.cuda.synchronize()
+        assert torch.equal(got[i], ref.cpu()), f"step {i}"
+    assert torch.equal(kc_h, kc_d) and torch.equal(vc_h, vc_d)
+    # one step on fresh caches against the oracle (repeated steps are not idempotent: a candidate that
+    # writes into the block the others copy changes what the next step's copies carry)
+    kc1, vc1 = w.key_cache.clone(), w.value_cache.clone()
+    out1, done1 = pipe.step(qs[0], host["new_k"], host["new_v"], host["block_tables"], host["context_lens"],
+                            host["group_start"], host["shared_blocks"], kc1, vc1, w.scale,
+                            max_group_size=max_group, copy_pairs=host["copy_pairs"])
+    done1.synchronize()
+    w.q = qs[0].to(DEV)
+    rk, rv, oref = oracle_step(w)
+    assert_cache_equal(kc1, rk, "host-step key_cache")
+    assert_cache_equal(vc1, rv, "host-step value_cache")
+    assert_close(f64(out1), oref, *tol_for(w), what="shared-prefix host step")
