@@ -918,17 +918,26 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
           }
         }
         if (!F8 && (ragged || bad)) zero_v_rows(j, bad);
-        // this half of row r of P into TMEM lane r
+        // this half of row r of P into TMEM lane r: the stacked tile's one part in a 32-column store
+        // (measured +0.9%); elsewhere 16 columns at a time (32-column stores measured -1.9% on prefill,
+        // and spill with fp8 caches)
+        if constexpr (STACK) {
+          if (lo_part)
+            tmem_st32(tmem_p(h, g + j) + lane_off, plo);
+          else
+            tmem_st32(tmem_p(h, g + j) + lane_off, ph);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pw[16], lw[16];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pw[16], lw[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            pw[k] = lo_part ? plo[16 * c + k] : ph[16 * c + k];
-            lw[k] = plo[16 * c + k];
+            for (int k = 0; k < 16; ++k) {
+              pw[k] = ph[16 * c + k];
+              lw[k] = plo[16 * c + k];
+            }
+            tmem_st16(tmem_p(h, g + j) + lane_off + 16 * c, pw);
+            if constexpr (!F8) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
           }
-          tmem_st16(tmem_p(h, g + j) + lane_off + 16 * c, pw);
-          if constexpr (!F8 && !STACK) tmem_st16(tmem_plo(h) + lane_off + 16 * c, lw);
         }
         tmem_st_wait();
         tc_fence_before();
