@@ -107,8 +107,10 @@ struct MqTcTraits {
   // P . V two tiles back has read its stage, so it has about two tiles' time
   // to land.
   // (stacked rows: two K stages -- K is read by the S MMAs alone, issued as soon as it lands -- and the
-  // third stage's space holds the P exchange buffers below)
-  static constexpr int NSK = STACK ? 2 : 3, NSV = 3;
+  // third stage's space holds the P exchange buffers below.  Unstacked bf16: two K stages and four V
+  // stages -- a V stage is freed only by the P . V a tile after the S that frees a K stage, and the
+  // V tiles of the last, ragged tile of a unit held the softmax warps back.)
+  static constexpr int NSK = (STACK || !F8) ? 2 : 3, NSV = (!STACK && !F8) ? 4 : 3;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + TILE;
   static constexpr int V_OFF = K_OFF + NSK * TILE;
