@@ -52,9 +52,9 @@
 //              scores from TMEM, applies the causal / context mask, keeps a
 //              reference max (O_h is rescaled only when a score passes it by
 //              more than 2^8), and writes its 64 probabilities into P_h.
-//   warp 8     TMA producer of Q and the K tiles (three-stage ring; one 4-D box
+//   warp 8     TMA producer of Q and the K tiles (a ring of 2-3 stages; one 4-D box
 //              per block and 64-dim half); owns the TMEM allocation.
-//   warp 10    TMA producer of the V tiles (three-stage ring).
+//   warp 10    TMA producer of the V tiles (a ring of 3-4 stages).
 //   warp 11    MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers; completion is signalled through
 //              tcgen05.commit on mbarriers.
