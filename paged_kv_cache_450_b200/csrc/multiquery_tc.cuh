@@ -19,9 +19,9 @@
 //
 // Persistent CTAs: one CTA per SM (the launch has min(units, SMs) CTAs) takes
 // one unit of every round of CTAs-many units of the unit list, which is ordered
-// longest context first (the last query tile of a sequence first): unit c of
-// even rounds, unit CTAs - 1 - c of odd rounds (a CTA that got one of the
-// longest units of a round gets one of the shortest of the next).  Barrier
+// by KV tiles, most first: unit c of even rounds, unit CTAs - 1 - c of odd
+// rounds (a CTA that got one of the longest units of a round gets one of the
+// shortest of the next).  Barrier
 // phases and ring stages run on per-CTA counters across units, so the next
 // unit's Q and first K / V tiles load while the current unit finishes, and the
 // TMEM allocation, the barrier set-up and the CTA launch are paid once per SM
@@ -133,7 +133,7 @@ struct MqTcTraits {
   static constexpr int NPB = (STACK || F8) ? 2 : 1;
   static constexpr int NBAR = 2 + 2 * NSK + 2 * NSV + 8 + (F8 ? 1 + NSK + NSV : STACK ? 1 : 0);
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;   // TMEM base address written by tcgen05.alloc
-  // the sequence of each of the CTA's first MAX_UNITS units (longest-first rank -> sequence)
+  // the rank group of each of the CTA's first MAX_UNITS units
   static constexpr int MAX_UNITS = 64;
   static constexpr int UNIT_OFF = SLOT_OFF + 16;
   // 13 warps with fp8 caches (the two widening warps), 12 otherwise: each sub-partition's registers
@@ -223,9 +223,9 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
   return __all_sync(kFullMask, mbar_wait_sleep(bar, parity, status));
 }
 
-// One work unit: (query tile qt, KV head hk) = x, partition = y, longest-first
-// rank = z of the unit list (x fastest), its sequence b.  Every thread of the
-// CTA computes the same description from the same global data.
+// One work unit: query tile qt and KV head hk of sequence b, partition part.
+// Every thread of the CTA computes the same description from the same global
+// data.
 struct MqUnit {
   int b, hk, qt, part;
   int q0, q_len, rows_total, base_pos, row_last;
@@ -236,13 +236,11 @@ struct MqUnit {
 enum { kRun = 0, kSkip = 1, kZero = 2, kBadQuery = 3 };
 
 template <int BS, int G>
-__device__ __forceinline__ MqUnit mq_unit(const MultiQueryParams& p, int64_t u, int b, int gx, int gy) {
+__device__ __forceinline__ MqUnit mq_unit(const MultiQueryParams& p, int b, int hk, int qt, int y) {
   MqUnit U;
-  const int x = static_cast<int>(u % gx), y = static_cast<int>((u / gx) % gy);
-  const int Hkv = p.num_kv_heads, n_qt = gx / Hkv;
   U.b = b;
-  U.hk = x % Hkv;
-  U.qt = n_qt - 1 - x / Hkv;  // the last query tile of a sequence sees the most tokens: it goes first
+  U.hk = hk;
+  U.qt = qt;
   U.part = y;
   U.table = nullptr;
   U.nt = U.nb = U.nparts = 0;
@@ -292,32 +290,37 @@ __device__ __forceinline__ int64_t cta_unit(int k) {
   return static_cast<int64_t>(k) * gridDim.x + c;
 }
 
-// Longest work first.  Unit rank z takes the sequence whose context is the
-// z-th longest (ties by index: a permutation of the sequences), so that the
-// units that start last are the short ones.  Each thread ranks whole
-// sequences from the context lengths staged in `scratch` (shared memory no
-// load has reached yet) and records the sequence of every unit of this CTA
-// with that rank.  Fewer than 1025 sequences and MAX_UNITS rounds; otherwise
-// units keep the sequences' order (unit_b unused).
-__device__ __forceinline__ void rank_units(const MultiQueryParams& p, int gxy, int n_rounds, int* scratch,
-                                           int* unit_b) {
-  const int B = p.num_seqs;
-  for (int i = threadIdx.x; i < B; i += blockDim.x) scratch[i] = p.context_lens[i];
+// Longest work first.  The units are ranked in groups that take the same
+// time: with at most MAX_GROUPS (sequence, partition, query tile) triples, a
+// group is one triple (its KV heads' units, keyed by the triple's KV tiles);
+// otherwise, with at most MAX_GROUPS sequences, a group is a whole sequence
+// (keyed by its context length).  Group rank r (descending key, ties by group
+// index: a permutation) takes units r * per_group .. of the unit list, so the
+// units that start last are the short ones.  Each thread ranks whole groups
+// from the keys staged in `scratch` (shared memory no load has reached yet)
+// and records the group of every unit of this CTA with that rank.
+enum { kRankNone = 0, kRankSeqs = 1, kRankGroups = 2 };
+constexpr int MAX_GROUPS = 1024;
+
+template <typename Key>
+__device__ __forceinline__ void rank_unit_groups(int n_groups, int per_group, int n_rounds, int* scratch,
+                                                 int* unit_g, Key key) {
+  for (int i = threadIdx.x; i < n_groups; i += blockDim.x) scratch[i] = key(i);
   __syncthreads();
-  for (int t = threadIdx.x; t < B; t += blockDim.x) {
+  for (int t = threadIdx.x; t < n_groups; t += blockDim.x) {
     const int lt = scratch[t];
     int r = 0;
 #pragma unroll 4
-    for (int j = 0; j < B; ++j) {
+    for (int j = 0; j < n_groups; ++j) {
       const int lj = scratch[j];
       r += (lj > lt) || (lj == lt && j < t);
     }
-    // this CTA's units u with u / gxy == r lie in rounds u_lo / CTAs .. (u_hi - 1) / CTAs
-    const int64_t u_lo = static_cast<int64_t>(r) * gxy, u_hi = u_lo + gxy;  // [u_lo, u_hi)
+    // this CTA's units u with u / per_group == r lie in rounds u_lo / CTAs .. (u_hi - 1) / CTAs
+    const int64_t u_lo = static_cast<int64_t>(r) * per_group, u_hi = u_lo + per_group;  // [u_lo, u_hi)
     const int64_t k_hi = min(static_cast<int64_t>(n_rounds) - 1, (u_hi - 1) / gridDim.x);
     for (int64_t k = u_lo / gridDim.x; k <= k_hi; ++k) {
       const int64_t u = cta_unit(static_cast<int>(k));
-      if (u >= u_lo && u < u_hi) unit_b[k] = t;
+      if (u >= u_lo && u < u_hi) unit_g[k] = t;
     }
   }
   fence_proxy_async_smem();  // the scratch writes before the tile loads that later land there
@@ -386,10 +389,26 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
   const int gx = Hkv * n_qt, gy = p.max_partitions;
   const int64_t n_all = static_cast<int64_t>(gx) * gy * p.num_seqs;
   const int n_units = static_cast<int>((n_all + gridDim.x - 1) / gridDim.x);  // rounds (the last may miss this CTA)
-  int* unit_b = reinterpret_cast<int*>(data + T::UNIT_OFF);
-  const bool ranked = p.num_seqs <= 1024 && n_units <= T::MAX_UNITS;
-  if (ranked) rank_units(p, gx * gy, n_units, reinterpret_cast<int*>(data + T::V_OFF), unit_b);
-  // unit k of this CTA (kind kSkip past the last unit)
+  // the group of each of this CTA's units (see rank_unit_groups)
+  int* unit_g = reinterpret_cast<int*>(data + T::UNIT_OFF);
+  const int64_t n_triples = static_cast<int64_t>(p.num_seqs) * gy * n_qt;
+  const int rank_mode = n_units > T::MAX_UNITS         ? kRankNone
+                        : n_triples <= MAX_GROUPS      ? kRankGroups
+                        : p.num_seqs <= MAX_GROUPS     ? kRankSeqs
+                                                       : kRankNone;
+  int* scratch = reinterpret_cast<int*>(data + T::V_OFF);
+  if (rank_mode == kRankGroups) {
+    // triple g = (b * gy + y) * n_qt + (n_qt - 1 - qt), keyed by its KV tiles (0 when it has none)
+    rank_unit_groups(static_cast<int>(n_triples), Hkv, n_units, scratch, unit_g, [&](int g) {
+      const MqUnit U = mq_unit<BS, G>(p, g / (n_qt * gy), 0, n_qt - 1 - g % n_qt, (g / n_qt) % gy);
+      return U.kind == kRun ? U.nt : 0;
+    });
+  } else if (rank_mode == kRankSeqs) {
+    rank_unit_groups(p.num_seqs, gx * gy, n_units, scratch, unit_g, [&](int b) { return p.context_lens[b]; });
+  }
+  // unit k of this CTA (kind kSkip past the last unit).  In sequence order, unit u is x = u % gx (KV head
+  // fastest, then the query tiles from the last: it sees the most tokens), partition (u / gx) % gy,
+  // sequence u / (gx * gy).
   auto unit_at = [&](int k) {
     const int64_t u = cta_unit(k);
     if (u >= n_all) {
@@ -398,8 +417,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       U.nt = 0;
       return U;
     }
-    const int z = static_cast<int>(u / (static_cast<int64_t>(gx) * gy));
-    return mq_unit<BS, G>(p, u, ranked ? unit_b[k] : z, gx, gy);
+    if (rank_mode == kRankGroups) {
+      const int g = unit_g[k];
+      return mq_unit<BS, G>(p, g / (n_qt * gy), static_cast<int>(u % Hkv), n_qt - 1 - g % n_qt, (g / n_qt) % gy);
+    }
+    const int x = static_cast<int>(u % gx), y = static_cast<int>((u / gx) % gy);
+    const int b = rank_mode == kRankSeqs ? unit_g[k] : static_cast<int>(u / (static_cast<int64_t>(gx) * gy));
+    return mq_unit<BS, G>(p, b, x % Hkv, n_qt - 1 - x / Hkv, y);
   };
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   // 32-byte output stores need 32-byte aligned rows (rows are 256 bytes; the bases only promise 16)

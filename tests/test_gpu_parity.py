@@ -603,15 +603,17 @@ def test_multiquery_full_size_sampled(name):
     _mq_check(mw, rows=rows, what=name)
 
 
-@pytest.mark.parametrize("case", ["rounds-ranked", "over-1024-sequences", "over-64-rounds"])
+@pytest.mark.parametrize("case", ["rounds-ranked", "sequence-ranked", "over-1024-sequences", "over-64-rounds"])
 def test_multiquery_persistent_many_units(case):
     """The tcgen05 kernel's persistent CTAs over many units: about 8 units per CTA with the
-    longest-first ranking; more than 1024 sequences and more than 64 units per CTA, where units keep
-    the sequences' order; empty query sets and sequences whose rows span two 128-row units among
+    longest-first ranking of (sequence, partition, query tile) triples; more than 1024 triples, where
+    whole sequences are ranked; more than 1024 sequences and more than 64 units per CTA, where units
+    keep the sequences' order; empty query sets and sequences whose rows span two 128-row units among
     them.  Sampled rows against the oracle."""
-    rng = np.random.default_rng({"rounds-ranked": 31, "over-1024-sequences": 32, "over-64-rounds": 33}[case])
-    if case == "rounds-ranked":
-        B, hq, hkv = 300, 8, 2
+    rng = np.random.default_rng({"rounds-ranked": 31, "sequence-ranked": 34, "over-1024-sequences": 32,
+                                 "over-64-rounds": 33}[case])
+    if case in ("rounds-ranked", "sequence-ranked"):
+        B, hq, hkv = (300 if case == "rounds-ranked" else 600), 8, 2
         q_lens = [int(x) if x > 3 else 0 for x in rng.integers(0, 41, B)]      # up to 160 rows: two units
         ctxs = [int(max(q, c)) for q, c in zip(q_lens, rng.integers(50, 601, B))]
     elif case == "over-1024-sequences":
