@@ -617,8 +617,10 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         if (j == U.nt - 1) tc_commit(q_empty);  // the unit's S MMAs are its only readers of Q
         return true;
       };
-      // P . V of tile jj of unit ku (tile gjj of the CTA)
-      auto issue_pv = [&](int jj, int gjj, int ku) -> bool {
+      // P . V of tile jj of unit ku (tile gjj of the CTA); half1_past: every token of the tile's second half
+      // lies past the unit's tokens (a unit's last tile, not its first: O_1 is already written), so its
+      // P . V would add zeros and is left out
+      auto issue_pv = [&](int jj, int gjj, int ku, bool half1_past) -> bool {
         const int sv = gjj % T::NSV;
         const uint64_t vd0 = vdb + ((sv * T::TILE) >> 4);
         // the V tile (bf16: landed; fp8: widened)
@@ -627,14 +629,21 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         if (jj == 0 && ku > 0 && !mbar_wait_bounded(o_free, (ku - 1) & 1, p.status)) return false;
         if (!mbar_wait_bounded(p_full(gjj), (gjj >> 1) & 1, p.status)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // O_h += P_h(jj) . V_h(jj)
+        // O_h += P_h(jj) . V_h(jj); the branch is taken once, before the MMAs (a branch between MMAs
+        // costs the issuing thread)
+        auto pv_half = [&](int h) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 8 packed TMEM columns of P per k-step
             const uint64_t vdesc = vd0 + (((64 * h + 16 * kk) * 128) >> 4);
             tc_mma_bf16_tmem_a(tmem_o(h), tmem_p(h, gjj) + 8 * kk, vdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
             if constexpr (!F8 && !STACK) tc_mma_bf16_tmem_a(tmem_o(h), tmem_plo(h) + 8 * kk, vdesc, idesc_pv, 1u);
           }
+        };
+        if (half1_past) {
+          pv_half(0);
+        } else {
+          pv_half(0);
+          pv_half(1);
         }
         tc_commit(pv_done(gjj));
         tc_commit(v_empty(sv));
@@ -646,15 +655,17 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         const MqUnit U = unit_at(k);
         if (U.kind != kRun) continue;
         if (do_s && !(ok = mbar_wait_bounded(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
+        // tile j's second half lies past the unit's tokens (only a last tile can; never the first)
+        auto half1_past = [&](int j) { return j > 0 && U.tok_begin + j * T::TOK + 64 >= U.tok_end; };
         if (do_s && do_pv) {  // one issuer: per iteration j, S(j) then P . V(j - 1)
           for (int j = 0; ok && j <= U.nt; ++j) {
             if (j < U.nt) ok = issue_s(U, j, g + j);
-            if (ok && j > 0) ok = issue_pv(j - 1, g + j - 1, ku);
+            if (ok && j > 0) ok = issue_pv(j - 1, g + j - 1, ku, half1_past(j - 1));
           }
         } else if (do_s) {
           for (int j = 0; ok && j < U.nt; ++j) ok = issue_s(U, j, g + j);
         } else {
-          for (int j = 0; ok && j < U.nt; ++j) ok = issue_pv(j, g + j, ku);
+          for (int j = 0; ok && j < U.nt; ++j) ok = issue_pv(j, g + j, ku, half1_past(j));
         }
         g += U.nt;
         ++ku;
