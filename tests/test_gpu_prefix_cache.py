@@ -154,7 +154,7 @@ def test_prefix_cache_tables_drive_decode_and_multiquery():
     lens = [len(t) for t, _ in prompts]
     check_attention(pool, reqs, lens, seed=50)
 
-    # round 2: the requests finish, LRU eviction frees blocks, new requests reuse the freed ids
+    # second wave: the requests finish, LRU eviction frees blocks, new requests reuse the freed ids
     for (toks, extra), ids in zip(prompts, reqs):
         pool.cache.release(toks, len(toks) // BS, extra)
         if len(toks) % BS:
