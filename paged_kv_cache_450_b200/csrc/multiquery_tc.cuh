@@ -54,17 +54,20 @@
 //              more than 2^8), and writes its 64 probabilities into P_h.
 //   warp 8     TMA producer of Q and the K tiles (a ring of 2-3 stages; one 4-D box
 //              per block and 64-dim half); owns the TMEM allocation.
-//   warp 10    TMA producer of the V tiles (a ring of 3-4 stages).
+//   warp 10    TMA producer of the V tiles (a ring of 3-4 stages; warp 12 with
+//              fp8 caches).
 //   warp 11    MMA issuer: one thread issues S_j as soon as the softmax has
 //              taken S_{j-1} into registers; completion is signalled through
 //              tcgen05.commit on mbarriers.
 //   warp 9     bf16 caches: the P_j . V_j issuer (its own waits and commits, so
 //              the two issuing threads' barrier work overlaps the other's MMAs).
-//   warps 9, 12  fp8 caches: widen the K (9) and V (12) tiles; warp 11 issues
-//              both MMA streams (S_j, then P_{j-1} . V_{j-1}).
+//   fp8 caches: warps 10 and 11 widen the K and V tiles (sub-partitions 2 and
+//              3, idle in grouped verification, whose rows fill only lane
+//              quarters 0 and 1), warp 9 issues both MMA streams (S_j, then
+//              P_{j-1} . V_{j-1}) and warp 12 produces V.
 // Caches of fp8 (E4M3, F8 = true): the producer warps TMA each tile's raw codes
 // (128 bytes per token row) into the upper half of the tile's own ring stage;
-// warps 9 and 12 then widen them exactly to fp16 in place (one thread per token
+// warps 10 and 11 then widen them exactly to fp16 in place (one thread per token
 // row reads the raw row whole, then writes its two fp16 halves; V rows that
 // must not contribute are zeroed there) -- the rings have the bf16 layout and
 // depths, so widening overlaps the MMAs; the softmax warps round their Q rows to
@@ -139,8 +142,12 @@ struct MqTcTraits {
   // 13 warps with fp8 caches (the two widening warps), 12 otherwise: each sub-partition's registers
   // hold at most three warps of the bf16 kernel's ~140 registers (four would cap them at 128)
   static constexpr int THREADS = F8 ? 416 : 384;
-  static constexpr int W_K = 8, W_KWIDEN = 9, W_V = 10, W_MMA = 11, W_VWIDEN = 12;
-  // the P . V issuer: warp 9 with bf16 caches (idle otherwise), the S issuer itself with fp8 caches
+  // warp w runs on sub-partition w % 4.  fp8 caches: the two widening warps on sub-partitions 2 and 3,
+  // whose softmax warps have no rows when a (sequence, KV head) has at most 64 (grouped verification),
+  // the single MMA issuer on 1 and the V producer on 0
+  static constexpr int W_K = 8, W_KWIDEN = F8 ? 10 : 9, W_V = F8 ? 12 : 10, W_MMA = F8 ? 9 : 11,
+                       W_VWIDEN = F8 ? 11 : 12;
+  // the P . V issuer: warp 9 with bf16 caches, the S issuer itself with fp8 caches
   static constexpr int W_PV = F8 ? W_MMA : 9;
   static constexpr int N_ISSUERS = W_PV == W_MMA ? 1 : 2;
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or (stacked bf16, fp16)
@@ -590,8 +597,8 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
   } else if (warp == T::W_MMA || warp == T::W_PV) {  // ---------------- MMA issuers ----------------------
     // bf16 caches: warp 11 issues the S MMAs and warp 9 the P . V MMAs, each with its own waits and
     // commits, so one thread's barrier work overlaps the other's MMAs in the tensor pipe (the two
-    // streams touch disjoint TMEM columns; their order is set by the barriers alone).  fp8 caches
-    // (warp 9 widens K): warp 11 issues both, S(j) then P . V(j - 1).
+    // streams touch disjoint TMEM columns; their order is set by the barriers alone).  fp8 caches:
+    // warp 9 issues both, S(j) then P . V(j - 1).
     if (lane == 0) {
       constexpr uint32_t idesc_s = F8 ? idesc_f16_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
