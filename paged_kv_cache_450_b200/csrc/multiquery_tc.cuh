@@ -63,8 +63,8 @@
 //              the two issuing threads' barrier work overlaps the other's MMAs).
 //   fp8 caches: warps 10 and 11 widen the K and V tiles (sub-partitions 2 and
 //              3, idle in grouped verification, whose rows fill only lane
-//              quarters 0 and 1), warp 9 issues both MMA streams (S_j, then
-//              P_{j-1} . V_{j-1}) and warp 12 produces V.
+//              quarters 0 and 1), warp 9 issues the S MMAs, warp 13 the
+//              P . V MMAs, and warp 12 produces V.
 // Caches of fp8 (E4M3, F8 = true): the producer warps TMA each tile's raw codes
 // (128 bytes per token row) into the upper half of the tile's own ring stage;
 // warps 10 and 11 then widen them exactly to fp16 in place (one thread per token
@@ -139,17 +139,18 @@ struct MqTcTraits {
   // the rank group of each of the CTA's first MAX_UNITS units
   static constexpr int MAX_UNITS = 64;
   static constexpr int UNIT_OFF = SLOT_OFF + 16;
-  // 13 warps with fp8 caches (the two widening warps), 12 otherwise: each sub-partition's registers
-  // hold at most three warps of the bf16 kernel's ~140 registers (four would cap them at 128)
-  static constexpr int THREADS = F8 ? 416 : 384;
+  // 14 warps with fp8 caches (the two widening warps and a second issuer), 12 otherwise: each
+  // sub-partition's registers hold at most three warps of the bf16 kernel's ~155 registers (four would
+  // cap them at 128); the fp8 instances take ~125
+  static constexpr int THREADS = F8 ? 448 : 384;
   // warp w runs on sub-partition w % 4.  fp8 caches: the two widening warps on sub-partitions 2 and 3,
   // whose softmax warps have no rows when a (sequence, KV head) has at most 64 (grouped verification),
-  // the single MMA issuer on 1 and the V producer on 0
+  // the two MMA issuers (S: warp 9, P . V: warp 13) on 1 and the V producer on 0
   static constexpr int W_K = 8, W_KWIDEN = F8 ? 10 : 9, W_V = F8 ? 12 : 10, W_MMA = F8 ? 9 : 11,
                        W_VWIDEN = F8 ? 11 : 12;
-  // the P . V issuer: warp 9 with bf16 caches, the S issuer itself with fp8 caches
-  static constexpr int W_PV = F8 ? W_MMA : 9;
-  static constexpr int N_ISSUERS = W_PV == W_MMA ? 1 : 2;
+  // the P . V issuer (its own waits and commits beside the S issuer's)
+  static constexpr int W_PV = F8 ? 13 : 9;
+  static constexpr int N_ISSUERS = 2;
   // S 128 | O_0 128 | O_1 128 | P: bf16 hi 0,1 (32 + 32) and lo 0,1 (32 + 32), or (stacked bf16, fp16)
   // buffer 0: halves 0,1 (32 + 32), buffer 1: halves 0,1 (32 + 32)
   static constexpr uint32_t TMEM_COLS = 512;
@@ -598,13 +599,13 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
     // bf16 caches: warp 11 issues the S MMAs and warp 9 the P . V MMAs, each with its own waits and
     // commits, so one thread's barrier work overlaps the other's MMAs in the tensor pipe (the two
     // streams touch disjoint TMEM columns; their order is set by the barriers alone).  fp8 caches:
-    // warp 9 issues both, S(j) then P . V(j - 1).
+    // warp 9 the S MMAs and warp 13 the P . V MMAs.
     if (lane == 0) {
       constexpr uint32_t idesc_s = F8 ? idesc_f16_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 128, 1) : idesc_bf16_f32(128, 128, 1);
       const uint64_t qd0 = smem_desc_sw128(base + T::Q_OFF, 16, 1024);         // K-major Q (and K, offset)
       const uint64_t vdb = smem_desc_sw128(base + T::V_OFF, T::HALF, 1024);     // N-major V
-      const bool do_s = warp == T::W_MMA, do_pv = warp == T::W_PV;
+      const bool do_s = warp == T::W_MMA;  // else the P . V issuer
       // S of tile j of the unit (tile gj of the CTA)
       auto issue_s = [&](const MqUnit& U, int j, int gj) -> bool {
         const int sk = gj % T::NSK;
@@ -664,12 +665,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         if (do_s && !(ok = mbar_wait_bounded(F8 || STACK ? q_ready : q_full, ku & 1, p.status))) break;
         // tile j's second half lies past the unit's tokens (only a last tile can; never the first)
         auto half1_past = [&](int j) { return j > 0 && U.tok_begin + j * T::TOK + 64 >= U.tok_end; };
-        if (do_s && do_pv) {  // one issuer: per iteration j, S(j) then P . V(j - 1)
-          for (int j = 0; ok && j <= U.nt; ++j) {
-            if (j < U.nt) ok = issue_s(U, j, g + j);
-            if (ok && j > 0) ok = issue_pv(j - 1, g + j - 1, ku, half1_past(j - 1));
-          }
-        } else if (do_s) {
+        if (do_s) {
           for (int j = 0; ok && j < U.nt; ++j) ok = issue_s(U, j, g + j);
         } else {
           for (int j = 0; ok && j < U.nt; ++j) ok = issue_pv(j, g + j, ku, half1_past(j));
