@@ -694,8 +694,16 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       if (ok) ok = warp_wait_bounded(bar, parity, p.status);
       return ok;
     };
+    // fp8 caches with at most 64 rows per (sequence, KV head) (grouped verification): lane quarters 2
+    // and 3 have no rows in any unit, so their warps take no part, and the warp of lane quarter 0 of
+    // each token half arrives for them on q_ready, s_free, p_full and o_free (8 arrivals each) -- those
+    // barriers never wait for warps that would only wake to arrive.  (It holds for every unit of the
+    // launch, so no warp runs ahead of the barrier phases.  bf16 caches: such warps zero their share of
+    // V rows, and with at most 64 rows the stacked tile fills every quarter.)
+    const bool skip_q23 = F8 && p.max_q_len * G <= 64;
+    const uint32_t arrive_n = skip_q23 && quarter == 0 ? 3u : 1u;
     int g = 0, ku = 0;  // tiles consumed; units
-    for (int k = 0; k < n_units; ++k) {
+    for (int k = 0; k < (skip_q23 && quarter >= 2 ? 0 : n_units); ++k) {
       const MqUnit U = unit_at(k);
       if (U.kind == kBadQuery) {
         if (threadIdx.x == 0) set_status(p.status, PKV_STATUS_BAD_QUERY_LOC);
@@ -731,7 +739,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(q_ready);
+        if (lane == 0) mbar_arrive_cnt(q_ready, arrive_n);
       }
       if constexpr (STACK) {  // Q rows 0-63 (this warp's 64-dim half) copied below themselves, same phase
         if (lo_part) {
@@ -821,7 +829,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) mbar_arrive_cnt(s_free, arrive_n);
 
         // blocks of this half tile with a bad id (their tokens are masked, their V rows zeroed)
         const unsigned bad_blocks = half_tile_bad(t0);
@@ -982,7 +990,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(g + j));
+        if (lane == 0) mbar_arrive_cnt(p_full(g + j), arrive_n);
       }
       g += nt;
       wait(pv_done(g - 1), ((g - 1) >> 1) & 1);  // (and so every earlier P . V)
@@ -1110,7 +1118,7 @@ __global__ void __launch_bounds__(MqTcTraits<BS, F8, STACK>::THREADS, 1)
       // and every softmax warp has read O before the next unit's first P . V overwrites it
       tc_fence_before();
       asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0) mbar_arrive_cnt(o_free, arrive_n);
       ++ku;
     }
   }
