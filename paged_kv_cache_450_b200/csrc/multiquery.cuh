@@ -116,7 +116,31 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC, 0, F8>::THREADS, MqTraits<BS
   int* ids = reinterpret_cast<int*>(data + T::STAGE_AREA + T::RAW_AREA + T::BAR_BYTES);
 
   const int Hkv = p.num_kv_heads;
-  const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y, b = blockIdx.z;
+  const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y;
+  // Longest work first: CTAs start in grid order, so grid row z takes the sequence with the z-th
+  // longest context (ties by index: a permutation) and the CTAs that start last are the short ones.
+  // The lengths are staged in the stage area, which no load has reached yet.  (With more than 128
+  // sequences the grid has more waves to even out and the ranking would cost more: sequence order.)
+  int b = blockIdx.z;
+  if (p.num_seqs <= 128) {
+    int* lens = reinterpret_cast<int*>(data);
+    int* pick = lens + 128;
+    for (int i = threadIdx.x; i < p.num_seqs; i += blockDim.x) lens[i] = p.context_lens[i];
+    __syncthreads();
+    for (int j = threadIdx.x; j < p.num_seqs; j += blockDim.x) {
+      const int lj = lens[j];
+      int r = 0;
+      for (int i = 0; i < p.num_seqs; ++i) {
+        const int li = lens[i];
+        r += (li > lj) || (li == lj && i < j);
+      }
+      if (r == static_cast<int>(blockIdx.z)) *pick = j;
+    }
+    __syncthreads();
+    b = *pick;
+    fence_proxy_async_smem();  // these writes before the tile loads that later land there
+    __syncthreads();
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int q0, q_len;
   if (!query_rows_ok(p, b, q0, q_len)) {  // before any load or store
