@@ -119,12 +119,15 @@ __global__ void __launch_bounds__(MqTraits<BS, NWC, 0, F8>::THREADS, MqTraits<BS
   const int hk = blockIdx.x % Hkv, qt = blockIdx.x / Hkv, part = blockIdx.y;
   // Longest work first: CTAs start in grid order, so grid row z takes the sequence with the z-th
   // longest context (ties by index: a permutation) and the CTAs that start last are the short ones.
-  // The lengths are staged in the stage area, which no load has reached yet.  (With more than 128
-  // sequences the grid has more waves to even out and the ranking would cost more: sequence order.)
+  // The lengths are staged in the stage area, which no load has reached yet.  Each CTA's ranking
+  // takes ~B^2 comparisons, so it runs only where it is cheap beside the CTA's work and the tail
+  // matters: at most 64 sequences (more CTAs, more waves to even out) and a block table of at least
+  // 1024 tokens.  (In the decode kernel, with 256 sequences and ~10000 short CTAs, the same ranking
+  // measured 18% slower.)
   int b = blockIdx.z;
-  if (p.num_seqs <= 128) {
+  if (p.num_seqs <= 64 && p.max_blocks_per_seq * BS >= 1024) {
     int* lens = reinterpret_cast<int*>(data);
-    int* pick = lens + 128;
+    int* pick = lens + 64;
     for (int i = threadIdx.x; i < p.num_seqs; i += blockDim.x) lens[i] = p.context_lens[i];
     __syncthreads();
     for (int j = threadIdx.x; j < p.num_seqs; j += blockDim.x) {
