@@ -12,7 +12,7 @@ of a full block a function of its chained hash (a block with the same prefix
 holds the same K/V, as it would in a model).  Decode and multi-query attention
 over those tables are checked against the CPU oracle on the same tables, and
 against the same requests laid out in private copies (bit-identical: the
-kernels' arithmetic does not depend on where a block sits).  A second round
+kernels' arithmetic does not depend on where a block sits).  A second wave
 releases, evicts and reuses physical blocks.
 """
 import numpy as np
